@@ -1,0 +1,185 @@
+/*
+ * deco_moe.h -- C ABI of the B200 (sm_100a) DECO sparse MoE FFN layer.
+ *
+ * The layer is the DECO mixture-of-experts FFN as described in
+ *   [arXiv] "DECO: Sparse Mixture-of-Experts with Dense-Comparable Performance
+ *           on End-Side Devices" (arXiv 2605.10933), §1 Introduction and §2
+ *           "Router design" / "Expert design";
+ *   [press] the qidianchuan.cn summary of the same paper, part 2 (core design:
+ *           router paragraph, NormSiLU paragraphs, non-gated experts).
+ *
+ *   z   = x W_r^T + b_r                    router logits, one per routed expert
+ *   e is active for a token iff z_e > 0    (a zero or negative score is ignored)
+ *   r   = ReLU(z)                          raw routing weight, not renormalised
+ *   u   = x W_bar_up^T                     mean up-projection (precomputed mean)
+ *   a_e = SiLU(RMSNorm(x W_up[e]^T - u))   NormSiLU, RMS over the d_e features,
+ *                                          eps inside the square root, no gain
+ *   y   = W_s_down SiLU(W_s_up x)          always-on shared expert
+ *       + sum_{e active, ascending} s_e r_e W_down[e] a_e
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer argument named as a tensor is a DEVICE pointer to memory the
+ *    caller owns; the library never allocates, frees or keeps a pointer after
+ *    the call returns.  Matrices are row-major with the nn.Linear convention
+ *    [out_features][in_features], so every row is contiguous along the
+ *    contracted axis.  Device pointers must be 16-byte aligned.
+ *  - x, out and all weight matrices use the layer's storage dtype (fp32 or
+ *    bf16); b_r and s are always fp32.  Arithmetic is fp32 with fp32
+ *    accumulation; router activation decisions are exact (see below).
+ *  - All calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL is the legacy default stream) and never synchronise, except
+ *    deco_moe_device_error.  They do not allocate, so a sequence of calls can
+ *    be captured in a CUDA graph.
+ *  - Arguments are checked on the host before anything is launched; on any
+ *    error nothing is launched and a non-zero status is returned.  A status of
+ *    DECO_ERR_CUDA means a launch failed (cudaGetLastError was not success).
+ *  - `x` must not alias `out`.
+ *
+ * Exact routing: the activation decision z_e > 0 is made on the exact real
+ * value of b_r[e] + sum_k x_k W_r[e,k] over the stored operands.  The kernels
+ * compute z in fp32 with a rigorous error bound and re-evaluate the sign
+ * exactly (integer accumulation of the exact products) whenever the fp32 value
+ * lies inside the bound, so active sets, counts and permutations are
+ * reproducible bit for bit on any GPU and match an exact CPU evaluation.
+ */
+#ifndef DECO_MOE_H_
+#define DECO_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DECO_OK = 0,
+  DECO_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer   */
+  DECO_ERR_UNSUPPORTED = 2,   /* valid but unsupported shape or dtype         */
+  DECO_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required   */
+  DECO_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
+  DECO_ERR_DEVICE = 5         /* a kernel reported an error (see device_error) */
+} deco_status_t;
+
+typedef enum { DECO_F32 = 0, DECO_BF16 = 1 } deco_dtype_t;
+
+/* Shape of one layer call.
+ *   T        tokens in the batch (>= 0; T == 0 is a no-op)
+ *   d_model  model width D: multiple of 64, 64..16384
+ *   E        routed experts: 1..256
+ *   d_e      routed expert width: multiple of 64, 64..512
+ *   d_s      shared expert width: multiple of 64, 64..16384
+ *   dtype    storage dtype of x, out and every weight matrix
+ *   rms_eps  epsilon added to the mean square inside NormSiLU's square root
+ *   residual 0: out = layer(x); 1: out = x + layer(x), rounded once        */
+typedef struct {
+  int T;
+  int d_model;
+  int E;
+  int d_e;
+  int d_s;
+  int dtype;      /* deco_dtype_t */
+  float rms_eps;
+  int residual;
+} deco_moe_shape_t;
+
+/* The layer's weights (device pointers, storage dtype unless noted).
+ *   W_r      [E][D]        router projection
+ *   b_r      [E]     fp32  router bias
+ *   W_up     [E][d_e][D]   routed up-projections
+ *   W_bar_up [d_e][D]      mean of W_up over the E experts (deco_moe_mean_up)
+ *   W_down   [E][D][d_e]   routed down-projections
+ *   s        [E]     fp32  learnable expert-wise router scaling
+ *   W_s_up   [d_s][D]      shared expert up-projection
+ *   W_s_down [D][d_s]      shared expert down-projection                    */
+typedef struct {
+  const void* W_r;
+  const float* b_r;
+  const void* W_up;
+  const void* W_bar_up;
+  const void* W_down;
+  const float* s;
+  const void* W_s_up;
+  const void* W_s_down;
+} deco_moe_weights_t;
+
+/* Routing outputs of deco_moe_routing (device pointers; any may be NULL to
+ * skip that output except where noted).
+ *   r        [T][E] fp32   ReLU(z): the logit where active, 0 elsewhere
+ *   active   [T][E] u8     1 where z > 0 (exact), else 0
+ *   counts   [E]    i32    tokens routed to each expert
+ *   offsets  [E+1]  i32    exclusive prefix sum of counts; offsets[E] = P
+ *   perm     [T*E]  i32    token of each (token, expert) pair, pairs ordered by
+ *                          expert then token, ascending; the first P entries
+ *                          are valid (capacity must be T*E)
+ *   n_tok    [T]    i32    number of active experts of each token          */
+typedef struct {
+  float* r;
+  uint8_t* active;
+  int* counts;
+  int* offsets;
+  int* perm;
+  int* n_tok;
+} deco_routing_t;
+
+/* Bytes of device workspace deco_moe_forward / deco_moe_routing need for
+ * `shape`.  Returns DECO_ERR_INVALID_ARG / DECO_ERR_UNSUPPORTED for a shape the
+ * forward call would reject. */
+deco_status_t deco_moe_workspace_size(const deco_moe_shape_t* shape, size_t* bytes);
+
+/* Forward pass of one DECO MoE FFN layer ([arXiv] §1; [press] part 2):
+ * out[T][D] = layer(x[T][D]) (plus x when shape->residual).
+ * `workspace` is device scratch of at least deco_moe_workspace_size bytes,
+ * 256-byte aligned, owned by the caller; its contents need no initialisation
+ * and are overwritten.  Two calls that overlap on the GPU must not share one
+ * workspace. */
+deco_status_t deco_moe_forward(const deco_moe_shape_t* shape, const void* x,
+                               const deco_moe_weights_t* w, void* out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* The router and the token->expert tables alone ([press] part 2 router
+ * paragraph: a token activates every expert whose ReLU score is positive, so
+ * the count per token varies).  Only w->W_r and w->b_r are read.  counts,
+ * offsets and perm follow a stable counting sort by expert. */
+deco_status_t deco_moe_routing(const deco_moe_shape_t* shape, const void* x,
+                               const deco_moe_weights_t* w, const deco_routing_t* out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* The precomputed mean up-projection of NormSiLU ([press] part 2: the mean of
+ * all experts' up-projection weights is fixed at inference and computed once):
+ * W_bar_up[j][k] = (1/E) sum_{e ascending} W_up[e][j][k], summed and divided in
+ * fp64, rounded once (to nearest, ties to even) to `dtype`. */
+deco_status_t deco_moe_mean_up(int E, int d_e, int d_model, int dtype, const void* W_up,
+                               void* W_bar_up, void* stream);
+
+/* Equal-parameter dense non-gated FFN, the "Dense" comparison of [arXiv] §5:
+ * out[T][D] = W2 SiLU(W1 x), W1 [d_ff][D], W2 [D][d_ff].  d_ff multiple of 64,
+ * d_model as for the layer. */
+deco_status_t deco_dense_ffn_workspace_size(int T, int d_model, int d_ff, int dtype,
+                                            size_t* bytes);
+deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, const void* x,
+                                     const void* W1, const void* W2, void* out,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the device error word a kernel may have
+ * set in `workspace` (0 = none; 1 = a non-finite router operand) and clears
+ * it.  Returns DECO_ERR_CUDA if the synchronisation fails. */
+deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
+
+/* Kernel timing hook for benchmarks.  While set (events != NULL), every later
+ * deco_moe_forward call on this process records events[2*i] on its stream just
+ * before its i-th kernel and events[2*i+1] just after it, for i < n_events/2;
+ * the kernels are, in order: router, expert counts, expert scatter,
+ * up-projection, down-projection.  `events` are cudaEvent_t handles owned by the
+ * caller (passed as void*) and must outlive the calls.  Pass NULL to stop.
+ * Not thread-safe; meant for a single benchmarking thread. */
+deco_status_t deco_moe_set_profiling(void* const* events, int n_events);
+
+/* A static, human-readable name for a status code. */
+const char* deco_status_string(deco_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DECO_MOE_H_ */

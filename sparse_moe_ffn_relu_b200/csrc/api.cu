@@ -1,0 +1,408 @@
+// Host side of the C ABI declared in include/deco_moe.h: argument checks,
+// workspace plan and the launch sequence.  No allocation, no synchronisation
+// (except deco_moe_device_error), so every call can be graph-captured.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/deco_moe.h"
+#include "simt_kernels.cuh"
+
+namespace deco {
+namespace {
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Workspace layout of one forward / routing call.
+struct Plan {
+  size_t err, r, act, u, hs, counts, offsets, n_tok, perm, pair_of, tiles, n_tiles, H, total;
+  int tile_rows;
+};
+
+inline size_t elem_size(int dtype) { return dtype == DECO_F32 ? 4 : 2; }
+
+// rows of x staged per CTA: 16 when the tile fits in 128 KB of shared memory
+inline int token_tile(int D, int dtype) { return (16 * (size_t)D * elem_size(dtype) <= 131072) ? 16 : 8; }
+
+Plan make_plan(const deco_moe_shape_t& s) {
+  Plan p{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t T = s.T, E = s.E, P = T * E;
+  p.tile_rows = token_tile(s.d_model, s.dtype);
+  p.err = take(16);
+  p.r = take(T * E * 4);
+  p.act = take(T * E);
+  p.u = take(T * s.d_e * 4);
+  p.hs = take(T * s.d_s * 4);
+  p.counts = take(E * 4);
+  p.offsets = take((E + 1) * 4);
+  p.n_tok = take(T * 4);
+  p.perm = take(P * 4);
+  p.pair_of = take(P * 4);
+  p.tiles = take((P / p.tile_rows + E) * 16);
+  p.n_tiles = take(4);
+  p.H = take(P * s.d_e * 4);
+  p.total = off;
+  return p;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+deco_status_t check_shape(const deco_moe_shape_t* s) {
+  if (!s) return DECO_ERR_INVALID_ARG;
+  if (s->T < 0 || s->d_model <= 0 || s->E <= 0 || s->d_e <= 0 || s->d_s <= 0)
+    return DECO_ERR_INVALID_ARG;
+  if (s->dtype != DECO_F32 && s->dtype != DECO_BF16) return DECO_ERR_INVALID_ARG;
+  if (!(s->rms_eps >= 0.f) || !std::isfinite(s->rms_eps)) return DECO_ERR_INVALID_ARG;
+  if (s->residual != 0 && s->residual != 1) return DECO_ERR_INVALID_ARG;
+  if (s->d_model % 64 || s->d_model > 16384) return DECO_ERR_UNSUPPORTED;
+  if (s->E > 256) return DECO_ERR_UNSUPPORTED;
+  if (s->d_e % 64 || s->d_e > 512) return DECO_ERR_UNSUPPORTED;
+  if (s->d_s % 64 || s->d_s > 16384) return DECO_ERR_UNSUPPORTED;
+  if (s->T > (1 << 20)) return DECO_ERR_UNSUPPORTED;
+  return DECO_OK;
+}
+
+deco_status_t check_weights(const deco_moe_weights_t* w, bool router_only) {
+  if (!w || !w->W_r || !w->b_r) return DECO_ERR_INVALID_ARG;
+  if (!aligned16(w->W_r)) return DECO_ERR_INVALID_ARG;
+  if (router_only) return DECO_OK;
+  const void* ps[] = {w->W_up, w->W_bar_up, w->W_down, w->s, w->W_s_up, w->W_s_down};
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return DECO_ERR_INVALID_ARG;
+  return DECO_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// Opt every kernel into the dynamic shared memory it may use (once per device).
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// benchmark timing hook (deco_moe_set_profiling)
+cudaEvent_t const* g_prof_events = nullptr;
+int g_prof_n = 0;
+
+inline void prof_mark(int idx, cudaStream_t st) {
+  if (g_prof_events && idx < g_prof_n) cudaEventRecord(g_prof_events[idx], st);
+}
+
+// ---------------------------------------------------------------------------
+template <typename T, int TT>
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  const size_t smem = (size_t)TT * a.D * sizeof(T) + kWarps * kLimbs * sizeof(unsigned long long);
+  cudaError_t err = allow_smem(k_route<T, TT>, smem);
+  if (err != cudaSuccess) return err;
+  const int R = a.E + a.d_e + a.d_s;
+  dim3 grid((R + kWarps - 1) / kWarps, (a.T + TT - 1) / TT);
+  k_route<T, TT><<<grid, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t route_any(const RouteArgs& a, int tt, cudaStream_t st) {
+  return tt == 16 ? launch_route<T, 16>(a, st) : launch_route<T, 8>(a, st);
+}
+
+template <typename T, int TT>
+cudaError_t launch_up(const UpArgs& a, int max_tiles, cudaStream_t st) {
+  const size_t smem = (size_t)TT * a.D * sizeof(T) + (size_t)TT * (a.d_e / kCluster) * sizeof(float);
+  cudaError_t err = allow_smem(k_up<T, TT>, smem);
+  if (err != cudaSuccess) return err;
+  int clusters = std::min(max_tiles, std::max(1, 2 * num_sms() / kCluster));
+  k_up<T, TT><<<clusters * kCluster, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_down(const DownArgs& a, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  constexpr int TT = 16, RPW = 2;
+  const size_t smem = sizeof(float) * TT * kDownK + sizeof(uint32_t) * (size_t)std::max(a.E, 1);
+  cudaError_t err = allow_smem(k_down<T, TT, RPW>, smem);
+  if (err != cudaSuccess) return err;
+  dim3 grid(a.D / (kWarps * RPW), (a.T + TT - 1) / TT);
+  k_down<T, TT, RPW><<<grid, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+// router + tables (shared by forward and routing)
+template <typename T>
+cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
+                        unsigned char* ws, const Plan& p, bool with_mean_shared, float* r,
+                        uint8_t* act, int* counts, int* offsets, int* perm, int* n_tok,
+                        cudaStream_t st) {
+  RouteArgs ra{};
+  ra.x = x;
+  ra.T = s.T;
+  ra.D = s.d_model;
+  ra.W_r = w.W_r;
+  ra.b_r = w.b_r;
+  ra.E = s.E;
+  ra.W_bar = w.W_bar_up;
+  ra.d_e = with_mean_shared ? s.d_e : 0;
+  ra.W_s_up = w.W_s_up;
+  ra.d_s = with_mean_shared ? s.d_s : 0;
+  ra.r = r;
+  ra.act = act;
+  ra.u = reinterpret_cast<float*>(ws + p.u);
+  ra.hs = reinterpret_cast<float*>(ws + p.hs);
+  ra.err = reinterpret_cast<int*>(ws + p.err);
+  prof_mark(0, st);
+  cudaError_t err = route_any<T>(ra, token_tile(s.d_model, s.dtype), st);
+  if (err != cudaSuccess) return err;
+  prof_mark(1, st);
+  prof_mark(2, st);
+  k_count<<<s.E + (s.T + kThreads - 1) / kThreads, kThreads, 0, st>>>(act, s.T, s.E, counts, n_tok);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  prof_mark(3, st);
+  prof_mark(4, st);
+  k_scatter<<<s.E, kThreads, 0, st>>>(act, s.T, s.E, counts, offsets, perm,
+                                       reinterpret_cast<int*>(ws + p.pair_of),
+                                       reinterpret_cast<int4*>(ws + p.tiles),
+                                       reinterpret_cast<int*>(ws + p.n_tiles), p.tile_rows);
+  prof_mark(5, st);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t run_forward(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
+                        void* out, unsigned char* ws, const Plan& p, cudaStream_t st) {
+  float* r = reinterpret_cast<float*>(ws + p.r);
+  uint8_t* act = reinterpret_cast<uint8_t*>(ws + p.act);
+  int* counts = reinterpret_cast<int*>(ws + p.counts);
+  cudaError_t err = run_routing<T>(s, x, w, ws, p, true, r, act, counts,
+                                   reinterpret_cast<int*>(ws + p.offsets),
+                                   reinterpret_cast<int*>(ws + p.perm),
+                                   reinterpret_cast<int*>(ws + p.n_tok), st);
+  if (err != cudaSuccess) return err;
+  UpArgs ua{};
+  ua.x = x;
+  ua.D = s.d_model;
+  ua.W_up = w.W_up;
+  ua.d_e = s.d_e;
+  ua.u = reinterpret_cast<const float*>(ws + p.u);
+  ua.perm = reinterpret_cast<const int*>(ws + p.perm);
+  ua.tiles = reinterpret_cast<const int4*>(ws + p.tiles);
+  ua.n_tiles = reinterpret_cast<const int*>(ws + p.n_tiles);
+  ua.H = reinterpret_cast<float*>(ws + p.H);
+  ua.eps = s.rms_eps;
+  const int max_tiles = (int)((size_t)s.T * s.E / p.tile_rows + s.E);
+  prof_mark(6, st);
+  err = p.tile_rows == 16 ? launch_up<T, 16>(ua, max_tiles, st) : launch_up<T, 8>(ua, max_tiles, st);
+  if (err != cudaSuccess) return err;
+  prof_mark(7, st);
+  DownArgs da{};
+  da.T = s.T;
+  da.D = s.d_model;
+  da.E = s.E;
+  da.d_e = s.d_e;
+  da.d_s = s.d_s;
+  da.act = act;
+  da.r = r;
+  da.s = w.s;
+  da.pair_of = reinterpret_cast<const int*>(ws + p.pair_of);
+  da.H = reinterpret_cast<const float*>(ws + p.H);
+  da.W_down = w.W_down;
+  da.W_s_down = w.W_s_down;
+  da.hs = reinterpret_cast<const float*>(ws + p.hs);
+  da.x = x;
+  da.out = out;
+  da.residual = s.residual;
+  prof_mark(8, st);
+  err = launch_down<T>(da, st);
+  prof_mark(9, st);
+  return err;
+}
+
+std::mutex g_smem_mutex;   // serialises first-use attribute setting
+
+}  // namespace
+}  // namespace deco
+
+using namespace deco;
+
+extern "C" {
+
+const char* deco_status_string(deco_status_t s) {
+  switch (s) {
+    case DECO_OK: return "ok";
+    case DECO_ERR_INVALID_ARG: return "invalid argument";
+    case DECO_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case DECO_ERR_WORKSPACE: return "workspace missing or too small";
+    case DECO_ERR_CUDA: return "CUDA error";
+    case DECO_ERR_DEVICE: return "device-side error";
+  }
+  return "unknown status";
+}
+
+deco_status_t deco_moe_workspace_size(const deco_moe_shape_t* shape, size_t* bytes) {
+  if (!bytes) return DECO_ERR_INVALID_ARG;
+  const deco_status_t st = check_shape(shape);
+  if (st != DECO_OK) return st;
+  *bytes = make_plan(*shape).total;
+  return DECO_OK;
+}
+
+deco_status_t deco_moe_forward(const deco_moe_shape_t* shape, const void* x,
+                               const deco_moe_weights_t* w, void* out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  deco_status_t st = check_shape(shape);
+  if (st != DECO_OK) return st;
+  if ((st = check_weights(w, false)) != DECO_OK) return st;
+  if (shape->T == 0) return DECO_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out) || x == out) return DECO_ERR_INVALID_ARG;
+  const Plan p = make_plan(*shape);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DECO_ERR_WORKSPACE;
+  if (workspace_bytes < p.total) return DECO_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t cs = as_stream(stream);
+  std::lock_guard<std::mutex> lock(g_smem_mutex);
+  if (cudaMemsetAsync(ws + p.err, 0, 16, cs) != cudaSuccess) return DECO_ERR_CUDA;
+  const cudaError_t err = shape->dtype == DECO_F32 ? run_forward<float>(*shape, x, *w, out, ws, p, cs)
+                                                   : run_forward<bf16>(*shape, x, *w, out, ws, p, cs);
+  return err == cudaSuccess ? DECO_OK : DECO_ERR_CUDA;
+}
+
+deco_status_t deco_moe_routing(const deco_moe_shape_t* shape, const void* x,
+                               const deco_moe_weights_t* w, const deco_routing_t* out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  deco_status_t st = check_shape(shape);
+  if (st != DECO_OK) return st;
+  if ((st = check_weights(w, true)) != DECO_OK) return st;
+  if (!out) return DECO_ERR_INVALID_ARG;
+  if (shape->T == 0) return DECO_OK;
+  if (!x || !aligned16(x)) return DECO_ERR_INVALID_ARG;
+  const Plan p = make_plan(*shape);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DECO_ERR_WORKSPACE;
+  if (workspace_bytes < p.total) return DECO_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t cs = as_stream(stream);
+  float* r = out->r ? out->r : reinterpret_cast<float*>(ws + p.r);
+  uint8_t* act = out->active ? out->active : reinterpret_cast<uint8_t*>(ws + p.act);
+  int* counts = out->counts ? out->counts : reinterpret_cast<int*>(ws + p.counts);
+  int* offsets = out->offsets ? out->offsets : reinterpret_cast<int*>(ws + p.offsets);
+  int* perm = out->perm ? out->perm : reinterpret_cast<int*>(ws + p.perm);
+  int* n_tok = out->n_tok ? out->n_tok : reinterpret_cast<int*>(ws + p.n_tok);
+  std::lock_guard<std::mutex> lock(g_smem_mutex);
+  if (cudaMemsetAsync(ws + p.err, 0, 16, cs) != cudaSuccess) return DECO_ERR_CUDA;
+  const cudaError_t err =
+      shape->dtype == DECO_F32
+          ? run_routing<float>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs)
+          : run_routing<bf16>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs);
+  return err == cudaSuccess ? DECO_OK : DECO_ERR_CUDA;
+}
+
+deco_status_t deco_moe_mean_up(int E, int d_e, int d_model, int dtype, const void* W_up,
+                               void* W_bar_up, void* stream) {
+  if (E <= 0 || d_e <= 0 || d_model <= 0 || !W_up || !W_bar_up) return DECO_ERR_INVALID_ARG;
+  if (dtype != DECO_F32 && dtype != DECO_BF16) return DECO_ERR_INVALID_ARG;
+  if (W_up == W_bar_up) return DECO_ERR_INVALID_ARG;
+  const size_t n = (size_t)d_e * d_model;
+  const int blocks = (int)std::min<size_t>((n + 255) / 256, 4096);
+  cudaStream_t cs = as_stream(stream);
+  if (dtype == DECO_F32)
+    k_mean_up<float><<<blocks, 256, 0, cs>>>(static_cast<const float*>(W_up),
+                                              static_cast<float*>(W_bar_up), E, n);
+  else
+    k_mean_up<bf16><<<blocks, 256, 0, cs>>>(static_cast<const bf16*>(W_up),
+                                             static_cast<bf16*>(W_bar_up), E, n);
+  return cudaGetLastError() == cudaSuccess ? DECO_OK : DECO_ERR_CUDA;
+}
+
+// dense FFN: workspace = [err | hs [T][d_ff] fp32]
+deco_status_t deco_dense_ffn_workspace_size(int T, int d_model, int d_ff, int dtype, size_t* bytes) {
+  if (!bytes || T < 0 || d_model <= 0 || d_ff <= 0) return DECO_ERR_INVALID_ARG;
+  if (dtype != DECO_F32 && dtype != DECO_BF16) return DECO_ERR_INVALID_ARG;
+  if (d_model % 64 || d_model > 16384 || d_ff % 64 || d_ff > (1 << 20) || T > (1 << 20))
+    return DECO_ERR_UNSUPPORTED;
+  *bytes = 256 + align256((size_t)T * d_ff * 4);
+  return DECO_OK;
+}
+
+deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, const void* x,
+                                     const void* W1, const void* W2, void* out, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  size_t need = 0;
+  deco_status_t st = deco_dense_ffn_workspace_size(T, d_model, d_ff, dtype, &need);
+  if (st != DECO_OK) return st;
+  if (T == 0) return DECO_OK;
+  if (!x || !W1 || !W2 || !out || x == out) return DECO_ERR_INVALID_ARG;
+  const void* ps[] = {x, W1, W2, out};
+  for (const void* q : ps)
+    if (!aligned16(q)) return DECO_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return DECO_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t cs = as_stream(stream);
+  std::lock_guard<std::mutex> lock(g_smem_mutex);
+  RouteArgs ra{};
+  ra.x = x;
+  ra.T = T;
+  ra.D = d_model;
+  ra.E = 0;
+  ra.d_e = 0;
+  ra.W_s_up = W1;
+  ra.d_s = d_ff;
+  ra.hs = reinterpret_cast<float*>(ws + 256);
+  ra.err = reinterpret_cast<int*>(ws);
+  DownArgs da{};
+  da.T = T;
+  da.D = d_model;
+  da.E = 0;
+  da.d_e = 64;
+  da.d_s = d_ff;
+  da.W_s_down = W2;
+  da.hs = ra.hs;
+  da.x = x;
+  da.out = out;
+  da.residual = 0;
+  cudaError_t err;
+  const int tt = token_tile(d_model, dtype);
+  if (dtype == DECO_F32) {
+    err = route_any<float>(ra, tt, cs);
+    if (err == cudaSuccess) err = launch_down<float>(da, cs);
+  } else {
+    err = route_any<bf16>(ra, tt, cs);
+    if (err == cudaSuccess) err = launch_down<bf16>(da, cs);
+  }
+  return err == cudaSuccess ? DECO_OK : DECO_ERR_CUDA;
+}
+
+deco_status_t deco_moe_set_profiling(void* const* events, int n_events) {
+  if (events && n_events < 0) return DECO_ERR_INVALID_ARG;
+  g_prof_events = events ? reinterpret_cast<cudaEvent_t const*>(events) : nullptr;
+  g_prof_n = events ? n_events : 0;
+  return DECO_OK;
+}
+
+deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream) {
+  if (!workspace || !code) return DECO_ERR_INVALID_ARG;
+  cudaStream_t cs = as_stream(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return DECO_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return DECO_ERR_CUDA;
+  *code = v;
+  if (cudaMemsetAsync(workspace, 0, sizeof(int), cs) != cudaSuccess) return DECO_ERR_CUDA;
+  return DECO_OK;
+}
+
+}  // extern "C"

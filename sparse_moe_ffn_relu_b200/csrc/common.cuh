@@ -1,0 +1,180 @@
+// Device helpers shared by the DECO MoE kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace deco {
+
+using bf16 = __nv_bfloat16;
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// 16-byte vector loads, widened to fp32.  VecN<T>::N elements per 16 bytes.
+
+template <typename T> struct VecN;
+template <> struct VecN<float> { static constexpr int N = 4; };
+template <> struct VecN<bf16> { static constexpr int N = 8; };
+
+__device__ __forceinline__ void unpack16(const uint4& q, float (&v)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void unpack16(const uint4& q, float (&v)[4]) {
+  v[0] = __uint_as_float(q.x);
+  v[1] = __uint_as_float(q.y);
+  v[2] = __uint_as_float(q.z);
+  v[3] = __uint_as_float(q.w);
+}
+
+// Streaming load of read-only weights: no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+template <typename T, int N>
+__device__ __forceinline__ void load_w(const T* p, float (&v)[N]) {
+  static_assert(N == VecN<T>::N, "vector width");
+  unpack16(ld_stream16(p), v);
+}
+template <typename T, int N>
+__device__ __forceinline__ void load_s(const T* p, float (&v)[N]) {
+  static_assert(N == VecN<T>::N, "vector width");
+  unpack16(*reinterpret_cast<const uint4*>(p), v);
+}
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;  // xor butterfly: every lane holds the identical total
+}
+
+// SiLU(h) = h * sigmoid(h) = h / (1 + exp(-h)); expf overflow gives -0 in the limit.
+__device__ __forceinline__ float silu_f(float h) { return h / (1.0f + expf(-h)); }
+
+// ---------------------------------------------------------------------------
+// Exact sign of b + sum_k x_k w_k over fp32-representable operands.
+//
+// Every fp32 value is m * 2^e with an integer m < 2^24 and e >= -149, so every
+// product x_k w_k is M * 2^f with M < 2^48 and f >= -298.  The sum is
+// accumulated exactly in a fixed-point integer with its least significant bit
+// at 2^-298, kept as kLimbs signed 64-bit limbs of 32 bits each (the spare
+// 32 bits of every limb absorb carries).  Products of finite fp32 values
+// reach at most 2^(208+48) and a sum of at most 2^16 of them 2^272, far below
+// the top limb.  One warp evaluates one sum; limbs live in shared memory.
+
+constexpr int kLimbs = 20;          // 640 bits with the LSB at 2^-298
+constexpr int kLsbExp = -298;
+
+struct FpParts {
+  uint32_t m;   // integer significand (0 for zero)
+  int e;        // exponent of the significand's LSB
+  bool neg;
+  bool finite;
+};
+
+__device__ __forceinline__ FpParts fp_parts(float f) {
+  const uint32_t b = __float_as_uint(f);
+  const uint32_t ef = (b >> 23) & 0xffu;
+  const uint32_t frac = b & 0x7fffffu;
+  FpParts p;
+  p.neg = (b >> 31) != 0;
+  p.finite = ef != 0xffu;
+  if (ef == 0) {
+    p.m = frac;
+    p.e = -149;
+  } else {
+    p.m = frac | 0x800000u;
+    p.e = int(ef) - 150;
+  }
+  return p;
+}
+
+__device__ __forceinline__ void limb_add(unsigned long long* limbs, int i, unsigned long long v,
+                                         bool neg) {
+  if (v) atomicAdd(&limbs[i], neg ? (0ull - v) : v);
+}
+
+// adds (-1)^neg * M * 2^(o + kLsbExp), M < 2^48, o >= 0
+__device__ __forceinline__ void limbs_add_scaled(unsigned long long* limbs, unsigned long long M,
+                                                 int o, bool neg) {
+  const int i = o >> 5, sh = o & 31;
+  const unsigned long long lo = M & 0xffffffffull, hi = M >> 32;
+  const unsigned long long a = lo << sh;   // < 2^63
+  const unsigned long long c = hi << sh;   // < 2^47
+  limb_add(limbs, i, a & 0xffffffffull, neg);
+  limb_add(limbs, i + 1, (a >> 32) + (c & 0xffffffffull), neg);
+  limb_add(limbs, i + 2, c >> 32, neg);
+}
+
+// Exact sign (-1, 0, +1) of b + sum_{k<D} x[k] w[k]; called by all 32 lanes of
+// one warp with the same arguments.  `limbs` is this warp's kLimbs-entry shared
+// buffer.  Sets *nonfinite if an operand is Inf/NaN (the result is then 0).
+template <typename Tx, typename Tw>
+__device__ int exact_sign_warp(const Tx* x, const Tw* w, int D, float b,
+                               unsigned long long* limbs, bool* nonfinite) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < kLimbs; i += 32) limbs[i] = 0ull;
+  __syncwarp();
+  bool bad = false;
+  for (int k = lane; k < D; k += 32) {
+    const FpParts px = fp_parts(to_f32(x[k]));
+    const FpParts pw = fp_parts(to_f32(w[k]));
+    bad |= !(px.finite && pw.finite);
+    if (px.m && pw.m && px.finite && pw.finite) {
+      limbs_add_scaled(limbs, (unsigned long long)px.m * pw.m, px.e + pw.e - kLsbExp,
+                       px.neg != pw.neg);
+    }
+  }
+  if (lane == 0) {
+    const FpParts pb = fp_parts(b);
+    bad |= !pb.finite;
+    if (pb.m && pb.finite) limbs_add_scaled(limbs, pb.m, pb.e - kLsbExp, pb.neg);
+  }
+  bad = __any_sync(kFull, bad);
+  __syncwarp();
+  int sign = 0;
+  if (lane == 0) {
+    long long carry = 0;
+    bool nz = false;
+    for (int i = 0; i < kLimbs; ++i) {
+      const long long v = (long long)limbs[i] + carry;
+      nz |= (v & 0xffffffffll) != 0;
+      carry = v >> 32;   // arithmetic shift: floor division by 2^32
+    }
+    sign = carry < 0 ? -1 : ((carry > 0 || nz) ? 1 : 0);
+  }
+  sign = __shfl_sync(kFull, sign, 0);
+  __syncwarp();
+  if (bad) {
+    *nonfinite = true;
+    return 0;
+  }
+  return sign;
+}
+
+// gamma_n = n u / (1 - n u) with u = 2^-24: the classical bound on the
+// relative error of an n-step fp32 recursive (FMA) summation.
+__device__ __forceinline__ float gamma_f32(int n) {
+  const double nu = double(n) * 5.9604644775390625e-8;
+  return float(nu / (1.0 - nu));
+}
+
+}  // namespace deco

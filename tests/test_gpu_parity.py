@@ -1,0 +1,182 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Routing (active sets, counts, offsets, permutation,
+per-token counts) must match bit for bit; outputs within max|err| <= 1e-4 *
+RMS (fp32) or 2e-2 * RMS (bf16) of the oracle's fp64 output."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from parity_util import (case, check_close, oracle_forward, oracle_logits, to_gpu, to_oracle)
+from synth import LayerShape, make_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _routing_check(deco, shape, L, G, z_exact=None, tokens=None):
+    x64 = O.to_f64(L["x"])
+    W_r64, b_r64 = O.to_f64(L["W_r"]), O.to_f64(L["b_r"])
+    res = deco.routing(G["x"], G)
+    torch.cuda.synchronize()
+    act_gpu = _np(res["active"]).astype(bool)
+    if tokens is None:
+        z = oracle_logits(x64, W_r64, b_r64) if z_exact is None else z_exact
+        act = z > 0
+        np.testing.assert_array_equal(act_gpu, act)
+        counts, offsets, perm, n_tok = O.routing_tables(act)
+        np.testing.assert_array_equal(_np(res["counts"]), counts)
+        np.testing.assert_array_equal(_np(res["offsets"]), offsets)
+        np.testing.assert_array_equal(_np(res["perm"])[: offsets[-1]], perm)
+        np.testing.assert_array_equal(_np(res["n_tok"])[: shape.T], n_tok)
+        r = _np(res["r"])
+        scale = np.abs(z).max()
+        assert np.abs(r - np.where(act, z, 0.0)).max() <= 1e-5 * scale
+        return act
+    # full-size case: exact active sets on sampled tokens, table properties on all
+    z = oracle_logits(x64[tokens], W_r64, b_r64)
+    np.testing.assert_array_equal(act_gpu[tokens], z > 0)
+    counts, offsets, perm, n_tok = O.routing_tables(act_gpu)
+    np.testing.assert_array_equal(_np(res["counts"]), counts)
+    np.testing.assert_array_equal(_np(res["offsets"]), offsets)
+    np.testing.assert_array_equal(_np(res["perm"])[: offsets[-1]], perm)
+    np.testing.assert_array_equal(_np(res["n_tok"])[: shape.T], n_tok)
+    return act_gpu
+
+
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["tiny_f32", "edge_decode_t1", "large_t16"])
+def test_mean_up_bit_exact(lib, name):
+    shape, L = case(name)
+    G = to_gpu(L, lib)
+    ref = O.mean_up(O.to_f64(L["W_up"]), shape.dtype)
+    np.testing.assert_array_equal(G["W_bar_up"].double().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "edge_decode_t1", "edge_decode_t4",
+                                  "edge_decode_t16", "large_t16", "edge_prefill_t4096"])
+def test_routing_bit_exact(lib, name):
+    shape, L = case(name)
+    G = to_gpu(L, lib)
+    act = _routing_check(lib, shape, L, G)
+    if name == "edge_prefill_t4096":
+        assert not act[::64].any()          # planted zero-expert tokens
+        ratio = act.mean()
+        assert 0.1 < ratio < 0.3
+
+
+def test_routing_full_size_large_layer(lib):
+    shape, L = case("large_t16384")
+    G = to_gpu(L, lib)
+    toks = np.random.default_rng(0).choice(shape.T, 48, replace=False)
+    _routing_check(lib, shape, L, G, tokens=np.sort(toks))
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "edge_decode_t1", "edge_decode_t4",
+                                  "edge_decode_t16", "large_t16"])
+def test_forward_parity_full(lib, name):
+    shape, L = case(name)
+    G = to_gpu(L, lib)
+    out = lib.forward(G["x"], G, eps=shape.eps)
+    torch.cuda.synchronize()
+    ref = oracle_forward(O.to_f64(L["x"]), to_oracle(L, shape.dtype), shape.eps, range(shape.T))
+    check_close(out.double().cpu().numpy(), ref, shape.dtype, name)
+
+
+@pytest.mark.parametrize("name,n", [("edge_prefill_t4096", 96), ("large_t16384", 24)])
+def test_forward_parity_full_size_sampled(lib, name, n):
+    shape, L = case(name)
+    G = to_gpu(L, lib)
+    out = lib.forward(G["x"], G, eps=shape.eps)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    toks = np.sort(np.concatenate([rng.choice(shape.T, n, replace=False), [0, 64, shape.T - 1]]))
+    ref = oracle_forward(O.to_f64(L["x"]), to_oracle(L, shape.dtype), shape.eps, toks)
+    check_close(out.double().cpu().numpy()[toks], ref, shape.dtype, name)
+
+
+# --------------------------------------------------------------------------
+# edge cases: ragged batches, degenerate routing, residual, dtypes
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T,ratio", [(1, 0.2), (37, 0.2), (70, 0.05), (19, 1.0), (23, 0.0)])
+def test_forward_edge_cases(lib, dtype, T, ratio):
+    shape = LayerShape(T, 256, 8, 128, 192, dtype)
+    L = make_layer(shape, 21, ratio=ratio if ratio > 0 else 0.2)
+    if ratio == 0.0:
+        L["b_r"] = torch.full_like(L["b_r"], -1e4)       # no token routes anywhere
+    G = to_gpu(L, lib)
+    out = lib.forward(G["x"], G, eps=shape.eps)
+    torch.cuda.synchronize()
+    L64 = to_oracle(L, dtype)
+    ref, z, act = O.layer_forward_tokens(O.to_f64(L["x"]), L64, shape.eps)
+    if ratio == 1.0:
+        assert act.all()
+    if ratio == 0.0:
+        assert not act.any()
+    check_close(out.double().cpu().numpy(), ref, dtype, f"T={T} ratio={ratio}")
+
+
+def test_single_expert_and_wide_expert(lib):
+    for shape in [LayerShape(9, 128, 1, 64, 64, "f32"), LayerShape(12, 192, 5, 512, 64, "bf16")]:
+        L = make_layer(shape, 3, ratio=0.7)
+        G = to_gpu(L, lib)
+        out = lib.forward(G["x"], G, eps=shape.eps)
+        torch.cuda.synchronize()
+        ref = O.layer_forward(O.to_f64(L["x"]), to_oracle(L, shape.dtype), shape.eps)
+        check_close(out.double().cpu().numpy(), ref, shape.dtype, str(shape))
+
+
+def test_residual_stack_of_eight_layers(lib):
+    base = case("large_t16")[0]
+    layers = [make_layer(base, 3, layer=l) for l in range(8)]
+    x0 = layers[0]["x"]
+    x = x0.cuda()
+    for L in layers:
+        G = to_gpu({k: v for k, v in L.items() if k != "x"}, lib)
+        x = lib.forward(x, G, eps=base.eps, residual=True)
+    torch.cuda.synchronize()
+    L64 = [to_oracle({k: v for k, v in L.items() if k != "x"}, "bf16") for L in layers]
+    ref = O.stack_forward(O.to_f64(x0), L64, base.eps, "bf16")
+    d = x.double().cpu().numpy() - ref
+    delta = ref - O.to_f64(x0)        # the stack's own contribution
+    rms = float(np.sqrt(np.mean(delta * delta)))
+    assert np.abs(d).max() <= 2e-2 * rms * 8, (np.abs(d).max(), rms)
+
+
+def test_forward_is_deterministic(lib):
+    shape, L = case("edge_prefill_t4096")
+    G = to_gpu(L, lib)
+    a = lib.forward(G["x"], G).clone()
+    b = lib.forward(G["x"], G)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_dense_ffn_parity(lib):
+    for dtype, (T, D, d_ff) in [("f32", (13, 256, 1152)), ("bf16", (16, 2048, 17408))]:
+        from synth import make_dense
+        Dn = make_dense(T, D, d_ff, dtype, 4)
+        out = lib.dense_ffn(Dn["x"].cuda(), Dn["W1"].cuda(), Dn["W2"].cuda())
+        torch.cuda.synchronize()
+        ref = O.dense_ffn(O.to_f64(Dn["x"]), O.to_f64(Dn["W1"]), O.to_f64(Dn["W2"]))
+        check_close(out.double().cpu().numpy(), ref, dtype, f"dense {dtype}")
+
+
+def test_nonfinite_router_input_sets_device_error(lib):
+    shape = LayerShape(4, 256, 8, 128, 128, "f32")
+    L = make_layer(shape, 2)
+    L["x"][1, 3] = float("nan")
+    G = to_gpu(L, lib)
+    ws = lib.alloc_workspace(lib.layer_shape(G["x"], G))
+    lib.forward(G["x"], G, workspace=ws)
+    assert lib.device_error(ws) == 1
+    assert lib.device_error(ws) == 0          # cleared
+    L["x"][1, 3] = 0.0
+    G["x"] = L["x"].cuda()
+    lib.forward(G["x"], G, workspace=ws)
+    assert lib.device_error(ws) == 0
