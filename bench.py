@@ -246,6 +246,10 @@ def main():
     # instrumented graphs: events around every kernel of every forward
     nk = len(deco.KERNELS)
     ev = {T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for T in DECODE_TS}
+    for es in ev.values():          # torch creates CUDA events lazily, on first record
+        for e in es:
+            e.record(stream)
+    torch.cuda.synchronize()
     igraphs = []
     for G in copies:
         g = torch.cuda.CUDAGraph()

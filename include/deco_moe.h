@@ -175,6 +175,11 @@ deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
  * Not thread-safe; meant for a single benchmarking thread. */
 deco_status_t deco_moe_set_profiling(void* const* events, int n_events);
 
+/* The name and description of the CUDA error behind the last DECO_ERR_CUDA
+ * status returned on the calling thread ("" if none).  The string is owned by
+ * the library and stays valid until the next call on this thread. */
+const char* deco_last_cuda_error(void);
+
 /* A static, human-readable name for a status code. */
 const char* deco_status_string(deco_status_t status);
 

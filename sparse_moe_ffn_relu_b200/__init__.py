@@ -30,7 +30,10 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace", 4: "
 
 class DecoError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {_lib.deco_status_string(code).decode()} (status {code})")
+        msg = f"{what}: {_lib.deco_status_string(code).decode()} (status {code})"
+        if code == 4:
+            msg += f" -- {_lib.deco_last_cuda_error().decode()}"
+        super().__init__(msg)
         self.code = code
 
 
@@ -67,9 +70,11 @@ for _name, _args in _sig.items():
     _f.restype = ctypes.c_int
 _lib.deco_status_string.argtypes = [ctypes.c_int]
 _lib.deco_status_string.restype = ctypes.c_char_p
+_lib.deco_last_cuda_error.argtypes = []
+_lib.deco_last_cuda_error.restype = ctypes.c_char_p
 
 # every symbol include/deco_moe.h declares
-EXPORTS = tuple(_sig) + ("deco_status_string",)
+EXPORTS = tuple(_sig) + ("deco_status_string", "deco_last_cuda_error")
 
 
 def _check(code: int, what: str):
@@ -191,7 +196,10 @@ def set_profiling(events):
         _prof_keep = None
         _check(_lib.deco_moe_set_profiling(None, 0), "set_profiling")
         return
-    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    handles = [e.cuda_event for e in events]
+    if not all(handles):
+        raise ValueError("set_profiling: every event must exist (record it once first)")
+    arr = (ctypes.c_void_p * len(events))(*handles)
     _prof_keep = (arr, events)
     _check(_lib.deco_moe_set_profiling(arr, len(events)), "set_profiling")
 

@@ -19,6 +19,11 @@ NVCC_FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
     "-Xcompiler", "-fPIC", "-shared",
     "--expt-relaxed-constexpr",
+    # one CUDA runtime per process: link the shared libcudart.so.12, so that
+    # stream and event handles created by the host program (e.g. PyTorch,
+    # which loads its own libcudart.so.12 first) are valid in this library
+    "-cudart", "shared",
+    "-Xlinker", "-rpath,/usr/local/cuda/lib64",
 ]
 
 

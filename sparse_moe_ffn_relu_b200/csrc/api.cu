@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <mutex>
 
 #include "../../include/deco_moe.h"
@@ -95,12 +96,24 @@ cudaError_t allow_smem(K kernel, size_t bytes) {
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+thread_local char g_cuda_msg[256] = "";
+
+// maps a CUDA error to DECO_ERR_CUDA and remembers its text for deco_last_cuda_error
+deco_status_t cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return DECO_OK;
+  snprintf(g_cuda_msg, sizeof(g_cuda_msg), "%s: %s (%s)", where, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return DECO_ERR_CUDA;
+}
+
 // benchmark timing hook (deco_moe_set_profiling)
 cudaEvent_t const* g_prof_events = nullptr;
 int g_prof_n = 0;
 
 inline void prof_mark(int idx, cudaStream_t st) {
-  if (g_prof_events && idx < g_prof_n) cudaEventRecord(g_prof_events[idx], st);
+  // external: a real event-record node when the call is being graph-captured
+  if (g_prof_events && idx < g_prof_n)
+    cudaEventRecordWithFlags(g_prof_events[idx], st, cudaEventRecordExternal);
 }
 
 // ---------------------------------------------------------------------------
@@ -241,6 +254,8 @@ using namespace deco;
 
 extern "C" {
 
+const char* deco_last_cuda_error(void) { return g_cuda_msg; }
+
 const char* deco_status_string(deco_status_t s) {
   switch (s) {
     case DECO_OK: return "ok";
@@ -275,10 +290,11 @@ deco_status_t deco_moe_forward(const deco_moe_shape_t* shape, const void* x,
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   cudaStream_t cs = as_stream(stream);
   std::lock_guard<std::mutex> lock(g_smem_mutex);
-  if (cudaMemsetAsync(ws + p.err, 0, 16, cs) != cudaSuccess) return DECO_ERR_CUDA;
-  const cudaError_t err = shape->dtype == DECO_F32 ? run_forward<float>(*shape, x, *w, out, ws, p, cs)
-                                                   : run_forward<bf16>(*shape, x, *w, out, ws, p, cs);
-  return err == cudaSuccess ? DECO_OK : DECO_ERR_CUDA;
+  cudaError_t err = cudaMemsetAsync(ws + p.err, 0, 16, cs);
+  if (err != cudaSuccess) return cuda_status(err, "forward: clearing the error word");
+  err = shape->dtype == DECO_F32 ? run_forward<float>(*shape, x, *w, out, ws, p, cs)
+                                 : run_forward<bf16>(*shape, x, *w, out, ws, p, cs);
+  return cuda_status(err, "forward");
 }
 
 deco_status_t deco_moe_routing(const deco_moe_shape_t* shape, const void* x,
@@ -302,12 +318,12 @@ deco_status_t deco_moe_routing(const deco_moe_shape_t* shape, const void* x,
   int* perm = out->perm ? out->perm : reinterpret_cast<int*>(ws + p.perm);
   int* n_tok = out->n_tok ? out->n_tok : reinterpret_cast<int*>(ws + p.n_tok);
   std::lock_guard<std::mutex> lock(g_smem_mutex);
-  if (cudaMemsetAsync(ws + p.err, 0, 16, cs) != cudaSuccess) return DECO_ERR_CUDA;
-  const cudaError_t err =
-      shape->dtype == DECO_F32
-          ? run_routing<float>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs)
-          : run_routing<bf16>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs);
-  return err == cudaSuccess ? DECO_OK : DECO_ERR_CUDA;
+  cudaError_t err = cudaMemsetAsync(ws + p.err, 0, 16, cs);
+  if (err != cudaSuccess) return cuda_status(err, "routing: clearing the error word");
+  err = shape->dtype == DECO_F32
+            ? run_routing<float>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs)
+            : run_routing<bf16>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs);
+  return cuda_status(err, "routing");
 }
 
 deco_status_t deco_moe_mean_up(int E, int d_e, int d_model, int dtype, const void* W_up,
@@ -324,7 +340,7 @@ deco_status_t deco_moe_mean_up(int E, int d_e, int d_model, int dtype, const voi
   else
     k_mean_up<bf16><<<blocks, 256, 0, cs>>>(static_cast<const bf16*>(W_up),
                                              static_cast<bf16*>(W_bar_up), E, n);
-  return cudaGetLastError() == cudaSuccess ? DECO_OK : DECO_ERR_CUDA;
+  return cuda_status(cudaGetLastError(), "mean_up");
 }
 
 // dense FFN: workspace = [err | hs [T][d_ff] fp32]
@@ -383,7 +399,7 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
     err = route_any<bf16>(ra, tt, cs);
     if (err == cudaSuccess) err = launch_down<bf16>(da, cs);
   }
-  return err == cudaSuccess ? DECO_OK : DECO_ERR_CUDA;
+  return cuda_status(err, "dense_ffn");
 }
 
 deco_status_t deco_moe_set_profiling(void* const* events, int n_events) {
@@ -397,12 +413,11 @@ deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream) {
   if (!workspace || !code) return DECO_ERR_INVALID_ARG;
   cudaStream_t cs = as_stream(stream);
   int v = 0;
-  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, cs) != cudaSuccess)
-    return DECO_ERR_CUDA;
-  if (cudaStreamSynchronize(cs) != cudaSuccess) return DECO_ERR_CUDA;
+  cudaError_t err = cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, cs);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(cs);
+  if (err != cudaSuccess) return cuda_status(err, "device_error");
   *code = v;
-  if (cudaMemsetAsync(workspace, 0, sizeof(int), cs) != cudaSuccess) return DECO_ERR_CUDA;
-  return DECO_OK;
+  return cuda_status(cudaMemsetAsync(workspace, 0, sizeof(int), cs), "device_error: clear");
 }
 
 }  // extern "C"
