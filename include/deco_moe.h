@@ -166,6 +166,36 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
  * it.  Returns DECO_ERR_CUDA if the synchronisation fails. */
 deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
 
+/* Size of the library's built-in device scratch used by
+ * deco_moe_forward_static: 16 MiB on every GPU that loads the library. */
+#define DECO_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* deco_moe_forward without a caller-provided workspace.  The paper has no
+ * counterpart for this; it exists for callers that cannot allocate device
+ * memory on their execution path -- for example a host whose memory budget is
+ * fixed and fully handed out before it starts running layers, or a plugin
+ * called back from another runtime that owns every allocation -- where a
+ * cudaMalloc would fail, or would synchronise the device and stall the other
+ * work on it.  Instead of a workspace argument, it uses a scratch array of
+ * DECO_STATIC_SCRATCH_BYTES compiled into the library (static device memory,
+ * held by every GPU that loads the library until the process exits).  It
+ * allocates nothing, and runs the same kernels, with the same results, as
+ * deco_moe_forward.
+ *  - Shapes whose deco_moe_workspace_size exceeds DECO_STATIC_SCRATCH_BYTES
+ *    are rejected with DECO_ERR_WORKSPACE before anything is launched (decode
+ *    batches of the layers in this library fit: e.g. T = 16 needs ~1.1 MB at
+ *    d_model 2048 / 64 experts and ~2.3 MB at d_model 4096 / 128 experts).
+ *  - The first call on each device looks up the scratch array's device
+ *    address (cudaGetSymbolAddress, a runtime call made with that device
+ *    current); make that first call before any stream capture on the device.
+ *  - All calls on a device share the one array.  Calls whose executions
+ *    overlap on the GPU (different streams, or several threads) race on it and
+ *    give wrong results; serialise them, e.g. on one stream.  Each call
+ *    clears what must start at zero; the rest is overwritten.
+ * Other arguments, results and errors are those of deco_moe_forward. */
+deco_status_t deco_moe_forward_static(const deco_moe_shape_t* shape, const void* x,
+                                      const deco_moe_weights_t* w, void* out, void* stream);
+
 /* Kernel timing hook for benchmarks.  While set (events != NULL), every later
  * deco_moe_forward call on this process records events[2*i] on its stream just
  * before its i-th kernel and events[2*i+1] just after it, for i < n_events/2;

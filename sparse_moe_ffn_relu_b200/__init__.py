@@ -63,6 +63,7 @@ _sig = {
     "deco_dense_ffn_forward": [ctypes.c_int] * 4 + [_vp] * 4 + [_vp, _sz, _vp],
     "deco_moe_device_error": [_vp, ctypes.POINTER(ctypes.c_int), _vp],
     "deco_moe_set_profiling": [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int],
+    "deco_moe_forward_static": [ctypes.POINTER(Shape), _vp, ctypes.POINTER(Weights), _vp, _vp],
 }
 for _name, _args in _sig.items():
     _f = getattr(_lib, _name)
@@ -129,6 +130,25 @@ def forward(x: torch.Tensor, L: dict, out=None, workspace=None, eps=1e-6, residu
     w = _weights(L)
     _check(_lib.deco_moe_forward(ctypes.byref(shape), _ptr(x), ctypes.byref(w), _ptr(out),
                                  _ptr(workspace), workspace.numel(), _stream(stream)), "forward")
+    return out
+
+
+STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def forward_static(x: torch.Tensor, L: dict, out=None, eps=1e-6, residual=False,
+                   stream=None) -> torch.Tensor:
+    """forward() on the library's built-in 16 MiB device scratch instead of a
+    workspace, for callers that cannot allocate device memory while running
+    layers.  Calls on one device share that scratch: do not let them overlap
+    on the GPU.  The first call on a device should come before any stream
+    capture.  Raises DecoError (status 3) if the shape needs more scratch."""
+    shape = layer_shape(x, L, eps, residual)
+    if out is None:
+        out = torch.empty_like(x)
+    w = _weights(L)
+    _check(_lib.deco_moe_forward_static(ctypes.byref(shape), _ptr(x), ctypes.byref(w), _ptr(out),
+                                        _stream(stream)), "forward_static")
     return out
 
 

@@ -421,3 +421,57 @@ deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// deco_moe_forward_static: the forward pass on a library-owned static scratch
+// array instead of a caller workspace, for callers that cannot allocate.
+
+namespace deco {
+namespace {
+
+// The scratch every deco_moe_forward_static call on a device uses.  Host code
+// must not pass `g_static_scratch` itself to a kernel: on the host the name is
+// only a stand-in for the symbol, so its device address is looked up once per
+// device with cudaGetSymbolAddress and cached here.
+static __device__ __align__(256) unsigned char g_static_scratch[DECO_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mutex;
+void* g_static_ptr[kMaxDevices] = {};
+
+// address of this device's scratch array (set up on the first call per device)
+cudaError_t static_scratch(unsigned char** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (err != cudaSuccess) return err;
+    g_static_ptr[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_static_ptr[dev]);
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace deco
+
+extern "C" deco_status_t deco_moe_forward_static(const deco_moe_shape_t* shape, const void* x,
+                                                 const deco_moe_weights_t* w, void* out,
+                                                 void* stream) {
+  deco_status_t st = check_shape(shape);
+  if (st != DECO_OK) return st;
+  if ((st = check_weights(w, false)) != DECO_OK) return st;
+  if (shape->T == 0) return DECO_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out) || x == out) return DECO_ERR_INVALID_ARG;
+  if (make_plan(*shape).total > DECO_STATIC_SCRATCH_BYTES) return DECO_ERR_WORKSPACE;
+  unsigned char* scratch = nullptr;
+  const cudaError_t err = static_scratch(&scratch);
+  if (err != cudaSuccess) return cuda_status(err, "forward_static: scratch address");
+  // the forward pass clears the error word it keeps at the start of the
+  // scratch and overwrites everything else it reads
+  return deco_moe_forward(shape, x, w, out, scratch, DECO_STATIC_SCRATCH_BYTES, stream);
+}
