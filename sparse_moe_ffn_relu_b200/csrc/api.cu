@@ -10,6 +10,7 @@
 
 #include "../../include/deco_moe.h"
 #include "simt_kernels.cuh"
+#include "decode_kernels.cuh"
 
 namespace deco {
 namespace {
@@ -18,7 +19,7 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace layout of one forward / routing call.
 struct Plan {
-  size_t err, r, act, u, hs, counts, offsets, n_tok, perm, pair_of, tiles, n_tiles, H, total;
+  size_t err, r, act, u, hs, counts, offsets, n_tok, perm, pair_of, tiles, n_tiles, H, A, done, total;
   int tile_rows;
 };
 
@@ -49,7 +50,9 @@ Plan make_plan(const deco_moe_shape_t& s) {
   p.pair_of = take(P * 4);
   p.tiles = take((P / p.tile_rows + E) * 16);
   p.n_tiles = take(4);
-  p.H = take(P * s.d_e * 4);
+  p.H = take(P * s.d_e * 4);       // general path: activations; decode path: centred c
+  p.A = take(P * s.d_e * 2);       // decode path: NormSiLU activations (bf16)
+  p.done = take(E * 4);            // decode path: finished rows per expert
   p.total = off;
   return p;
 }
@@ -195,9 +198,105 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// decode path: bf16, T <= 16 (weight-streaming kernels, see decode_kernels.cuh)
+
+// kd_down stage: 32 KB, or one expert's weight rows plus its activation rows
+uint32_t down_stage_bytes(const deco_moe_shape_t& s, int sms) {
+  const uint32_t rows = (uint32_t)((s.d_model + sms - 1) / sms);
+  const uint32_t need = rows * s.d_e * 2 + (uint32_t)s.T * s.d_e * 2;
+  return std::max<uint32_t>(32768u, (need + 127u) & ~127u);
+}
+
+bool decode_eligible(const deco_moe_shape_t& s, int sms) {
+  if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT) return false;
+  if (s.d_model % 256 || s.d_model > 4096) return false;
+  if (s.E > 256 || s.d_e > 512) return false;
+  if ((s.d_model + sms - 1) / sms > 32) return false;          // <= 32 output rows per CTA
+  // shared activations (and r) in shared memory next to >= 2 ring stages
+  if (dec::smem_plan(((uint32_t)s.T * s.d_s * 2 + 127u) / 128u * 128u + (uint32_t)s.T * s.E * 4,
+                     down_stage_bytes(s, sms)).nstages < 2)
+    return false;
+  if (dec::smem_plan((uint32_t)s.T * s.d_model * 2, dec::kStageBytes).nstages < 2) return false;
+  return true;
+}
+
+template <typename K>
+cudaError_t launch_dec(K kernel, const dec::Args& a, uint32_t operand_bytes, uint32_t stage_bytes,
+                       bool pdl, int grid, cudaStream_t st) {
+  const dec::SmemPlan sp = dec::smem_plan(operand_bytes, stage_bytes);
+  if (sp.nstages < 2) return cudaErrorInvalidConfiguration;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(dec::kThreads);
+  cfg.dynamicSmemBytes = sp.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
+                       void* out, unsigned char* ws, const Plan& p, int sms, cudaStream_t st) {
+  dec::Args a{};
+  a.T = s.T;
+  a.D = s.d_model;
+  a.E = s.E;
+  a.d_e = s.d_e;
+  a.d_s = s.d_s;
+  a.eps = s.rms_eps;
+  a.residual = s.residual;
+  a.x = static_cast<const bf16*>(x);
+  a.W_r = static_cast<const bf16*>(w.W_r);
+  a.b_r = w.b_r;
+  a.W_bar = static_cast<const bf16*>(w.W_bar_up);
+  a.W_up = static_cast<const bf16*>(w.W_up);
+  a.W_down = static_cast<const bf16*>(w.W_down);
+  a.s = w.s;
+  a.W_s_up = static_cast<const bf16*>(w.W_s_up);
+  a.W_s_down = static_cast<const bf16*>(w.W_s_down);
+  a.r = reinterpret_cast<float*>(ws + p.r);
+  a.act = reinterpret_cast<uint8_t*>(ws + p.act);
+  a.u = reinterpret_cast<float*>(ws + p.u);
+  a.hs = reinterpret_cast<bf16*>(ws + p.hs);
+  a.C = reinterpret_cast<float*>(ws + p.H);
+  a.A = reinterpret_cast<bf16*>(ws + p.A);
+  a.done = reinterpret_cast<int*>(ws + p.done);
+  a.err = reinterpret_cast<int*>(ws + p.err);
+  a.out = static_cast<bf16*>(out);
+  a.down_stage = down_stage_bytes(s, sms);
+  const uint32_t xbytes = (uint32_t)s.T * s.d_model * 2;
+  const uint32_t hbytes = (((uint32_t)s.T * s.d_s * 2 + 127) & ~127u) + (uint32_t)s.T * s.E * 4;
+  // with timing events between the kernels each one is timed on its own
+  const bool pdl = g_prof_events == nullptr;
+  prof_mark(0, st);
+  cudaError_t err = launch_dec(dec::kd_route, a, xbytes, dec::kStageBytes, false, sms, st);
+  if (err != cudaSuccess) return err;
+  prof_mark(1, st);
+  prof_mark(2, st);
+  prof_mark(3, st);
+  prof_mark(4, st);
+  prof_mark(5, st);
+  prof_mark(6, st);
+  err = launch_dec(dec::kd_up, a, xbytes, dec::kStageBytes, pdl, sms, st);
+  if (err != cudaSuccess) return err;
+  prof_mark(7, st);
+  prof_mark(8, st);
+  err = launch_dec(dec::kd_down, a, hbytes, a.down_stage, pdl, sms, st);
+  prof_mark(9, st);
+  return err;
+}
+
 template <typename T>
 cudaError_t run_forward(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
                         void* out, unsigned char* ws, const Plan& p, cudaStream_t st) {
+  const int sms = num_sms();
+  if (decode_eligible(s, sms)) return run_decode(s, x, w, out, ws, p, sms, st);
   float* r = reinterpret_cast<float*>(ws + p.r);
   uint8_t* act = reinterpret_cast<uint8_t*>(ws + p.act);
   int* counts = reinterpret_cast<int*>(ws + p.counts);

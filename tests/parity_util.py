@@ -2,6 +2,7 @@
 GPU, evaluate the oracle (optionally in a spawn process pool), compare."""
 from __future__ import annotations
 
+import json
 import multiprocessing as mp
 import os
 
@@ -93,5 +94,11 @@ def check_close(got: np.ndarray, ref: np.ndarray, dtype: str, what=""):
         return 0.0
     excess = np.abs(got - ref) - half_ulp(ref, dtype)
     err = float(max(excess.max(), 0.0))
+    log = os.environ.get("DECO_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"what": what, "dtype": dtype, "err_over_rms": err / rms if rms else 0.0,
+                                "raw_max_over_rms": float(np.abs(got - ref).max()) / rms if rms else 0.0})
+                    + "\n")
     assert err <= TOL[dtype] * rms, f"{what}: max|err| {err:.3e} > {TOL[dtype]} * RMS {rms:.3e}"
     return err / rms if rms else 0.0

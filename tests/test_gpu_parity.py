@@ -132,20 +132,32 @@ def test_single_expert_and_wide_expert(lib):
 
 
 def test_residual_stack_of_eight_layers(lib):
+    """The 8-layer residual stack of the larger layer shape.
+
+    Each layer is checked on the oracle's own input to that layer (its stack
+    state, a bf16 tensor) at the stated tolerance.  Without a normalisation
+    between layers the stack's activations grow ~3.6x per layer (x_{l+1} =
+    x_l + layer(x_l), with the layer's output scaling with |x|), so small
+    per-layer differences compound; the GPU's own 8-layer stack is therefore
+    compared end to end in norm, not element-wise."""
     base = case("large_t16")[0]
     layers = [make_layer(base, 3, layer=l) for l in range(8)]
-    x0 = layers[0]["x"]
-    x = x0.cuda()
-    for L in layers:
-        G = to_gpu({k: v for k, v in L.items() if k != "x"}, lib)
-        x = lib.forward(x, G, eps=base.eps, residual=True)
-    torch.cuda.synchronize()
-    L64 = [to_oracle({k: v for k, v in L.items() if k != "x"}, "bf16") for L in layers]
-    ref = O.stack_forward(O.to_f64(x0), L64, base.eps, "bf16")
-    d = x.double().cpu().numpy() - ref
-    delta = ref - O.to_f64(x0)        # the stack's own contribution
-    rms = float(np.sqrt(np.mean(delta * delta)))
-    assert np.abs(d).max() <= 2e-2 * rms * 8, (np.abs(d).max(), rms)
+    x = O.to_f64(layers[0]["x"])
+    xg = layers[0]["x"].cuda()
+    for l, L in enumerate(layers):
+        W = {k: v for k, v in L.items() if k != "x"}
+        G = to_gpu(W, lib)
+        L64 = to_oracle(W, "bf16")
+        xin = torch.from_numpy(x).to(torch.bfloat16).cuda()      # exact: x is bf16-valued
+        out = lib.forward(xin, G, eps=base.eps, residual=True)
+        xg = lib.forward(xg, G, eps=base.eps, residual=True)
+        torch.cuda.synchronize()
+        ref = x + O.layer_forward(x, L64, base.eps)
+        check_close(out.double().cpu().numpy(), ref, "bf16", f"stack layer {l}")
+        x = O.round_storage(ref, "bf16")
+    d = xg.double().cpu().numpy() - x
+    rel = float(np.linalg.norm(d) / np.linalg.norm(x))
+    assert rel <= 0.1, rel
 
 
 def test_forward_is_deterministic(lib):
@@ -180,3 +192,22 @@ def test_nonfinite_router_input_sets_device_error(lib):
     G["x"] = L["x"].cuda()
     lib.forward(G["x"], G, workspace=ws)
     assert lib.device_error(ws) == 0
+
+
+@pytest.mark.parametrize("T,ratio", [(1, 0.0), (1, 1.0), (5, 0.2), (16, 0.0), (16, 1.0), (11, 0.4)])
+def test_decode_path_edge_cases(lib, T, ratio):
+    # bf16, T <= 16, d_model a multiple of 256: the weight-streaming decode kernels
+    shape = LayerShape(T, 512, 16, 256, 256, "bf16")
+    L = make_layer(shape, 31, ratio=ratio if ratio > 0 else 0.2)
+    if ratio == 0.0:
+        L["b_r"] = torch.full_like(L["b_r"], -1e4)
+    G = to_gpu(L, lib)
+    out = lib.forward(G["x"], G, eps=shape.eps)
+    torch.cuda.synchronize()
+    ref, z, act = O.layer_forward_tokens(O.to_f64(L["x"]), to_oracle(L, "bf16"), shape.eps)
+    assert act.all() if ratio == 1.0 else True
+    check_close(out.double().cpu().numpy(), ref, "bf16", f"decode T={T} ratio={ratio}")
+    # repeated calls reuse the workspace (counters, activations) and agree bitwise
+    out2 = lib.forward(G["x"], G, eps=shape.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
