@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--profile-tokens", type=int, default=0,
+                    help="profiling mode: only run eager forward passes of the edge layer at this "
+                         "batch size (warmup + steps), print nothing; for ncu captures")
     return ap.parse_args()
 
 
@@ -187,6 +190,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.profile_tokens:
+        profile_only(args)
         return
 
     import numpy as np
@@ -383,6 +389,26 @@ def main():
         del g
     if dist is not None:
         dist.destroy_process_group()
+
+
+def profile_only(args):
+    """Eager forward passes of the edge layer at one batch size, for ncu:
+    warmup forwards first, then `steps` more; kernels in launch order
+    route, up, down (decode path) or route, count, scatter, up, down."""
+    import torch
+
+    import sparse_moe_ffn_relu_b200 as deco
+    from synth import CONFIGS, LayerShape, make_layer
+    base = CONFIGS["edge_decode_t16"]["shape"]
+    shape = LayerShape(args.profile_tokens, base.D, base.E, base.d_e, base.d_s, base.dtype)
+    L = make_layer(shape, CONFIGS["edge_decode_t16"]["seed"])
+    G = {k: v.cuda() for k, v in L.items()}
+    G["W_bar_up"] = deco.mean_up(G["W_up"])
+    ws = deco.alloc_workspace(deco.layer_shape(G["x"], G))
+    out = torch.empty_like(G["x"])
+    for _ in range(args.warmup + args.steps):
+        deco.forward(G["x"], G, out=out, workspace=ws)
+    torch.cuda.synchronize()
 
 
 def extras(deco, dev, stream, P):

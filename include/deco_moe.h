@@ -167,8 +167,8 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
 deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
 
 /* Size of the library's built-in device scratch used by
- * deco_moe_forward_static: 16 MiB on every GPU that loads the library. */
-#define DECO_STATIC_SCRATCH_BYTES (16u << 20)
+ * deco_moe_forward_static: 32 MiB on every GPU that loads the library. */
+#define DECO_STATIC_SCRATCH_BYTES (32u << 20)
 
 /* deco_moe_forward without a caller-provided workspace.  The paper has no
  * counterpart for this; it exists for callers that cannot allocate device
@@ -183,8 +183,8 @@ deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
  * deco_moe_forward.
  *  - Shapes whose deco_moe_workspace_size exceeds DECO_STATIC_SCRATCH_BYTES
  *    are rejected with DECO_ERR_WORKSPACE before anything is launched (decode
- *    batches of the layers in this library fit: e.g. T = 16 needs ~1.1 MB at
- *    d_model 2048 / 64 experts and ~2.3 MB at d_model 4096 / 128 experts).
+ *    batches of the layers in this library fit: e.g. T = 16 needs ~20 MB at
+ *    d_model 2048 / 64 experts and ~26 MB at d_model 4096 / 128 experts).
  *  - The first call on each device looks up the scratch array's device
  *    address (cudaGetSymbolAddress, a runtime call made with that device
  *    current); make that first call before any stream capture on the device.

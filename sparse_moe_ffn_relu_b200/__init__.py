@@ -133,12 +133,12 @@ def forward(x: torch.Tensor, L: dict, out=None, workspace=None, eps=1e-6, residu
     return out
 
 
-STATIC_SCRATCH_BYTES = 16 << 20
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 def forward_static(x: torch.Tensor, L: dict, out=None, eps=1e-6, residual=False,
                    stream=None) -> torch.Tensor:
-    """forward() on the library's built-in 16 MiB device scratch instead of a
+    """forward() on the library's built-in 32 MiB device scratch instead of a
     workspace, for callers that cannot allocate device memory while running
     layers.  Calls on one device share that scratch: do not let them overlap
     on the GPU.  The first call on a device should come before any stream

@@ -1,8 +1,11 @@
 // Host side of the C ABI declared in include/deco_moe.h: argument checks,
 // workspace plan and the launch sequence.  No allocation, no synchronisation
 // (except deco_moe_device_error), so every call can be graph-captured.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -19,11 +22,21 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace layout of one forward / routing call.
 struct Plan {
-  size_t err, r, act, u, hs, counts, offsets, n_tok, perm, pair_of, tiles, n_tiles, H, A, done, total;
+  size_t err, r, act, u, hs, counts, offsets, n_tok, perm, pair_of, tiles, n_tiles, H, total;
+  // decode path (T <= 16)
+  size_t hs16, C16, a_cmp, cnt;
+  size_t cnt_bytes;
   int tile_rows;
+  int sms;
 };
 
 inline size_t elem_size(int dtype) { return dtype == DECO_F32 ? 4 : 2; }
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
 
 // rows of x staged per CTA: 16 when the tile fits in 128 KB of shared memory
 inline int token_tile(int D, int dtype) { return (16 * (size_t)D * elem_size(dtype) <= 131072) ? 16 : 8; }
@@ -50,9 +63,15 @@ Plan make_plan(const deco_moe_shape_t& s) {
   p.pair_of = take(P * 4);
   p.tiles = take((P / p.tile_rows + E) * 16);
   p.n_tiles = take(4);
-  p.H = take(P * s.d_e * 4);       // general path: activations; decode path: centred c
-  p.A = take(P * s.d_e * 2);       // decode path: NormSiLU activations (bf16)
-  p.done = take(E * 4);            // decode path: finished rows per expert
+  p.H = take(P * s.d_e * 4);       // general path: NormSiLU activations
+  if (s.T <= dec::kMaxT) {         // decode path buffers (see decode_kernels.cuh)
+    p.sms = num_sms();
+    p.hs16 = take((size_t)dec::kTok * s.d_s * 4);         // [16][hi d_s | lo d_s] bf16
+    p.C16 = take(E * dec::kTok * s.d_e * 4);               // [E][16][d_e] fp32
+    p.a_cmp = take(E * dec::kTok * s.d_e * 4);             // [E][16][hi d_e | lo d_e] bf16
+    p.cnt_bytes = E * 4;
+    p.cnt = take(p.cnt_bytes);
+  }
   p.total = off;
   return p;
 }
@@ -82,12 +101,6 @@ deco_status_t check_weights(const deco_moe_weights_t* w, bool router_only) {
   for (const void* p : ps)
     if (!p || !aligned16(p)) return DECO_ERR_INVALID_ARG;
   return DECO_OK;
-}
-
-int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n;
 }
 
 // Opt every kernel into the dynamic shared memory it may use (once per device).
@@ -201,37 +214,31 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
 // ---------------------------------------------------------------------------
 // decode path: bf16, T <= 16 (weight-streaming kernels, see decode_kernels.cuh)
 
-// kd_down stage: 32 KB, or one expert's weight rows plus its activation rows
-uint32_t down_stage_bytes(const deco_moe_shape_t& s, int sms) {
-  const uint32_t rows = (uint32_t)((s.d_model + sms - 1) / sms);
-  const uint32_t need = rows * s.d_e * 2 + (uint32_t)s.T * s.d_e * 2;
-  return std::max<uint32_t>(32768u, (need + 127u) & ~127u);
-}
-
 bool decode_eligible(const deco_moe_shape_t& s, int sms) {
   if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT) return false;
   if (s.d_model % 256 || s.d_model > 4096) return false;
-  if (s.E > 256 || s.d_e > 512) return false;
-  if ((s.d_model + sms - 1) / sms > 32) return false;          // <= 32 output rows per CTA
-  // shared activations (and r) in shared memory next to >= 2 ring stages
-  if (dec::smem_plan(((uint32_t)s.T * s.d_s * 2 + 127u) / 128u * 128u + (uint32_t)s.T * s.E * 4,
-                     down_stage_bytes(s, sms)).nstages < 2)
+  if (s.E > 256 || s.d_e > 512 || s.d_e % 64 || s.d_s % 64 || s.d_s > 2048) return false;
+  if ((s.E + 7) / 8 >= sms) return false;                     // router CTAs leave room
+  const int R = dec::down_rows(s.d_model, sms);
+  if (R > 32) return false;                                    // two 16-row m-tiles per CTA
+  // one routed expert's slab plus its activation rows fit one stage
+  if (((uint32_t)R * s.d_e * 2 + 127u) / 128u * 128u + (uint32_t)s.T * s.d_e * 4 > dec::kStageBytes) return false;
+  const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
+  if (dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).nstages < 2) return false;
+  if (dec::smem_plan(xop, dec::kStageBytes).nstages < 2) return false;
+  if (dec::smem_plan((uint32_t)dec::kTok * s.d_s * 4 + 8 * 2048 + (uint32_t)s.d_e * 4, dec::kStageBytes).nstages < 2)
     return false;
-  if (dec::smem_plan((uint32_t)s.T * s.d_model * 2, dec::kStageBytes).nstages < 2) return false;
   return true;
 }
 
 template <typename K>
-cudaError_t launch_dec(K kernel, const dec::Args& a, uint32_t operand_bytes, uint32_t stage_bytes,
-                       bool pdl, int grid, cudaStream_t st) {
-  const dec::SmemPlan sp = dec::smem_plan(operand_bytes, stage_bytes);
-  if (sp.nstages < 2) return cudaErrorInvalidConfiguration;
-  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+cudaError_t launch_dec(K kernel, const dec::Args& a, uint32_t smem_total, bool pdl, int grid, cudaStream_t st) {
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(dec::kThreads);
-  cfg.dynamicSmemBytes = sp.total;
+  cfg.dynamicSmemBytes = smem_total;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -242,7 +249,7 @@ cudaError_t launch_dec(K kernel, const dec::Args& a, uint32_t operand_bytes, uin
 }
 
 cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
-                       void* out, unsigned char* ws, const Plan& p, int sms, cudaStream_t st) {
+                       void* out, unsigned char* ws, const Plan& p, cudaStream_t st) {
   dec::Args a{};
   a.T = s.T;
   a.D = s.d_model;
@@ -263,19 +270,24 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
   a.r = reinterpret_cast<float*>(ws + p.r);
   a.act = reinterpret_cast<uint8_t*>(ws + p.act);
   a.u = reinterpret_cast<float*>(ws + p.u);
-  a.hs = reinterpret_cast<bf16*>(ws + p.hs);
-  a.C = reinterpret_cast<float*>(ws + p.H);
-  a.A = reinterpret_cast<bf16*>(ws + p.A);
-  a.done = reinterpret_cast<int*>(ws + p.done);
+  a.hs = reinterpret_cast<bf16*>(ws + p.hs16);
+  a.C = reinterpret_cast<float*>(ws + p.C16);
+  a.a_cmp = reinterpret_cast<bf16*>(ws + p.a_cmp);
+  a.cnt_u = reinterpret_cast<int*>(ws + p.cnt);
   a.err = reinterpret_cast<int*>(ws + p.err);
   a.out = static_cast<bf16*>(out);
-  a.down_stage = down_stage_bytes(s, sms);
-  const uint32_t xbytes = (uint32_t)s.T * s.d_model * 2;
-  const uint32_t hbytes = (((uint32_t)s.T * s.d_s * 2 + 127) & ~127u) + (uint32_t)s.T * s.E * 4;
+  // completion counters start at zero every call
+  cudaError_t err = cudaMemsetAsync(ws + p.cnt, 0, p.cnt_bytes, st);
+  if (err != cudaSuccess) return err;
+  const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
+  const uint32_t route_smem = std::max(dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).total,
+                                       dec::smem_plan(xop, dec::kStageBytes).total);
+  const uint32_t down_smem =
+      dec::smem_plan((uint32_t)dec::kTok * s.d_s * 4 + 8 * 2048 + (uint32_t)s.d_e * 4, dec::kStageBytes).total;
   // with timing events between the kernels each one is timed on its own
   const bool pdl = g_prof_events == nullptr;
   prof_mark(0, st);
-  cudaError_t err = launch_dec(dec::kd_route, a, xbytes, dec::kStageBytes, false, sms, st);
+  err = launch_dec(dec::kd_route, a, route_smem, false, p.sms, st);
   if (err != cudaSuccess) return err;
   prof_mark(1, st);
   prof_mark(2, st);
@@ -283,11 +295,11 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
   prof_mark(4, st);
   prof_mark(5, st);
   prof_mark(6, st);
-  err = launch_dec(dec::kd_up, a, xbytes, dec::kStageBytes, pdl, sms, st);
+  err = launch_dec(dec::kd_up, a, dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).total, pdl, p.sms, st);
   if (err != cudaSuccess) return err;
   prof_mark(7, st);
   prof_mark(8, st);
-  err = launch_dec(dec::kd_down, a, hbytes, a.down_stage, pdl, sms, st);
+  err = launch_dec(dec::kd_down, a, down_smem, pdl, p.sms, st);
   prof_mark(9, st);
   return err;
 }
@@ -295,8 +307,7 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
 template <typename T>
 cudaError_t run_forward(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
                         void* out, unsigned char* ws, const Plan& p, cudaStream_t st) {
-  const int sms = num_sms();
-  if (decode_eligible(s, sms)) return run_decode(s, x, w, out, ws, p, sms, st);
+  if (s.T <= dec::kMaxT && decode_eligible(s, p.sms)) return run_decode(s, x, w, out, ws, p, st);
   float* r = reinterpret_cast<float*>(ws + p.r);
   uint8_t* act = reinterpret_cast<uint8_t*>(ws + p.act);
   int* counts = reinterpret_cast<int*>(ws + p.counts);

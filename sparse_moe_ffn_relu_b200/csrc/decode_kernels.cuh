@@ -4,26 +4,48 @@
 // most 16 tokens, and only the routed experts that some token activates need
 // to be read (the paper's point about sparse activation saving memory access,
 // "DECO: Sparse Mixture-of-Experts with Dense-Comparable Performance on
-// End-Side Devices", §1 and §5).  The three kernels therefore stream weights:
+// End-Side Devices", §1 and §5).  Three kernels stream the weights once:
 //
-//   kd_route  rows [W_r ; W_bar_up ; W_s_up]  -> r, active, u, SiLU(shared up)
-//   kd_up     rows of W_up[e] for the union of active experts -> centred
-//             activations c = g - u; the CTA that completes an expert applies
-//             NormSiLU's RMS normalisation and SiLU to that expert's tokens
-//   kd_down   each CTA owns a block of output rows and walks the shared
-//             expert, then the active experts in ascending order, so every
-//             output element is summed in one fixed order (no atomics)
+//   kd_route  router rows W_r (exact activation decisions, CUDA cores), and
+//             the mean up-projection W_bar_up and shared up-projection W_s_up
+//             (tensor cores) -> r, active, u = x W_bar_up^T, SiLU(x W_s_up^T)
+//   kd_up     W_up[e] of the union of active experts (tensor cores); the CTA
+//             that completes an expert applies NormSiLU (subtract u, RMS over
+//             d_e, SiLU) and writes s_e * r_e * a for its tokens
+//   kd_down   each CTA owns a block of output rows and accumulates the shared
+//             expert and every active expert's down-projection for them
 //
-// Every kernel runs one CTA per SM with 8 consumer warps and 1 producer warp.
-// The producer streams the CTA's weight rows into a ring of 32 KB shared-memory
-// stages with cp.async.bulk (evict-first in L2), signalled by mbarriers; the
-// consumers compute from shared memory.  Rows are split evenly over the CTAs.
+// Data movement: one CTA per SM, 8 consumer warps and 1 producer warp.  The
+// producer streams contiguous weight rows with bulk copies of >= 4 KB each
+// (cp.async.bulk, L2 evict-first) into a ring of shared-memory stages behind
+// mbarriers; on B200 a copy engine sustains HBM bandwidth with copies this
+// size, while small tensor-map boxes (2 KB) are limited by per-copy cost.
+// kd_route / kd_up give each CTA a contiguous range of weight rows at full
+// width and copy each row into a 16-byte padded shared-memory row, so that
+// ldmatrix reads of 8 rows hit 8 different bank groups; the 8 consumer warps
+// split the columns and add their partial sums in warp order.  kd_down gives
+// each CTA a block of output rows; each active expert's slab of those rows is
+// one contiguous copy, which a warp re-lays into a swizzled tile before use.
+// Activations a later kernel consumes are written in a layout its copies and
+// ldmatrix reads can use directly (an XOR swizzle of the 16-byte chunks inside
+// each row).
+//
+// Arithmetic: the projections are tiny dense contractions (16 tokens x 8..64
+// weight rows x K) done with mma.sync m16n8k16 (bf16 in, fp32 accumulate): a
+// tensor-core instruction per 16x8x16 tile keeps the instruction count far
+// below the memory time.  (tcgen05's smallest tile, M = 64, would make the
+// tensor core read several times the shared memory these tiles occupy.)
+// Intermediates fed back into a contraction (the shared expert's hidden
+// activations and the scaled NormSiLU outputs) are stored as a bf16 pair
+// hi + lo with lo = bf16(v - hi), and both halves are multiplied, so they
+// carry ~16 significant bits instead of 8.
+//
 // Waits are bounded: after ~1 s a wait gives up, sets bit 2 of the device
-// error word and the CTA stops issuing work (no hang, no trap).
-// Consecutive kernels use programmatic dependent launch: a kernel starts
-// while its predecessor drains and waits (griddepcontrol.wait) only before it
-// reads what the predecessor wrote.
+// error word and the CTA stops issuing work (no hang, no trap).  Consecutive
+// kernels use programmatic dependent launch.
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 
@@ -33,11 +55,13 @@ namespace dec {
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxT = 16;                      // decode batches
+constexpr int kTok = 16;                       // token rows of every activation tile
 constexpr uint32_t kStageBytes = 32768;
 constexpr int kMaxStages = 8;
 constexpr size_t kSmemLimit = 232448;          // 227 KB opt-in per CTA on sm_100
 constexpr long long kWaitCycles = 2000000000ll;  // ~1 s at 1.9 GHz
 constexpr int kErrTimeout = 2;
+constexpr int kKB = 64;                        // columns per weight tile (128 B of bf16)
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -102,13 +126,70 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// 2-D TMA tile load (coordinates: column, row); columns are a multiple of 64
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int col, int row, uint64_t* bar,
+                                       uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int col, int row, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+__device__ __forceinline__ void consumer_sync() {   // the 8 consumer warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& q, float (&v)[8]) { unpack16(q, v); }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// D[16 x 8] += A[16 x 16] B[16 x 8], bf16 inputs, fp32 accumulators
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Tiles of R rows x 64 bf16 columns, 128 B per row, at a 1024-B aligned
+// base: 16-byte chunk c of row r sits at chunk position c ^ (r & 7).  This is
+// the TMA 128-byte swizzle, and ldmatrix reads of 8 rows at one chunk hit 8
+// different bank groups.
+__device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk) {
+  return base + (uint32_t)row * 128u + ((uint32_t)(chunk ^ (row & 7)) << 4);
+}
+__host__ __device__ constexpr uint32_t tile_bytes(int rows) {   // rows x 128 B, 1024-B multiple
+  return (uint32_t)((rows * 128 + 1023) / 1024 * 1024);
+}
+
+// ldmatrix address of this lane for the A operand (16 token rows x 16 columns
+// at k-step ks of a 64-column tile)
+__device__ __forceinline__ uint32_t a_addr(uint32_t tile, int lane, int ks) {
+  return swz(tile, (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4));
+}
+// ... for the B operand, rows r0..r0+15 (x4: two n-tiles) or r0..r0+7 (x2)
+__device__ __forceinline__ uint32_t b_addr(uint32_t tile, int lane, int ks, int r0) {
+  return swz(tile, r0 + (lane & 7) + (lane >> 4) * 8, 2 * ks + ((lane >> 3) & 1));
+}
 
 // ---------------------------------------------------------------------------
 // Ring of weight stages shared by the three kernels.
@@ -121,9 +202,9 @@ struct Ring {
   int nstages;
 };
 
-// dynamic shared memory layout: [barriers 256 B][ring stages][kernel operand];
+// dynamic shared memory: [<=1 KB alignment slack][barriers 1 KB][ring][operand];
 // kStaticReserve bytes are left for each kernel's static __shared__ arrays.
-constexpr uint32_t kHeaderBytes = 256;
+constexpr uint32_t kHeaderBytes = 1024;
 constexpr uint32_t kStaticReserve = 1536;
 
 struct SmemPlan {
@@ -135,18 +216,19 @@ __host__ __device__ inline SmemPlan smem_plan(uint32_t operand_bytes, uint32_t s
   SmemPlan p;
   p.ring_off = kHeaderBytes;
   p.stage_bytes = stage_bytes;
-  const uint32_t room = (uint32_t)kSmemLimit - kStaticReserve - kHeaderBytes -
-                        ((operand_bytes + 127) & ~127u);
+  const uint32_t op = (operand_bytes + 1023u) & ~1023u;
+  const uint32_t room = (uint32_t)kSmemLimit - kStaticReserve - 1024u - kHeaderBytes - op;
   p.nstages = (int)(room / stage_bytes);
   if (p.nstages > kMaxStages) p.nstages = kMaxStages;
   p.op_off = p.ring_off + p.nstages * stage_bytes;
-  p.total = p.op_off + ((operand_bytes + 127) & ~127u);
+  p.total = p.op_off + op + 1024u;   // + alignment slack
   return p;
 }
 
-// barriers: full[8], empty[8], opbar, abort word (136 B of the 256 B header)
-__device__ __forceinline__ void ring_setup(unsigned char* smem, const SmemPlan& sp, Ring& ring,
-                                           uint64_t*& opbar, volatile int*& abort_flag) {
+// barriers: full[8], empty[8], opbar, abort word; returns the 1024-B aligned base
+__device__ __forceinline__ unsigned char* ring_setup(unsigned char* smem_raw, const SmemPlan& sp, Ring& ring,
+                                                     uint64_t*& opbar, volatile int*& abort_flag) {
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
   ring.full = bars;
   ring.empty = bars + kMaxStages;
@@ -165,6 +247,7 @@ __device__ __forceinline__ void ring_setup(unsigned char* smem, const SmemPlan& 
     fence_barrier_init();
   }
   __syncthreads();
+  return smem;
 }
 
 // ---------------------------------------------------------------------------
@@ -182,17 +265,22 @@ struct Args {
   const float* s;
   const bf16* W_s_up;
   const bf16* W_s_down;
-  float* r;         // [T][E]
-  uint8_t* act;     // [T][E]
-  float* u;         // [T][d_e]
-  bf16* hs;         // [T][d_s]   SiLU(x W_s_up^T)
-  float* C;         // [T][E][d_e] centred up-projection
-  bf16* A;          // [T][E][d_e] NormSiLU output
-  int* done;        // [E] rows of each expert finished by kd_up
+  float* r;          // [T][E]
+  uint8_t* act;      // [T][E]
+  float* u;          // [T][d_e]
+  bf16* hs;          // [16 tok][hi d_s | lo d_s], chunk-swizzled rows: SiLU(x W_s_up^T)
+  float* C;          // [E][16 tok][d_e] up-projection g = x W_up[e]^T (active experts)
+  bf16* a_cmp;       // [E][16 slots][hi d_e | lo d_e], chunk-swizzled rows: s_e r_e NormSiLU,
+                     // slot i = the i-th active token of expert e (ascending)
+  int* cnt_u;        // [E] finished rows per expert (zero at entry)
   int* err;
   bf16* out;
-  uint32_t down_stage;   // kd_down ring stage bytes (>= one expert's weights + activations)
 };
+
+// physical 16-byte chunk of logical chunk k in a row with index r: the low 3
+// bits are XOR-ed with the row index, so 8 consecutive rows of one logical
+// chunk sit in 8 different bank groups
+__host__ __device__ __forceinline__ int row_chunk(int r, int k) { return (k & ~7) | ((k ^ r) & 7); }
 
 // per-expert token masks and the ascending list of experts some token uses
 __device__ __forceinline__ void build_union(const Args& a, uint16_t* emask, uint8_t* ulist, int* U) {
@@ -218,13 +306,13 @@ __device__ __forceinline__ void build_union(const Args& a, uint16_t* emask, uint
   __syncthreads();
 }
 
-// Reduce N = 2^m per-lane values across the warp in 31-ish shuffles instead of
-// 5 per value: at each of the first m levels a lane keeps one half of its
-// values, sends the other half to its partner and adds what it receives;
-// the remaining 5 - m levels are plain butterflies.  Afterwards lane l holds
-// the warp total of value index (l >> (5 - m)) & (N - 1); every total is a
-// fixed-shape tree over the 32 lane partials (depth 5), so it is
-// deterministic and its rounding is that of a 5-level pairwise sum.
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& q, float (&v)[8]) { unpack16(q, v); }
+
+// Reduce N = 2^m per-lane values across the warp: at each of the first m
+// levels a lane keeps one half of its values, sends the other half to its
+// partner and adds what it receives; the remaining 5 - m levels are plain
+// butterflies.  Afterwards lane l holds the warp total of value index
+// (l >> (5 - m)) & (N - 1), a fixed 5-level tree over the 32 lane partials.
 template <int N>
 __device__ __forceinline__ float warp_reduce_scatter(float (&v)[N], int lane) {
   static_assert(N >= 1 && N <= 32 && (N & (N - 1)) == 0, "N must be a power of two <= 32");
@@ -250,335 +338,397 @@ __device__ __forceinline__ float warp_reduce_scatter(float (&v)[N], int lane) {
   return v[0];
 }
 
-constexpr int kMaxChunks = 16;   // D <= 4096 bf16: D/256 chunks of 8 per lane
-
-// load this lane's chunks (lane + 32 i, 8 bf16 each) of a row in shared memory
-__device__ __forceinline__ void load_row_chunks(const bf16* row, int nc, int lane, uint4 (&w)[kMaxChunks]) {
-#pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i)
-    if (i < nc) w[i] = *reinterpret_cast<const uint4*>(row + (size_t)(lane + 32 * i) * 8);
+// v as a bf16 pair (hi, lo = v - hi) at element j of a chunk-swizzled row of
+// 2L elements (hi part [0, L), lo part [L, 2L)); r is the row index
+__device__ __forceinline__ void store_row_hi_lo(bf16* row, int r, int L, int j, float v) {
+  const bf16 hi = __float2bfloat16_rn(v);
+  const bf16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+  row[row_chunk(r, j >> 3) * 8 + (j & 7)] = hi;
+  row[row_chunk(r, (L + j) >> 3) * 8 + (j & 7)] = lo;
 }
 
-// Partial dot products of one row (chunks in registers) with the token rows of
-// xs[16][D] selected by `tmask`; each lane sums its terms in chunk order.
-template <bool ABS>
-__device__ __forceinline__ void row_token_partials(const uint4 (&w)[kMaxChunks], int nc, const bf16* xs,
-                                                   int D, uint32_t tmask, int lane, float (&acc)[16],
-                                                   float (&aacc)[16]) {
-#pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    acc[t] = 0.f;
-    aacc[t] = 0.f;
-  }
-#pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
-    if (i < nc) {
-      float wv[8];
-      bf16x8_to_f32(w[i], wv);
-#pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        if ((tmask >> t) & 1u) {
-          float xv[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(xs + (size_t)t * D + (size_t)(lane + 32 * i) * 8), xv);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            acc[t] = fmaf(xv[k], wv[k], acc[t]);
-            if (ABS) aacc[t] = fmaf(fabsf(xv[k]), fabsf(wv[k]), aacc[t]);
-          }
-        }
-      }
+// ---------------------------------------------------------------------------
+// Row-range streaming (kd_route, kd_up): a CTA's rows are taken in chunks of
+// `rc` rows (one stage), each row one bulk copy into a padded smem row of
+// pitch D*2 + 16 bytes.  For a chunk, warp w multiplies the 16 token rows of x
+// by the chunk's rows over columns [w*D/8, (w+1)*D/8): one m16n8 tile per
+// 16-column step.  The 8 warps' 16 x 8 results are then added in warp order.
+
+__host__ __device__ inline uint32_t x_pitch(int D) { return (uint32_t)D * 2u + 16u; }
+__host__ __device__ inline int rows_per_chunk(int D) { return D <= 2048 ? 8 : 4; }
+__host__ __device__ inline uint32_t row_stage_bytes(int D) {
+  return ((uint32_t)rows_per_chunk(D) * x_pitch(D) + 1023u) & ~1023u;
+}
+
+__device__ __forceinline__ uint32_t x_addr(uint32_t xs, uint32_t pitch, int lane, int chunk) {
+  return xs + (uint32_t)((lane & 7) + ((lane >> 3) & 1) * 8) * pitch + (uint32_t)(chunk + (lane >> 4)) * 16u;
+}
+// B operand (8 weight rows x 16 columns) from padded rows; rows >= rc (a
+// chunk of fewer rows) repeat row 0, and their outputs are discarded
+__device__ __forceinline__ uint32_t w_addr(uint32_t ws, uint32_t pitch, int lane, int chunk, int rc) {
+  const int r = (lane & 7) < rc ? (lane & 7) : 0;
+  return ws + (uint32_t)r * pitch + (uint32_t)(chunk + ((lane >> 3) & 1)) * 16u;
+}
+
+// issue the T row copies of x into padded rows (one thread)
+__device__ __forceinline__ void stage_x(const Args& a, unsigned char* xs, uint64_t* bar) {
+  const uint32_t pitch = x_pitch(a.D);
+  mbar_expect_tx(bar, (uint32_t)a.T * a.D * 2);
+  for (int t = 0; t < a.T; ++t) bulk_g2s(xs + (size_t)t * pitch, a.x + (size_t)t * a.D, (uint32_t)a.D * 2, bar);
+}
+// zero the rows T..15 of the 16-row x operand (consumer threads)
+__device__ __forceinline__ void zero_x_tail(const Args& a, unsigned char* xs, int tid, int nthreads) {
+  const uint32_t pitch = x_pitch(a.D);
+  const int words = (int)(pitch / 16);
+  for (int i = tid; i < (kTok - a.T) * words; i += nthreads)
+    reinterpret_cast<uint4*>(xs + (size_t)(a.T + i / words) * pitch)[i % words] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// y[16 tok][8 rows] for one chunk; returns in `red_out` (thread o < 128 of the
+// consumer warps gets output o = tok*8 + row)
+__device__ __forceinline__ float chunk_gemv(uint32_t xs, uint32_t ws, uint32_t pitch, int D, int warp, int lane,
+                                            float* red, bool math) {
+  const int rc = rows_per_chunk(D);
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  if (math) {
+    const int c0 = warp * (D / 8) / 8, c1 = c0 + (D / 8) / 8;   // 16-byte chunks of this warp
+    for (int ch = c0; ch < c1; ch += 2) {
+      uint32_t a0, a1, a2, a3, b0, b1;
+      ldsm_x4(x_addr(xs, pitch, lane, ch), a0, a1, a2, a3);
+      ldsm_x2(w_addr(ws, pitch, lane, ch, rc), b0, b1);
+      mma16816(d, a0, a1, a2, a3, b0, b1);
     }
   }
+  // red: [8 warps][16 tok][8 rows]
+  const int tok = lane >> 2, col = 2 * (lane & 3);
+  *reinterpret_cast<float2*>(red + warp * 128 + tok * 8 + col) = make_float2(d[0], d[1]);
+  *reinterpret_cast<float2*>(red + warp * 128 + (tok + 8) * 8 + col) = make_float2(d[2], d[3]);
+  consumer_sync();
+  float v = 0.f;
+  const int o = threadIdx.x;
+  if (o < 128) {
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) v += red[w * 128 + o];
+  }
+  consumer_sync();
+  return v;
 }
 
 // ---------------------------------------------------------------------------
 // kd_route
+//
+// CTAs [0, Cr) with Cr = ceil(E / 8): router rows, 8 per CTA, one warp each,
+// on CUDA cores with an exact sign decision (see common.cuh).  The remaining
+// CTAs split the rows of [W_bar_up ; W_s_up] evenly and write
+// u = x W_bar_up^T and SiLU(x W_s_up^T) (as hi/lo pairs) for them.
 
-__global__ void __launch_bounds__(kThreads, 1) kd_route(Args a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ unsigned long long limbs[kConsumerWarps][kLimbs];   // 1280 B <= kStaticReserve
-  const uint32_t xbytes = (uint32_t)a.T * a.D * 2;
-  const SmemPlan sp = smem_plan(xbytes, kStageBytes);
+__global__ void __launch_bounds__(kThreads, 1) kd_route(const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ unsigned long long limbs[kConsumerWarps][kLimbs];   // 1280 B
+  const int Cr = (a.E + 7) / 8;
+  const bool router_cta = (int)blockIdx.x < Cr;
+  const uint32_t pitch = x_pitch(a.D);
+  // operand: x rows, then the 4 KB cross-warp reduction scratch
+  const SmemPlan sp = smem_plan(kTok * pitch + 4096, router_cta ? kStageBytes : row_stage_bytes(a.D));
   Ring ring;
   uint64_t* xbar;
   volatile int* abort_flag;
-  ring_setup(smem, sp, ring, xbar, abort_flag);
-  const bf16* xs = reinterpret_cast<const bf16*>(smem + sp.op_off);
+  unsigned char* smem = ring_setup(smem_raw, sp, ring, xbar, abort_flag);
+  unsigned char* xsm = smem + sp.op_off;
+  float* red = reinterpret_cast<float*>(xsm + kTok * pitch);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
-  if (blockIdx.x == 0)
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) a.done[e] = 0;
 
-  const int Ntot = a.E + a.d_e + a.d_s;
-  const int Q = (Ntot + gridDim.x - 1) / gridDim.x;
-  const int g0 = min(Ntot, (int)blockIdx.x * Q), g1 = min(Ntot, g0 + Q);
-  const int rowbytes = a.D * 2;
-  const int RPS = min(kConsumerWarps, (int)(kStageBytes / rowbytes));
-  const int WPR = kConsumerWarps / RPS;
-  auto seg_end = [&](int g) { return g < a.E ? a.E : (g < a.E + a.d_e ? a.E + a.d_e : Ntot); };
-  auto row_ptr = [&](int g) -> const bf16* {
-    if (g < a.E) return a.W_r + (size_t)g * a.D;
-    if (g < a.E + a.d_e) return a.W_bar + (size_t)(g - a.E) * a.D;
-    return a.W_s_up + (size_t)(g - a.E - a.d_e) * a.D;
+  if (router_cta) {
+    const int e0 = blockIdx.x * 8, ne = min(8, a.E - e0);
+    const uint32_t rowbytes = (uint32_t)a.D * 2;
+    const int per = (int)(kStageBytes / rowbytes);   // router rows per stage
+    if (warp == kConsumerWarps) {
+      if (lane == 0) {
+        const uint64_t pol = evict_first_policy();
+        stage_x(a, xsm, xbar);
+        for (int k = 0, done = 0; done < ne; ++k) {
+          const int n = min(per, ne - done);
+          mbar_expect_tx(&ring.full[k], n * rowbytes);
+          bulk_g2s(ring.stage + (size_t)k * kStageBytes, a.W_r + (size_t)(e0 + done) * a.D, n * rowbytes,
+                   &ring.full[k], pol);
+          done += n;
+        }
+      }
+      return;
+    }
+    const int nc = a.D / 256;
+    const int n_terms = a.D / 32 + 6;
+    const float gm = gamma_f32(n_terms);
+    const float bscale = 2.f * gm * (1.f + 2.f * gm);
+    const float tiny = float(n_terms) * 2.8025969e-45f;
+    bool bad = false;
+    // every consumer warp waits for x and for the stage of the rows of warp
+    // min(warp, ne - 1), so every issued copy is awaited before the CTA exits
+    const bool x_ok = mbar_wait(xbar, 0, abort_flag, a.err);
+    const int myrow = min(warp, ne - 1);
+    const int k = myrow / per, rs = myrow % per;
+    const bool w_ok = x_ok && mbar_wait(&ring.full[k], 0, abort_flag, a.err);
+    if (w_ok && warp < ne) {
+      const int e = e0 + warp;
+      const bf16* wrow = reinterpret_cast<const bf16*>(ring.stage + (size_t)k * kStageBytes + (size_t)rs * rowbytes);
+      constexpr int kMaxChunks = 16;
+      uint4 w[kMaxChunks];
+#pragma unroll
+      for (int i = 0; i < kMaxChunks; ++i)
+        if (i < nc) w[i] = *reinterpret_cast<const uint4*>(wrow + (size_t)(lane + 32 * i) * 8);
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      // each lane: its D/32 products in chunk order (z in v[t], sum |x w| in v[16+t])
+#pragma unroll
+      for (int i = 0; i < kMaxChunks; ++i) {
+        if (i < nc) {
+          float wv[8];
+          bf16x8_to_f32(w[i], wv);
+#pragma unroll
+          for (int t = 0; t < kTok; ++t) {
+            if (t < a.T) {
+              float xv[8];
+              bf16x8_to_f32(*reinterpret_cast<const uint4*>(xsm + (size_t)t * pitch + (size_t)(lane + 32 * i) * 16),
+                            xv);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                v[t] = fmaf(xv[q], wv[q], v[t]);
+                v[16 + t] = fmaf(fabsf(xv[q]), fabsf(wv[q]), v[16 + t]);
+              }
+            }
+          }
+        }
+      }
+      const float tot = warp_reduce_scatter<32>(v, lane);   // lane l: value l
+      const float S = __shfl_sync(kFull, tot, (lane + 16) & 31);
+      const float b = a.b_r[e];
+      const int t = lane;
+      const bool mine = t < a.T;
+      const float z = tot + b;
+      const float B = bscale * (S + fabsf(b)) + tiny;
+      const bool sure = fabsf(z) > B;
+      bool on = sure && z > 0.f;
+      // guard band: exact re-evaluation of the sign, one whole warp per score
+      unsigned need = __ballot_sync(kFull, mine && !sure);
+      while (need) {
+        const int tt = __ffs(need) - 1;
+        need &= need - 1;
+        const int sg = exact_sign_warp(reinterpret_cast<const bf16*>(xsm + (size_t)tt * pitch), wrow, a.D, b,
+                                       limbs[warp], &bad);
+        if (lane == tt) on = sg > 0;
+      }
+      if (mine) {
+        a.r[(size_t)t * a.E + e] = on ? fmaxf(z, 0.f) : 0.f;
+        a.act[(size_t)t * a.E + e] = on ? 1 : 0;
+      }
+    }
+    if (bad && lane == 0) atomicOr(a.err, 1);
+    return;
+  }
+
+  // rows of [W_bar_up ; W_s_up], split evenly over the remaining CTAs
+  const int nrows = a.d_e + a.d_s;
+  const int G = gridDim.x - Cr, c = blockIdx.x - Cr;
+  const int ra = (int)((long long)c * nrows / G), rb = (int)((long long)(c + 1) * nrows / G);
+  const int rc = rows_per_chunk(a.D);
+  const int nchunks = (rb - ra + rc - 1) / rc;
+  auto row_src = [&](int g) -> const bf16* {
+    return g < a.d_e ? a.W_bar + (size_t)g * a.D : a.W_s_up + (size_t)(g - a.d_e) * a.D;
   };
-
   if (warp == kConsumerWarps) {
-    if (lane == 0 && g0 < g1) {
+    if (lane == 0 && nchunks > 0) {
       const uint64_t pol = evict_first_policy();
-      mbar_expect_tx(xbar, xbytes);
-      bulk_g2s(smem + sp.op_off, a.x, xbytes, xbar);
-      int k = 0;
-      for (int g = g0; g < g1; ++k) {
-        const int n = min(RPS, min(g1, seg_end(g)) - g);
+      stage_x(a, xsm, xbar);
+      for (int k = 0; k < nchunks; ++k) {
         const int s = k % ring.nstages;
         if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
-        mbar_expect_tx(&ring.full[s], n * rowbytes);
-        bulk_g2s(ring.stage + (size_t)s * ring.stage_bytes, row_ptr(g), n * rowbytes, &ring.full[s], pol);
-        g += n;
+        const int g0 = ra + k * rc, n = min(rc, rb - g0);
+        mbar_expect_tx(&ring.full[s], (uint32_t)n * a.D * 2);
+        for (int i = 0; i < n; ++i)
+          bulk_g2s(ring.stage + (size_t)s * ring.stage_bytes + (size_t)i * pitch, row_src(g0 + i),
+                   (uint32_t)a.D * 2, &ring.full[s], pol);
       }
     }
     return;
   }
-
-  const int nc = a.D / 256;
-  const int n_terms = a.D / 32 + 6;
-  const float gm = gamma_f32(n_terms);
-  const float bscale = 2.f * gm * (1.f + 2.f * gm);
-  const float tiny = float(n_terms) * 2.8025969e-45f;
-  const uint32_t all_t = (a.T >= 32) ? 0xffffffffu : ((1u << a.T) - 1u);
-  bool bad = false;
-  // the activation copy is issued iff this CTA has rows; it is always awaited
-  const bool x_ok = g0 < g1 && mbar_wait(xbar, 0, abort_flag, a.err);
-  int k = 0;
-  for (int g = g0; x_ok && g < g1; ++k) {
-    const int n = min(RPS, min(g1, seg_end(g)) - g);
+  if (nchunks == 0) return;
+  zero_x_tail(a, xsm, threadIdx.x, kConsumerWarps * 32);
+  consumer_sync();
+  bool ok = mbar_wait(xbar, 0, abort_flag, a.err);
+  for (int k = 0; k < nchunks; ++k) {
     const int s = k % ring.nstages;
-    if (!mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err)) break;
-    const int rs = warp / WPR, sub = warp % WPR;
-    if (rs < n) {
-      const int row = g + rs;
-      const bf16* wrow =
-          reinterpret_cast<const bf16*>(ring.stage + (size_t)s * ring.stage_bytes + (size_t)rs * rowbytes);
-      uint4 w[kMaxChunks];
-      load_row_chunks(wrow, nc, lane, w);
-      // with two warps per row each takes every other token
-      const uint32_t tm = all_t & (WPR == 1 ? 0xffffffffu : (sub ? 0xaaaaaaaau : 0x55555555u));
-      float acc[16], aacc[16];
-      if (row < a.E) {
-        const int e = row;
-        row_token_partials<true>(w, nc, xs, a.D, tm, lane, acc, aacc);
-        float v[32];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          v[t] = acc[t];
-          v[16 + t] = aacc[t];
-        }
-        const float tot = warp_reduce_scatter<32>(v, lane);   // lane l: value l
-        const float S = __shfl_sync(kFull, tot, (lane + 16) & 31);
-        const float b = a.b_r[e];
-        const int t = lane;
-        const bool mine = t < 16 && ((tm >> t) & 1u);
-        const float z = tot + b;
-        const float B = bscale * (S + fabsf(b)) + tiny;
-        const bool sure = fabsf(z) > B;
-        bool on = sure && z > 0.f;
-        // guard band: exact re-evaluation of the sign, one whole warp per score
-        unsigned need = __ballot_sync(kFull, mine && !sure);
-        while (need) {
-          const int tt = __ffs(need) - 1;
-          need &= need - 1;
-          const int sg = exact_sign_warp(xs + (size_t)tt * a.D, wrow, a.D, b, limbs[warp], &bad);
-          if (lane == tt) on = sg > 0;
-        }
-        if (mine) {
-          a.r[(size_t)t * a.E + e] = on ? fmaxf(z, 0.f) : 0.f;
-          a.act[(size_t)t * a.E + e] = on ? 1 : 0;
-        }
+    ok = ok && mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err);
+    const float v = chunk_gemv(smem_u32(xsm), smem_u32(ring.stage + (size_t)s * ring.stage_bytes), pitch, a.D,
+                               warp, lane, red, ok);
+    if (ok && lane == 0) mbar_arrive(&ring.empty[s]);
+    const int o = threadIdx.x;
+    const int t = o >> 3, i = o & 7;
+    const int g = ra + k * rc + i;
+    if (ok && o < 128 && i < rc && g < rb) {
+      if (g < a.d_e) {
+        if (t < a.T) a.u[(size_t)t * a.d_e + g] = v;
       } else {
-        row_token_partials<false>(w, nc, xs, a.D, tm, lane, acc, aacc);
-        const float tot = warp_reduce_scatter<16>(acc, lane);   // lane l: token l >> 1
-        const int t = lane >> 1;
-        if ((lane & 1) == 0 && ((tm >> t) & 1u)) {
-          if (row < a.E + a.d_e)
-            a.u[(size_t)t * a.d_e + (row - a.E)] = tot;
-          else
-            a.hs[(size_t)t * a.d_s + (row - a.E - a.d_e)] = __float2bfloat16_rn(silu_f(tot));
-        }
+        const int j = g - a.d_e;   // shared hidden unit
+        store_row_hi_lo(a.hs + (size_t)t * 2 * a.d_s, t, a.d_s, j, t < a.T ? silu_f(v) : 0.f);
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&ring.empty[s]);
-    g += n;
   }
-  if (bad && lane == 0) atomicOr(a.err, 1);
 }
 
 // ---------------------------------------------------------------------------
-// kd_up
+// kd_up: the rows of W_up[e] for the active experts e (in union order), split
+// evenly over the CTAs; writes g = x W_up[e]^T; the CTA that completes an
+// expert applies NormSiLU to its active tokens and writes the compact,
+// scaled activations for kd_down.
 
-__global__ void __launch_bounds__(kThreads, 1) kd_up(Args a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  // static shared memory stays within kStaticReserve
+__global__ void __launch_bounds__(kThreads, 1) kd_up(const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint16_t emask[256];
   __shared__ uint8_t ulist[256];
   __shared__ int s_U;
-  __shared__ int touched_e[32], touched_n[32];
-  __shared__ int n_touched, fin[32], n_fin;
-  const uint32_t xbytes = (uint32_t)a.T * a.D * 2;
-  const SmemPlan sp = smem_plan(xbytes, kStageBytes);
+  __shared__ int fin_u[16], n_fin;
+  const uint32_t pitch = x_pitch(a.D);
+  const SmemPlan sp = smem_plan(kTok * pitch + 4096, row_stage_bytes(a.D));
   Ring ring;
   uint64_t* xbar;
   volatile int* abort_flag;
-  ring_setup(smem, sp, ring, xbar, abort_flag);
-  const bf16* xs = reinterpret_cast<const bf16*>(smem + sp.op_off);
+  unsigned char* smem = ring_setup(smem_raw, sp, ring, xbar, abort_flag);
+  unsigned char* xsm = smem + sp.op_off;
+  float* red = reinterpret_cast<float*>(xsm + kTok * pitch);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    n_touched = 0;
-    n_fin = 0;
-    // x does not depend on the router: stage it before waiting for it
-    mbar_expect_tx(xbar, xbytes);
-    bulk_g2s(smem + sp.op_off, a.x, xbytes, xbar);
-  }
-  pdl_wait();          // router outputs (act, u) and the zeroed counters
+  // x does not depend on the router: stage it before waiting for it
+  if (threadIdx.x == 0) stage_x(a, xsm, xbar);
+  if (warp < kConsumerWarps) zero_x_tail(a, xsm, threadIdx.x, kConsumerWarps * 32);
+  pdl_wait();          // router outputs and the completion counters
   pdl_trigger();
   build_union(a, emask, ulist, &s_U);
-  const int U = s_U;
-  const int Ntot = U * a.d_e;
-  const int Q = (Ntot + gridDim.x - 1) / gridDim.x;
-  const int g0 = min(Ntot, (int)blockIdx.x * Q), g1 = min(Ntot, g0 + Q);
-  const int rowbytes = a.D * 2;
-  const int RPS = min(kConsumerWarps, (int)(kStageBytes / rowbytes));
-  const int WPR = kConsumerWarps / RPS;
-
+  const int nrows = s_U * a.d_e;
+  const int c = blockIdx.x, G = gridDim.x;
+  const int ra = (int)((long long)c * nrows / G), rb = (int)((long long)(c + 1) * nrows / G);
+  const int rc = rows_per_chunk(a.D);
+  const int nchunks = (rb - ra + rc - 1) / rc;
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       const uint64_t pol = evict_first_policy();
-      int k = 0;
-      for (int g = g0; g < g1; ++k) {
-        const int e = ulist[g / a.d_e], j = g % a.d_e;
-        const int n = min(RPS, min(g1 - g, a.d_e - j));
+      for (int k = 0; k < nchunks; ++k) {
         const int s = k % ring.nstages;
         if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
-        mbar_expect_tx(&ring.full[s], n * rowbytes);
-        bulk_g2s(ring.stage + (size_t)s * ring.stage_bytes, a.W_up + ((size_t)e * a.d_e + j) * a.D,
-                 n * rowbytes, &ring.full[s], pol);
-        g += n;
+        const int g0 = ra + k * rc, n = min(rc, rb - g0);
+        mbar_expect_tx(&ring.full[s], (uint32_t)n * a.D * 2);
+        for (int i = 0; i < n; ++i) {
+          const int g = g0 + i;
+          bulk_g2s(ring.stage + (size_t)s * ring.stage_bytes + (size_t)i * pitch,
+                   a.W_up + ((size_t)ulist[g / a.d_e] * a.d_e + g % a.d_e) * a.D, (uint32_t)a.D * 2,
+                   &ring.full[s], pol);
+        }
       }
     }
   } else {
-    const int nc = a.D / 256;
-    // the activation copy was issued unconditionally: always await it
-    const bool x_ok = mbar_wait(xbar, 0, abort_flag, a.err);
-    int k = 0;
-    for (int g = g0; x_ok && g < g1; ++k) {
-      const int e = ulist[g / a.d_e], j = g % a.d_e;
-      const int n = min(RPS, min(g1 - g, a.d_e - j));
+    // the x copies were issued unconditionally: always await them
+    bool ok = mbar_wait(xbar, 0, abort_flag, a.err);
+    for (int k = 0; k < nchunks; ++k) {
       const int s = k % ring.nstages;
-      if (threadIdx.x == 0) {
-        if (n_touched > 0 && touched_e[n_touched - 1] == e) {
-          touched_n[n_touched - 1] += n;
-        } else if (n_touched < 32) {
-          touched_e[n_touched] = e;
-          touched_n[n_touched] = n;
-          ++n_touched;
-        }
+      ok = ok && mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err);
+      const float v = chunk_gemv(smem_u32(xsm), smem_u32(ring.stage + (size_t)s * ring.stage_bytes), pitch, a.D,
+                                 warp, lane, red, ok);
+      if (ok && lane == 0) mbar_arrive(&ring.empty[s]);
+      const int o = threadIdx.x;
+      const int t = o >> 3, i = o & 7;
+      const int g = ra + k * rc + i;
+      if (ok && o < 128 && i < rc && g < rb && t < a.T) {
+        const int e = ulist[g / a.d_e];
+        a.C[((size_t)e * kTok + t) * a.d_e + g % a.d_e] = v;
       }
-      if (!mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err)) break;
-      const int rs = warp / WPR, sub = warp % WPR;
-      if (rs < n) {
-        const int jr = j + rs;
-        const bf16* wrow =
-            reinterpret_cast<const bf16*>(ring.stage + (size_t)s * ring.stage_bytes + (size_t)rs * rowbytes);
-        uint4 w[kMaxChunks];
-        load_row_chunks(wrow, nc, lane, w);
-        const uint32_t tm =
-            (uint32_t)emask[e] & (WPR == 1 ? 0xffffffffu : (sub ? 0xaaaaaaaau : 0x55555555u));
-        float acc[16], aacc[16];
-        row_token_partials<false>(w, nc, xs, a.D, tm, lane, acc, aacc);
-        const float tot = warp_reduce_scatter<16>(acc, lane);   // lane l: token l >> 1
-        const int t = lane >> 1;
-        if ((lane & 1) == 0 && ((tm >> t) & 1u)) a.C[((size_t)t * a.E + e) * a.d_e + jr] = tot;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ring.empty[s]);
-      g += n;
     }
   }
-  // publish this CTA's rows; the CTA completing an expert normalises it
+  // publish; the CTA that completes an expert runs its NormSiLU
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0 && !*abort_flag) {
-    for (int i = 0; i < n_touched; ++i) {
-      const int e = touched_e[i];
-      const int old = atomicAdd(a.done + e, touched_n[i]);
-      if (old + touched_n[i] == a.d_e) fin[n_fin++] = e;
+  if (threadIdx.x == 0) {
+    n_fin = 0;
+    if (!*abort_flag) {
+      for (int g = ra; g < rb;) {
+        const int ue = g / a.d_e;
+        const int n = min(rb, (ue + 1) * a.d_e) - g;
+        const int old = atomicAdd(a.cnt_u + ulist[ue], n);
+        if (old + n == a.d_e && n_fin < 16) fin_u[n_fin++] = ue;
+        g += n;
+      }
     }
   }
   __syncthreads();
-  if (warp >= kConsumerWarps) return;
+  if (warp >= kConsumerWarps || n_fin == 0) return;
   __threadfence();
   const float inv_de = 1.f / float(a.d_e);
   int item = 0;
   for (int f = 0; f < n_fin; ++f) {
-    const int e = fin[f];
-    for (uint32_t m = emask[e]; m; m &= m - 1, ++item) {
+    const int e = ulist[fin_u[f]];
+    const float se = a.s[e];
+    int slot = 0;
+    for (uint32_t m = emask[e]; m; m &= m - 1, ++slot, ++item) {
       if (item % kConsumerWarps != warp) continue;
       const int t = __ffs(m) - 1;
-      const float* gr = a.C + ((size_t)t * a.E + e) * a.d_e;
-      const float* ur = a.u + (size_t)t * a.d_e;
-      float cv[16];   // d_e <= 512: 16 per lane
+      float cv[16];   // d_e <= 512: 16 values per lane
       float ss = 0.f;
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const int jj = lane + 32 * q;
+        const int j = lane + 32 * q;
         cv[q] = 0.f;
-        if (jj < a.d_e) {
-          cv[q] = __ldcg(gr + jj) - __ldcg(ur + jj);   // c = g - u
+        if (j < a.d_e) {
+          cv[q] = __ldcg(a.C + ((size_t)e * kTok + t) * a.d_e + j) - __ldcg(a.u + (size_t)t * a.d_e + j);
           ss = fmaf(cv[q], cv[q], ss);
         }
       }
       ss = warp_sum(ss);
       const float rinv = 1.f / sqrtf(ss * inv_de + a.eps);
-      bf16* ao = a.A + ((size_t)t * a.E + e) * a.d_e;
+      const float coef = se * __ldcg(a.r + (size_t)t * a.E + e);
+      bf16* row = a.a_cmp + ((size_t)e * kTok + slot) * 2 * a.d_e;
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const int jj = lane + 32 * q;
-        if (jj < a.d_e) ao[jj] = __float2bfloat16_rn(silu_f(cv[q] * rinv));
+        const int j = lane + 32 * q;
+        if (j < a.d_e) store_row_hi_lo(row, slot, a.d_e, j, coef * silu_f(cv[q] * rinv));
       }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// kd_down
-//
-// The CTA's work is a sequence of units: pieces of W_s_down[n0:n1][:] (the
-// shared expert) and then, for each active expert e in ascending order,
-// [W_down[e][n0:n1][:] | A[t][e][:] for its active tokens t, ascending].
-// Consecutive units are packed greedily into ring stages of a.down_stage
-// bytes; producer and consumers compute the same packing.
+// kd_down: CTA c owns output rows [n0, n1), at most 32.  Its units, packed
+// greedily into 32 KB stages, are the shared expert's row pieces
+// W_s_down[m0:m1][:] and then, per active expert e ascending, the slab
+// W_down[e][n0:n1][:] followed by the expert's compact activation rows.  Unit
+// u is multiplied by consumer warp u % 8: for each 64-column tile the warp
+// re-lays the slab's rows into a swizzled 16 x 64 scratch tile and runs
+// m16n8k16 steps with the weights as A (rows) and the token activations as B.
+// B rows of tokens that do not use the expert point at a zero row, so every
+// warp accumulates token-indexed results in registers; the 8 warps' sums are
+// added in warp order at the end (deterministic).
+
+__host__ __device__ inline int down_rows(int D, int G) { return (D + G - 1) / G; }
 
 struct DownUnits {
   int n0, n1, srows, nshared, nunits;
-  uint32_t wbytes, abytes_row;
 };
 
-__device__ __forceinline__ uint32_t unit_bytes(const Args& a, const DownUnits& du, const uint16_t* emask,
-                                               const uint8_t* ulist, int u) {
+__device__ __forceinline__ uint32_t down_unit_bytes(const Args& a, const DownUnits& du, const uint16_t* emask,
+                                                    const uint8_t* ulist, int u) {
   if (u < du.nshared) {
     const int m0 = du.n0 + u * du.srows, m1 = min(du.n1, m0 + du.srows);
     return (uint32_t)(m1 - m0) * a.d_s * 2;
   }
-  return du.wbytes + __popc(emask[ulist[u - du.nshared]]) * du.abytes_row;
+  const uint32_t w = (uint32_t)(du.n1 - du.n0) * a.d_e * 2;
+  const uint32_t act = (uint32_t)__popc(emask[ulist[u - du.nshared]]) * a.d_e * 4;
+  return ((w + 127u) & ~127u) + act;
 }
 
-// end of the stage that starts at unit u (at least one unit per stage)
-__device__ __forceinline__ int stage_end(const Args& a, const DownUnits& du, const uint16_t* emask,
-                                         const uint8_t* ulist, int u, uint32_t cap) {
-  uint32_t used = unit_bytes(a, du, emask, ulist, u);
+__device__ __forceinline__ int down_stage_end(const Args& a, const DownUnits& du, const uint16_t* emask,
+                                              const uint8_t* ulist, int u, uint32_t cap) {
+  uint32_t used = (down_unit_bytes(a, du, emask, ulist, u) + 127u) & ~127u;
   int v = u + 1;
   while (v < du.nunits) {
-    const uint32_t b = unit_bytes(a, du, emask, ulist, v);
+    const uint32_t b = (down_unit_bytes(a, du, emask, ulist, v) + 127u) & ~127u;
     if (used + b > cap) break;
     used += b;
     ++v;
@@ -586,83 +736,95 @@ __device__ __forceinline__ int stage_end(const Args& a, const DownUnits& du, con
   return v;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) kd_down(Args a) {
-  extern __shared__ __align__(128) unsigned char smem[];
+// re-lay columns [64c, 64c+64) of a row-major slab (nr rows, pitch bytes per
+// row) into a swizzled 16 x 64 tile at `tile`: tile row r takes slab row
+// sr0 + r, or zeros where that is outside [0, nr); one warp
+__device__ __forceinline__ void relayout_tile(const unsigned char* slab, uint32_t pitch, int sr0, int nr, int c,
+                                              unsigned char* tile, int lane) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int r = q * 4 + (lane >> 3), k = lane & 7;
+    const int sr = sr0 + r;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (sr >= 0 && sr < nr) v = *reinterpret_cast<const uint4*>(slab + (size_t)sr * pitch + (size_t)(c * 8 + k) * 16);
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((k ^ (r & 7)) << 4)) = v;
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThreads, 1) kd_down(const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint16_t emask[256];
   __shared__ uint8_t ulist[256];
   __shared__ int s_U;
-  const uint32_t hbytes = (uint32_t)a.T * a.d_s * 2;
-  const uint32_t rbytes = (uint32_t)a.T * a.E * 4;     // r staged next to hs
-  const uint32_t hpad = (hbytes + 127) & ~127u;
-  const SmemPlan sp = smem_plan(hpad + rbytes, a.down_stage);
+  // operand: hs rows (16 x 4 d_s bytes), per-warp scratch tiles (8 x 2 KB),
+  // a zero activation row (4 d_e bytes)
+  const uint32_t hbytes = (uint32_t)kTok * a.d_s * 4;
+  const SmemPlan sp = smem_plan(hbytes + 8 * 2048 + (uint32_t)a.d_e * 4, kStageBytes);
   Ring ring;
   uint64_t* hbar;
   volatile int* abort_flag;
-  ring_setup(smem, sp, ring, hbar, abort_flag);
-  const bf16* hsm = reinterpret_cast<const bf16*>(smem + sp.op_off);
-  float* r_s = reinterpret_cast<float*>(smem + sp.op_off + hpad);
+  unsigned char* smem = ring_setup(smem_raw, sp, ring, hbar, abort_flag);
+  unsigned char* hsm = smem + sp.op_off;
+  unsigned char* scratch = hsm + hbytes;
+  unsigned char* zrow = scratch + 8 * 2048;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < a.d_e / 4; i += blockDim.x) reinterpret_cast<uint4*>(zrow)[i] = make_uint4(0, 0, 0, 0);
   // The router's outputs are complete: this grid starts only after every CTA
   // of kd_up passed its own wait on the router.
   build_union(a, emask, ulist, &s_U);
-  for (int i = threadIdx.x; i < a.T * a.E; i += blockDim.x) r_s[i] = __ldcg(a.r + i);
-  __syncthreads();
   DownUnits du;
   du.n0 = (int)(((long long)blockIdx.x * a.D) / gridDim.x);
   du.n1 = (int)(((long long)(blockIdx.x + 1) * a.D) / gridDim.x);
   const int R = du.n1 - du.n0;
-  du.srows = max(1, (int)(a.down_stage / (a.d_s * 2)));
+  // shared pieces: a power of two >= 8 rows (so a piece never straddles two
+  // 16-row m-tiles), at most one stage
+  du.srows = 8;
+  while (du.srows * 2 * a.d_s * 2 <= (int)kStageBytes && du.srows < 32) du.srows *= 2;
   du.nshared = (R + du.srows - 1) / du.srows;
   du.nunits = du.nshared + s_U;
-  du.wbytes = (uint32_t)R * a.d_e * 2;
-  du.abytes_row = (uint32_t)a.d_e * 2;
-  const int n0 = du.n0, n1 = du.n1;
+  const uint32_t wbytes = (uint32_t)R * a.d_e * 2;
+  const uint32_t wpad = (wbytes + 127u) & ~127u;
 
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       const uint64_t pol = evict_first_policy();
       mbar_expect_tx(hbar, hbytes);
-      bulk_g2s(smem + sp.op_off, a.hs, hbytes, hbar);
-      // weights of stage k; activations are issued separately (after kd_up)
-      auto issue_w = [&](int u0, int u1, int s) {
+      bulk_g2s(hsm, a.hs, hbytes, hbar);
+      auto issue_w = [&](int v0, int v1, int s) {
         unsigned char* st = ring.stage + (size_t)s * ring.stage_bytes;
         uint32_t total = 0;
-        for (int u = u0; u < u1; ++u) total += unit_bytes(a, du, emask, ulist, u);
+        for (int u = v0; u < v1; ++u) total += down_unit_bytes(a, du, emask, ulist, u) - (u < du.nshared ? 0 : wpad - wbytes);
         mbar_expect_tx(&ring.full[s], total);
         uint32_t off = 0;
-        for (int u = u0; u < u1; ++u) {
+        for (int u = v0; u < v1; ++u) {
           if (u < du.nshared) {
-            const int m0 = n0 + u * du.srows, m1 = min(n1, m0 + du.srows);
-            const uint32_t bytes = (uint32_t)(m1 - m0) * a.d_s * 2;
-            bulk_g2s(st + off, a.W_s_down + (size_t)m0 * a.d_s, bytes, &ring.full[s], pol);
+            const int m0 = du.n0 + u * du.srows, m1 = min(du.n1, m0 + du.srows);
+            bulk_g2s(st + off, a.W_s_down + (size_t)m0 * a.d_s, (uint32_t)(m1 - m0) * a.d_s * 2, &ring.full[s], pol);
           } else {
             const int e = ulist[u - du.nshared];
-            bulk_g2s(st + off, a.W_down + ((size_t)e * a.D + n0) * a.d_e, du.wbytes, &ring.full[s], pol);
+            bulk_g2s(st + off, a.W_down + ((size_t)e * a.D + du.n0) * a.d_e, wbytes, &ring.full[s], pol);
           }
-          off += unit_bytes(a, du, emask, ulist, u);
+          off += (down_unit_bytes(a, du, emask, ulist, u) + 127u) & ~127u;
         }
       };
-      auto issue_a = [&](int u0, int u1, int s) {   // activations written by kd_up
+      auto issue_a = [&](int v0, int v1, int s) {   // activations written by kd_up
         unsigned char* st = ring.stage + (size_t)s * ring.stage_bytes;
         uint32_t off = 0;
-        for (int u = u0; u < u1; ++u) {
+        for (int u = v0; u < v1; ++u) {
           if (u >= du.nshared) {
             const int e = ulist[u - du.nshared];
-            int slot = 0;
-            for (uint32_t m = emask[e]; m; m &= m - 1, ++slot) {
-              const int t = __ffs(m) - 1;
-              bulk_g2s(st + off + du.wbytes + (size_t)slot * du.abytes_row,
-                       a.A + ((size_t)t * a.E + e) * a.d_e, du.abytes_row, &ring.full[s]);
-            }
+            const uint32_t n = (uint32_t)__popc(emask[e]) * a.d_e * 4;
+            bulk_g2s(st + off + wpad, a.a_cmp + (size_t)e * kTok * 2 * a.d_e, n, &ring.full[s]);
           }
-          off += unit_bytes(a, du, emask, ulist, u);
+          off += (down_unit_bytes(a, du, emask, ulist, u) + 127u) & ~127u;
         }
       };
       // weights of the first stages go out before kd_up has finished ...
       int u = 0, k = 0;
       int first_u[kMaxStages + 1];
       for (; u < du.nunits && k < ring.nstages; ++k) {
-        const int v = stage_end(a, du, emask, ulist, u, ring.stage_bytes);
+        const int v = down_stage_end(a, du, emask, ulist, u, ring.stage_bytes);
         first_u[k] = u;
         issue_w(u, v, k);
         u = v;
@@ -672,7 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1) kd_down(Args a) {
       // ... their activations only once it has
       for (int q = 0; q < k; ++q) issue_a(first_u[q], first_u[q + 1], q);
       for (; u < du.nunits; ++k) {
-        const int v = stage_end(a, du, emask, ulist, u, ring.stage_bytes);
+        const int v = down_stage_end(a, du, emask, ulist, u, ring.stage_bytes);
         const int s = k % ring.nstages;
         if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
         issue_w(u, v, s);
@@ -683,83 +845,103 @@ __global__ void __launch_bounds__(kThreads, 1) kd_down(Args a) {
     return;
   }
 
-  // consumer warp w owns rows n0 + w + 8q, q < 4; a row pair (q, q+1) and the
-  // 16 token slots make 32 partial sums reduced together, lane l ending with
-  // row (l >> 4) of the pair and token (l & 15)
-  float acc[2] = {0.f, 0.f};
-  const int my_t = lane & 15;
-  const bool ok = mbar_wait(hbar, 0, abort_flag, a.err);
+  // acc[m][n]: rows n0 + 16m .. +16, tokens 8n .. 8n+8 (C fragment layout)
+  float acc[2][2][4] = {};
+  unsigned char* my_tile = scratch + warp * 2048;
+  const uint32_t tile_u32 = smem_u32(my_tile);
+  const int ntiles = (a.T + 7) / 8;
+  bool ok = mbar_wait(hbar, 0, abort_flag, a.err);
   int k = 0;
-  for (int u0 = 0; ok && u0 < du.nunits; ++k) {
-    const int u1 = stage_end(a, du, emask, ulist, u0, ring.stage_bytes);
+  for (int v0 = 0; ok && v0 < du.nunits; ++k) {
+    const int v1 = down_stage_end(a, du, emask, ulist, v0, ring.stage_bytes);
     const int s = k % ring.nstages;
     if (!mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err)) break;
     const unsigned char* st = ring.stage + (size_t)s * ring.stage_bytes;
     uint32_t off = 0;
-    for (int u = u0; u < u1; ++u) {
-      const bool shared = u < du.nshared;
-      const int m0 = shared ? n0 + u * du.srows : n0;
-      const int m1 = shared ? min(n1, m0 + du.srows) : n1;
-      const int K = shared ? a.d_s : a.d_e;
-      const int e = shared ? -1 : ulist[u - du.nshared];
-      const uint32_t tmask = shared ? ((1u << a.T) - 1u) : (uint32_t)emask[e];
-      const bf16* wbase = reinterpret_cast<const bf16*>(st + off);
-      const bf16* act_base = shared ? hsm : reinterpret_cast<const bf16*>(st + off + du.wbytes);
+    for (int u = v0; u < v1; ++u) {
+      if (u % kConsumerWarps == warp) {
+        const bool shared = u < du.nshared;
+        const int m0 = shared ? du.n0 + u * du.srows : du.n0;
+        const int nr = shared ? min(du.n1, m0 + du.srows) - m0 : R;
+        const int K = shared ? a.d_s : a.d_e;
+        const uint32_t pitch = (uint32_t)K * 2;
+        // B rows: token t's activation row (hi part; lo is K columns later)
+        // and the row index its chunks are swizzled with (token or slot)
+        uint32_t brow[2];
+        int bsw[2];
+        uint32_t m_e = 0;
+        if (!shared) m_e = emask[ulist[u - du.nshared]];
 #pragma unroll
-      for (int qp = 0; qp < 2; ++qp) {
-        const int ra = n0 + warp + 16 * qp, rb = ra + 8;   // the pair's two rows
-        const bool has_a = ra >= m0 && ra < m1, has_b = rb >= m0 && rb < m1;
-        if (!(has_a || has_b)) continue;
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-        const bf16* wa = wbase + (size_t)(ra - m0) * K;
-        const bf16* wb = wbase + (size_t)(rb - m0) * K;
-        for (int c = lane; c < K / 8; c += 32) {
-          float fa[8], fb[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) fa[i] = fb[i] = 0.f;
-          if (has_a) bf16x8_to_f32(*reinterpret_cast<const uint4*>(wa + (size_t)c * 8), fa);
-          if (has_b) bf16x8_to_f32(*reinterpret_cast<const uint4*>(wb + (size_t)c * 8), fb);
-          int slot = 0;
-#pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            if ((tmask >> t) & 1u) {
-              const bf16* av = act_base + (size_t)(shared ? t : slot) * K;
-              float hv[8];
-              bf16x8_to_f32(*reinterpret_cast<const uint4*>(av + (size_t)c * 8), hv);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                v[t] = fmaf(fa[i], hv[i], v[t]);
-                v[16 + t] = fmaf(fb[i], hv[i], v[16 + t]);
-              }
-              ++slot;
-            }
+        for (int n = 0; n < 2; ++n) {
+          const int t = 8 * n + (lane & 7);
+          if (shared) {
+            brow[n] = smem_u32(hsm) + (uint32_t)t * 4 * a.d_s;
+            bsw[n] = t;
+          } else {
+            const bool on = t < a.T && ((m_e >> t) & 1u);
+            const int slot = __popc(m_e & ((1u << t) - 1u));
+            brow[n] = on ? smem_u32(st + off + wpad) + (uint32_t)slot * 4 * a.d_e : smem_u32(zrow);
+            bsw[n] = on ? slot : 0;
           }
         }
-        const float tot = warp_reduce_scatter<32>(v, lane);   // lane l: value l
-        const bool mine_row = (lane < 16) ? has_a : has_b;
-        if (mine_row && ((tmask >> my_t) & 1u)) {
-          if (shared)
-            acc[qp] += tot;
-          else
-            acc[qp] = fmaf(a.s[e] * r_s[my_t * a.E + e], tot, acc[qp]);
+        // output rows [rr0, rr0 + nr) relative to n0, in 16-row m-tiles
+        const int rr0 = m0 - du.n0;
+        for (int ms = rr0 / 16; ms <= (rr0 + nr - 1) / 16; ++ms) {
+          for (int c = 0; c < K / kKB; ++c) {
+            relayout_tile(st + off, pitch, 16 * ms - rr0, nr, c, my_tile, lane);
+#pragma unroll
+            for (int ks = 0; ks < kKB / 16; ++ks) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4(a_addr(tile_u32, lane, ks), a0, a1, a2, a3);
+              const int kc = c * 8 + 2 * ks + ((lane >> 3) & 1);   // logical 16-byte chunk of this lane's row
+#pragma unroll
+              for (int n = 0; n < 2; ++n) {
+                if (n < ntiles) {
+                  uint32_t bh0, bh1, bl0, bl1;
+                  ldsm_x2(brow[n] + (uint32_t)row_chunk(bsw[n], kc) * 16u, bh0, bh1);
+                  ldsm_x2(brow[n] + (uint32_t)row_chunk(bsw[n], kc + K / 8) * 16u, bl0, bl1);
+                  if (ms == 0) {
+                    mma16816(acc[0][n], a0, a1, a2, a3, bh0, bh1);
+                    mma16816(acc[0][n], a0, a1, a2, a3, bl0, bl1);
+                  } else {
+                    mma16816(acc[1][n], a0, a1, a2, a3, bh0, bh1);
+                    mma16816(acc[1][n], a0, a1, a2, a3, bl0, bl1);
+                  }
+                }
+              }
+            }
+            __syncwarp();
+          }
         }
       }
-      off += unit_bytes(a, du, emask, ulist, u);
+      off += (down_unit_bytes(a, du, emask, ulist, u) + 127u) & ~127u;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&ring.empty[s]);
-    u0 = u1;
+    v0 = v1;
   }
-  if (my_t < a.T && !*abort_flag) {
+  // add the 8 warps' accumulators in warp order; the scratch reuses stage 0,
+  // whose last copy every consumer warp has awaited
+  consumer_sync();
+  float* red = reinterpret_cast<float*>(ring.stage);   // [8 warps][16 values][32 lanes]
 #pragma unroll
-    for (int qp = 0; qp < 2; ++qp) {
-      const int m = n0 + warp + 16 * qp + (lane >= 16 ? 8 : 0);
-      if (m >= n1) continue;
-      float val = acc[qp];
-      if (a.residual) val += __bfloat162float(a.x[(size_t)my_t * a.D + m]);
-      a.out[(size_t)my_t * a.D + m] = __float2bfloat16_rn(val);
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) red[(warp * 16 + (m * 2 + n) * 4 + i) * 32 + lane] = acc[m][n][i];
+  consumer_sync();
+  if (*abort_flag || !ok) return;
+  for (int o = threadIdx.x; o < 16 * 32; o += kConsumerWarps * 32) {
+    const int q = o / 128, i = (o / 32) % 4, l = o % 32;
+    const int m = q >> 1, n = q & 1;
+    float v = 0.f;
+    for (int w = 0; w < kConsumerWarps; ++w) v += red[(w * 16 + q * 4 + i) * 32 + l];
+    const int row = du.n0 + 16 * m + (l >> 2) + 8 * (i >> 1);
+    const int t = 8 * n + 2 * (l & 3) + (i & 1);
+    if (t < a.T && row < du.n1) {
+      if (a.residual) v += __bfloat162float(a.x[(size_t)t * a.D + row]);
+      a.out[(size_t)t * a.D + row] = __float2bfloat16_rn(v);
     }
   }
 }
