@@ -162,8 +162,12 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then reads the device error word a kernel may have
- * set in `workspace` (0 = none; 1 = a non-finite router operand) and clears
- * it.  Returns DECO_ERR_CUDA if the synchronisation fails. */
+ * set in `workspace` and clears it.  Bits: 1 = a non-finite router operand;
+ * 2 = a kernel gave up waiting for its own data after about a second (a
+ * library fault, not an input property); 4 = on the bf16 prefill path
+ * (T > 16), a routed expert's output s_e r_e W_down[e] a left the fp16 range
+ * (|v| > 65504) in which it is staged before the combine, so the output is
+ * not valid.  0 = none.  Returns DECO_ERR_CUDA if the synchronisation fails. */
 deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
 
 /* Size of the library's built-in device scratch used by

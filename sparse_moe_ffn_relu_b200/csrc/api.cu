@@ -14,6 +14,7 @@
 #include "../../include/deco_moe.h"
 #include "simt_kernels.cuh"
 #include "decode_kernels.cuh"
+#include "prefill_kernels.cuh"
 
 namespace deco {
 namespace {
@@ -26,6 +27,8 @@ struct Plan {
   // decode path (T <= 16)
   size_t hs16, C16, a_cmp, cnt;
   size_t cnt_bytes;
+  // prefill path (bf16, T > 16): routed expert outputs, one bf16 row per pair
+  size_t v_pairs;
   int tile_rows;
   int sms;
 };
@@ -40,6 +43,12 @@ int num_sms() {
 
 // rows of x staged per CTA: 16 when the tile fits in 128 KB of shared memory
 inline int token_tile(int D, int dtype) { return (16 * (size_t)D * elem_size(dtype) <= 131072) ? 16 : 8; }
+
+// The tcgen05 prefill kernels (prefill_kernels.cuh) take bf16 batches of more
+// than 16 tokens whose routed experts fit one 256-column accumulator.
+bool prefill_eligible(const deco_moe_shape_t& s) {
+  return s.dtype == DECO_BF16 && s.T > dec::kMaxT && s.d_e <= pf::kBN;
+}
 
 Plan make_plan(const deco_moe_shape_t& s) {
   Plan p{};
@@ -63,9 +72,10 @@ Plan make_plan(const deco_moe_shape_t& s) {
   p.pair_of = take(P * 4);
   p.tiles = take((P / p.tile_rows + E) * 16);
   p.n_tiles = take(4);
-  p.H = take(P * s.d_e * 4);       // general path: NormSiLU activations
+  p.H = take(P * s.d_e * 4);       // NormSiLU activations (fp32; bf16 on the prefill path)
+  p.sms = num_sms();
+  if (prefill_eligible(s)) p.v_pairs = take(P * s.d_model * 2);
   if (s.T <= dec::kMaxT) {         // decode path buffers (see decode_kernels.cuh)
-    p.sms = num_sms();
     p.hs16 = take((size_t)dec::kTok * s.d_s * 4);         // [16][hi d_s | lo d_s] bf16
     p.C16 = take(E * dec::kTok * s.d_e * 4);               // [E][16][d_e] fp32
     p.a_cmp = take(E * dec::kTok * s.d_e * 4);             // [E][16][hi d_e | lo d_e] bf16
@@ -177,7 +187,7 @@ template <typename T>
 cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
                         unsigned char* ws, const Plan& p, bool with_mean_shared, float* r,
                         uint8_t* act, int* counts, int* offsets, int* perm, int* n_tok,
-                        cudaStream_t st) {
+                        cudaStream_t st, int tile_rows) {
   RouteArgs ra{};
   ra.x = x;
   ra.T = s.T;
@@ -206,7 +216,7 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
   k_scatter<<<s.E, kThreads, 0, st>>>(act, s.T, s.E, counts, offsets, perm,
                                        reinterpret_cast<int*>(ws + p.pair_of),
                                        reinterpret_cast<int4*>(ws + p.tiles),
-                                       reinterpret_cast<int*>(ws + p.n_tiles), p.tile_rows);
+                                       reinterpret_cast<int*>(ws + p.n_tiles), tile_rows);
   prof_mark(5, st);
   return cudaGetLastError();
 }
@@ -304,17 +314,167 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
   return err;
 }
 
+// ---------------------------------------------------------------------------
+// prefill path: bf16, T > 16 (tcgen05 GEMMs, see prefill_kernels.cuh)
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* q = nullptr;
+    cudaDriverEntryPointQueryResult res;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &q, 12000, cudaEnableDefault, &res) ==
+            cudaSuccess &&
+        res == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(q);
+  });
+  return fn;
+}
+
+// Tensor map over a row-major bf16 matrix [rows][cols]: boxes of 64 columns
+// (128 B, one swizzle atom) x box_rows rows, 128-byte swizzle; rows past the
+// end read as zeros.
+cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)pf::kBK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int MODE>
+cudaError_t launch_pf(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2, const pf::Args& a,
+                      int grid, cudaStream_t st) {
+  if (grid <= 0) return cudaSuccess;
+  cudaError_t err = allow_smem(pf::kp_gemm<MODE>, pf::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  pf::kp_gemm<MODE><<<grid, pf::kThreads, pf::kSmemBytes, st>>>(A, B, B2, a);
+  return cudaGetLastError();
+}
+
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w, void* out,
+                        unsigned char* ws, const Plan& p, cudaStream_t st) {
+  float* r = reinterpret_cast<float*>(ws + p.r);
+  uint8_t* act = reinterpret_cast<uint8_t*>(ws + p.act);
+  cudaError_t err = run_routing<bf16>(s, x, w, ws, p, false, r, act, reinterpret_cast<int*>(ws + p.counts),
+                                      reinterpret_cast<int*>(ws + p.offsets), reinterpret_cast<int*>(ws + p.perm),
+                                      reinterpret_cast<int*>(ws + p.n_tok), st, pf::kBM);
+  if (err != cudaSuccess) return err;
+  const int T = s.T, D = s.d_model, E = s.E, d_e = s.d_e, d_s = s.d_s;
+  const uint64_t P = (uint64_t)T * E;
+  pf::Args a{};
+  a.T = T;
+  a.D = D;
+  a.E = E;
+  a.d_e = d_e;
+  a.d_s = d_s;
+  a.eps = s.rms_eps;
+  a.residual = s.residual;
+  a.tiles = reinterpret_cast<const int4*>(ws + p.tiles);
+  a.n_row_tiles = reinterpret_cast<const int*>(ws + p.n_tiles);
+  a.x = static_cast<const bf16*>(x);
+  a.perm = reinterpret_cast<const int*>(ws + p.perm);
+  a.r = r;
+  a.s = w.s;
+  a.pair_of = reinterpret_cast<const int*>(ws + p.pair_of);
+  a.u = reinterpret_cast<float*>(ws + p.u);
+  a.hs = reinterpret_cast<bf16*>(ws + p.hs);
+  a.a_pairs = reinterpret_cast<bf16*>(ws + p.H);
+  a.v_pairs = reinterpret_cast<__half*>(ws + p.v_pairs);
+  a.out = static_cast<bf16*>(out);
+  a.err = reinterpret_cast<int*>(ws + p.err);
+  CUtensorMap mx, mbar, msup, mup, mapr, mdown, mhs, msdown;
+  if ((err = make_map(&mx, x, D, T, pf::kBM)) != cudaSuccess ||
+      (err = make_map(&mbar, w.W_bar_up, D, d_e, pf::kBN)) != cudaSuccess ||
+      (err = make_map(&msup, w.W_s_up, D, d_s, pf::kBN)) != cudaSuccess ||
+      (err = make_map(&mup, w.W_up, D, (uint64_t)E * d_e, pf::kBN)) != cudaSuccess ||
+      (err = make_map(&mapr, a.a_pairs, d_e, P, pf::kBM)) != cudaSuccess ||
+      (err = make_map(&mdown, w.W_down, d_e, (uint64_t)E * D, pf::kBN)) != cudaSuccess ||
+      (err = make_map(&mhs, a.hs, d_s, T, pf::kBM)) != cudaSuccess ||
+      (err = make_map(&msdown, w.W_s_down, d_s, D, pf::kBN)) != cudaSuccess)
+    return err;
+  const int row_tiles_max = (int)std::min<uint64_t>(P / pf::kBM + E, 1u << 30);
+  // u and SiLU(x W_s_up^T)
+  a.K = D;
+  a.nu = cdiv(d_e, pf::kBN);
+  a.n_tiles_n = a.nu + cdiv(d_s, pf::kBN);
+  a.m_tiles = cdiv(T, pf::kBM);
+  prof_mark(10, st);
+  err = launch_pf<pf::kProj>(mx, mbar, msup, a, std::min(a.m_tiles * a.n_tiles_n, p.sms), st);
+  if (err != cudaSuccess) return err;
+  prof_mark(11, st);
+  // routed up-projections with NormSiLU
+  a.bn = d_e;
+  prof_mark(6, st);
+  err = launch_pf<pf::kUp>(mx, mup, mup, a, std::min(row_tiles_max, p.sms), st);
+  if (err != cudaSuccess) return err;
+  prof_mark(7, st);
+  // routed down-projections, one output row per pair
+  a.K = d_e;
+  a.n_tiles_n = cdiv(D, pf::kBN);
+  prof_mark(8, st);
+  err = launch_pf<pf::kDown>(mapr, mdown, mdown, a, p.sms, st);
+  if (err != cudaSuccess) return err;
+  prof_mark(9, st);
+  // shared expert down-projection + combine + residual
+  a.K = d_s;
+  prof_mark(12, st);
+  err = launch_pf<pf::kShared>(mhs, msdown, msdown, a, std::min(a.m_tiles * a.n_tiles_n, p.sms), st);
+  prof_mark(13, st);
+  return err;
+}
+
+// dense FFN y = W2 SiLU(W1 x) on the same kernels (bf16, T > 16)
+cudaError_t run_dense_tc(int T, int D, int d_ff, const void* x, const void* W1, const void* W2, void* out,
+                         unsigned char* ws, cudaStream_t st) {
+  pf::Args a{};
+  a.T = T;
+  a.D = D;
+  a.E = 0;
+  a.d_e = 0;
+  a.d_s = d_ff;
+  a.x = static_cast<const bf16*>(x);
+  a.hs = reinterpret_cast<bf16*>(ws + 256);
+  a.out = static_cast<bf16*>(out);
+  a.err = reinterpret_cast<int*>(ws);
+  CUtensorMap mx, m1, mh, m2;
+  cudaError_t err;
+  if ((err = make_map(&mx, x, D, T, pf::kBM)) != cudaSuccess ||
+      (err = make_map(&m1, W1, D, d_ff, pf::kBN)) != cudaSuccess ||
+      (err = make_map(&mh, a.hs, d_ff, T, pf::kBM)) != cudaSuccess ||
+      (err = make_map(&m2, W2, d_ff, D, pf::kBN)) != cudaSuccess)
+    return err;
+  const int sms = num_sms();
+  a.K = D;
+  a.nu = 0;
+  a.n_tiles_n = cdiv(d_ff, pf::kBN);
+  a.m_tiles = cdiv(T, pf::kBM);
+  err = launch_pf<pf::kProj>(mx, m1, m1, a, std::min(a.m_tiles * a.n_tiles_n, sms), st);
+  if (err != cudaSuccess) return err;
+  a.K = d_ff;
+  a.n_tiles_n = cdiv(D, pf::kBN);
+  return launch_pf<pf::kShared>(mh, m2, m2, a, std::min(a.m_tiles * a.n_tiles_n, sms), st);
+}
+
 template <typename T>
 cudaError_t run_forward(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
                         void* out, unsigned char* ws, const Plan& p, cudaStream_t st) {
   if (s.T <= dec::kMaxT && decode_eligible(s, p.sms)) return run_decode(s, x, w, out, ws, p, st);
+  if (prefill_eligible(s)) return run_prefill(s, x, w, out, ws, p, st);
   float* r = reinterpret_cast<float*>(ws + p.r);
   uint8_t* act = reinterpret_cast<uint8_t*>(ws + p.act);
   int* counts = reinterpret_cast<int*>(ws + p.counts);
   cudaError_t err = run_routing<T>(s, x, w, ws, p, true, r, act, counts,
                                    reinterpret_cast<int*>(ws + p.offsets),
                                    reinterpret_cast<int*>(ws + p.perm),
-                                   reinterpret_cast<int*>(ws + p.n_tok), st);
+                                   reinterpret_cast<int*>(ws + p.n_tok), st, p.tile_rows);
   if (err != cudaSuccess) return err;
   UpArgs ua{};
   ua.x = x;
@@ -431,8 +591,10 @@ deco_status_t deco_moe_routing(const deco_moe_shape_t* shape, const void* x,
   cudaError_t err = cudaMemsetAsync(ws + p.err, 0, 16, cs);
   if (err != cudaSuccess) return cuda_status(err, "routing: clearing the error word");
   err = shape->dtype == DECO_F32
-            ? run_routing<float>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs)
-            : run_routing<bf16>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs);
+            ? run_routing<float>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs,
+                                 p.tile_rows)
+            : run_routing<bf16>(*shape, x, *w, ws, p, false, r, act, counts, offsets, perm, n_tok, cs,
+                                p.tile_rows);
   return cuda_status(err, "routing");
 }
 
@@ -501,6 +663,8 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
   da.out = out;
   da.residual = 0;
   cudaError_t err;
+  if (dtype == DECO_BF16 && T > dec::kMaxT)
+    return cuda_status(run_dense_tc(T, d_model, d_ff, x, W1, W2, out, ws, cs), "dense_ffn");
   const int tt = token_tile(d_model, dtype);
   if (dtype == DECO_F32) {
     err = route_any<float>(ra, tt, cs);

@@ -211,3 +211,37 @@ def test_decode_path_edge_cases(lib, T, ratio):
     out2 = lib.forward(G["x"], G, eps=shape.eps)
     torch.cuda.synchronize()
     assert torch.equal(out, out2)
+
+
+@pytest.mark.parametrize("shape,ratio,residual", [
+    (LayerShape(300, 320, 5, 192, 320, "bf16"), 0.3, False),    # ragged rows, columns and K
+    (LayerShape(129, 256, 3, 256, 64, "bf16"), 1.0, True),      # every pair active, residual
+    (LayerShape(17, 512, 16, 64, 576, "bf16"), 0.2, False),     # smallest prefill batch
+    (LayerShape(600, 1024, 12, 128, 1024, "bf16"), 0.0, False), # no pair active
+])
+def test_prefill_path_shapes(lib, shape, ratio, residual):
+    # bf16, T > 16: the tensor-core prefill kernels
+    L = make_layer(shape, 41, ratio=ratio if ratio > 0 else 0.2)
+    if ratio == 0.0:
+        L["b_r"] = torch.full_like(L["b_r"], -1e4)
+    G = to_gpu(L, lib)
+    out = lib.forward(G["x"], G, eps=shape.eps, residual=residual)
+    torch.cuda.synchronize()
+    ref, z, act = O.layer_forward_tokens(O.to_f64(L["x"]), to_oracle(L, "bf16"), shape.eps)
+    if ratio == 1.0:
+        assert act.all()
+    if residual:
+        ref = ref + O.to_f64(L["x"])
+    check_close(out.double().cpu().numpy(), ref, "bf16", f"prefill {shape} ratio={ratio}")
+    out2 = lib.forward(G["x"], G, eps=shape.eps, residual=residual)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+def test_dense_ffn_tensor_core_path(lib):
+    from synth import make_dense
+    Dn = make_dense(300, 512, 1216, "bf16", 5)      # T > 16, ragged rows and columns
+    out = lib.dense_ffn(Dn["x"].cuda(), Dn["W1"].cuda(), Dn["W2"].cuda())
+    torch.cuda.synchronize()
+    ref = O.dense_ffn(O.to_f64(Dn["x"]), O.to_f64(Dn["W1"]), O.to_f64(Dn["W2"]))
+    check_close(out.double().cpu().numpy(), ref, "bf16", "dense bf16 T=300")
