@@ -443,10 +443,31 @@ def extras(deco, dev, stream, P):
     n_t = act.sum(dim=1).double()
     D, E, de, ds = shape.D, shape.E, shape.d_e, shape.d_s
     flops = float((2 * D * E + 2 * D * de + n_t * 4 * D * de + 4 * D * ds).sum())
+    # per-kernel device time, eager calls with events between the kernels
+    names = deco.PREFILL_KERNELS
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]
+    kt = {k: [] for k in names}
+    with torch.cuda.stream(stream):
+        for e in ev:
+            e.record(stream)
+        deco.set_profiling(ev)
+        for _ in range(6):
+            deco.forward(G["x"], G, out=o, workspace=ws)
+            stream.synchronize()
+            for j, k in enumerate(names):
+                kt[k].append(ev[2 * j].elapsed_time(ev[2 * j + 1]))
+        deco.set_profiling(None)
+    kms = {k: statistics.mean(v[1:]) for k, v in kt.items()}
+    pairs = float(n_t.sum())
+    kflops = {"route": 2.0 * shape.T * D * E, "proj": 2.0 * shape.T * D * (de + ds), "up": 2.0 * pairs * D * de,
+              "down": 2.0 * pairs * de * D, "shared": 2.0 * shape.T * ds * D}
     out["prefill_t4096"] = {"ms": ms, "tokens_per_s": shape.T / (ms / 1e3),
                             "tflops": flops / (ms / 1e3) / 1e12,
                             "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / P["bf16"],
-                            "mean_activation": float(act.float().mean())}
+                            "mean_activation": float(act.float().mean()),
+                            "kernel_ms": {k: round(v, 4) for k, v in kms.items()},
+                            "kernel_tflops": {k: round(f / (kms[k] / 1e3) / 1e12, 1)
+                                              for k, f in kflops.items()}}
     d_ff = ds + E * de
     for T in (16, 4096):
         Dn = make_dense(T, D, d_ff, "bf16", 7)

@@ -204,8 +204,11 @@ def dense_ffn(x, W1, W2, out=None, workspace=None, stream=None) -> torch.Tensor:
     return out
 
 
-# kernels of one forward call, in launch order (deco_moe_set_profiling)
+# timing slots of deco_moe_set_profiling: slot i is bracketed by events 2i and
+# 2i+1.  The decode path (bf16, T <= 16) fills route, up and down; the general
+# path route..down; the prefill path (bf16, T > 16) all eight.
 KERNELS = ("route", "count", "scatter", "up", "down")
+PREFILL_KERNELS = KERNELS + ("proj", "shared", "combine")
 
 
 def set_profiling(events):

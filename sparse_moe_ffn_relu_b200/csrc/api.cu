@@ -27,8 +27,9 @@ struct Plan {
   // decode path (T <= 16)
   size_t hs16, C16, a_cmp, cnt;
   size_t cnt_bytes;
-  // prefill path (bf16, T > 16): routed expert outputs, one bf16 row per pair
-  size_t v_pairs;
+  // bf16, T > 16: ambiguous router pairs; prefill path: routed expert output
+  // rows (one fp16 row per pair) and the shared expert's fp32 output
+  size_t fb, v_pairs, s_out;
   int tile_rows;
   int sms;
 };
@@ -49,6 +50,10 @@ inline int token_tile(int D, int dtype) { return (16 * (size_t)D * elem_size(dty
 bool prefill_eligible(const deco_moe_shape_t& s) {
   return s.dtype == DECO_BF16 && s.T > dec::kMaxT && s.d_e <= pf::kBN;
 }
+
+// bf16 batches of more than 16 tokens are routed by the tiled router
+// (prefill_kernels.cuh), whatever path computes the experts
+bool tiled_router(const deco_moe_shape_t& s) { return s.dtype == DECO_BF16 && s.T > dec::kMaxT; }
 
 Plan make_plan(const deco_moe_shape_t& s) {
   Plan p{};
@@ -74,7 +79,11 @@ Plan make_plan(const deco_moe_shape_t& s) {
   p.n_tiles = take(4);
   p.H = take(P * s.d_e * 4);       // NormSiLU activations (fp32; bf16 on the prefill path)
   p.sms = num_sms();
-  if (prefill_eligible(s)) p.v_pairs = take(P * s.d_model * 2);
+  if (tiled_router(s)) p.fb = take(P * 8);
+  if (prefill_eligible(s)) {
+    p.v_pairs = take(P * s.d_model * 2);
+    p.s_out = take(T * s.d_model * 4);
+  }
   if (s.T <= dec::kMaxT) {         // decode path buffers (see decode_kernels.cuh)
     p.hs16 = take((size_t)dec::kTok * s.d_s * 4);         // [16][hi d_s | lo d_s] bf16
     p.C16 = take(E * dec::kTok * s.d_e * 4);               // [E][16][d_e] fp32
@@ -137,9 +146,15 @@ cudaEvent_t const* g_prof_events = nullptr;
 int g_prof_n = 0;
 
 inline void prof_mark(int idx, cudaStream_t st) {
-  // external: a real event-record node when the call is being graph-captured
-  if (g_prof_events && idx < g_prof_n)
+  if (!g_prof_events || idx >= g_prof_n) return;
+  // while the stream is being graph-captured the record must be external to
+  // become an event-record node; outside a capture that flag is illegal
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
     cudaEventRecordWithFlags(g_prof_events[idx], st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(g_prof_events[idx], st);
 }
 
 // ---------------------------------------------------------------------------
@@ -205,8 +220,27 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
   ra.hs = reinterpret_cast<float*>(ws + p.hs);
   ra.err = reinterpret_cast<int*>(ws + p.err);
   prof_mark(0, st);
-  cudaError_t err = route_any<T>(ra, token_tile(s.d_model, s.dtype), st);
-  if (err != cudaSuccess) return err;
+  cudaError_t err;
+  if (!with_mean_shared && tiled_router(s)) {
+    pf::RouterArgs rt{};
+    rt.x = static_cast<const bf16*>(x);
+    rt.W_r = static_cast<const bf16*>(w.W_r);
+    rt.b_r = w.b_r;
+    rt.T = s.T;
+    rt.D = s.d_model;
+    rt.E = s.E;
+    rt.r = r;
+    rt.act = act;
+    rt.fb = reinterpret_cast<int2*>(ws + p.fb);
+    rt.n_fb = reinterpret_cast<int*>(ws + p.err) + 1;   // zeroed with the error word
+    rt.err = reinterpret_cast<int*>(ws + p.err);
+    pf::k_router<<<dim3((s.T + pf::kRT - 1) / pf::kRT, (s.E + pf::kRE - 1) / pf::kRE), pf::kRThreads, 0, st>>>(rt);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    pf::k_router_exact<<<p.sms, 256, 0, st>>>(rt);
+  } else {
+    err = route_any<T>(ra, token_tile(s.d_model, s.dtype), st);
+  }
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   prof_mark(1, st);
   prof_mark(2, st);
   k_count<<<s.E + (s.T + kThreads - 1) / kThreads, kThreads, 0, st>>>(act, s.T, s.E, counts, n_tok);
@@ -388,6 +422,7 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   a.hs = reinterpret_cast<bf16*>(ws + p.hs);
   a.a_pairs = reinterpret_cast<bf16*>(ws + p.H);
   a.v_pairs = reinterpret_cast<__half*>(ws + p.v_pairs);
+  a.s_out = reinterpret_cast<float*>(ws + p.s_out);
   a.out = static_cast<bf16*>(out);
   a.err = reinterpret_cast<int*>(ws + p.err);
   CUtensorMap mx, mbar, msup, mup, mapr, mdown, mhs, msdown;
@@ -427,8 +462,13 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   a.K = d_s;
   prof_mark(12, st);
   err = launch_pf<pf::kShared>(mhs, msdown, msdown, a, std::min(a.m_tiles * a.n_tiles_n, p.sms), st);
+  if (err != cudaSuccess) return err;
   prof_mark(13, st);
-  return err;
+  // out = shared + routed rows in ascending expert order (+ x)
+  prof_mark(14, st);
+  pf::k_combine<<<T, pf::kCThreads, 0, st>>>(a.s_out, a.v_pairs, a.pair_of, a.x, a.out, D, E, s.residual);
+  prof_mark(15, st);
+  return cudaGetLastError();
 }
 
 // dense FFN y = W2 SiLU(W1 x) on the same kernels (bf16, T > 16)

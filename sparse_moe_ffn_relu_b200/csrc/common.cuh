@@ -1,6 +1,8 @@
 // Device helpers shared by the DECO MoE kernels (sm_100a).
 #pragma once
 
+#include <climits>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -124,31 +126,27 @@ __device__ __forceinline__ void limbs_add_scaled(unsigned long long* limbs, unsi
   limb_add(limbs, i + 2, c >> 32, neg);
 }
 
-// Exact sign (-1, 0, +1) of b + sum_{k<D} x[k] w[k]; called by all 32 lanes of
-// one warp with the same arguments.  `limbs` is this warp's kLimbs-entry shared
-// buffer.  Sets *nonfinite if an operand is Inf/NaN (the result is then 0).
+// Exact sign (-1, 0, +1) of b + sum_{k<D} x[k] w[k] in the full fixed-point
+// integer: the general routine, used when the register window below does not
+// hold every product.  Called by all 32 lanes of one warp with the same
+// arguments; `limbs` is this warp's kLimbs-entry shared buffer.
 template <typename Tx, typename Tw>
-__device__ int exact_sign_warp(const Tx* x, const Tw* w, int D, float b,
-                               unsigned long long* limbs, bool* nonfinite) {
+__device__ int exact_sign_warp_limbs(const Tx* x, const Tw* w, int D, float b,
+                                     unsigned long long* limbs) {
   const int lane = threadIdx.x & 31;
   for (int i = lane; i < kLimbs; i += 32) limbs[i] = 0ull;
   __syncwarp();
-  bool bad = false;
   for (int k = lane; k < D; k += 32) {
     const FpParts px = fp_parts(to_f32(x[k]));
     const FpParts pw = fp_parts(to_f32(w[k]));
-    bad |= !(px.finite && pw.finite);
-    if (px.m && pw.m && px.finite && pw.finite) {
+    if (px.m && pw.m)
       limbs_add_scaled(limbs, (unsigned long long)px.m * pw.m, px.e + pw.e - kLsbExp,
                        px.neg != pw.neg);
-    }
   }
   if (lane == 0) {
     const FpParts pb = fp_parts(b);
-    bad |= !pb.finite;
-    if (pb.m && pb.finite) limbs_add_scaled(limbs, pb.m, pb.e - kLsbExp, pb.neg);
+    if (pb.m) limbs_add_scaled(limbs, pb.m, pb.e - kLsbExp, pb.neg);
   }
-  bad = __any_sync(kFull, bad);
   __syncwarp();
   int sign = 0;
   if (lane == 0) {
@@ -163,11 +161,100 @@ __device__ int exact_sign_warp(const Tx* x, const Tw* w, int D, float b,
   }
   sign = __shfl_sync(kFull, sign, 0);
   __syncwarp();
+  return sign;
+}
+
+// The same sum in a window of kWin 32-bit limbs held in registers.  The
+// window's least significant bit sits at 2^base with base = f_max + 64 -
+// 32 kWin, f_max the largest exponent (of the least significant bit) among
+// the nonzero products and b: a product M 2^f with f >= base occupies bits
+// [f - base, f - base + 47] <= 32 kWin - 17 of the window, and every lane's
+// limb sums stay below 2^43 (at most D/32 + 1 terms below 2^33 each).  Each
+// lane adds its products to its own limbs (no shared memory, no atomics),
+// then the warp adds the limbs lane-wise and propagates carries.  A product
+// below the window (f < base: more than 128 bits under the largest one) sends
+// the sum to exact_sign_warp_limbs.
+constexpr int kWin = 6;
+
+__device__ __forceinline__ void win_add(long long (&L)[kWin], unsigned long long M, int o, bool neg) {
+  const int i = o >> 5, sh = o & 31;
+  const unsigned long long lo = M & 0xffffffffull, hi = M >> 32;
+  const unsigned long long a = lo << sh;   // < 2^63
+  const unsigned long long c = hi << sh;   // < 2^47
+  long long c0 = (long long)(a & 0xffffffffull);
+  long long c1 = (long long)((a >> 32) + (c & 0xffffffffull));
+  long long c2 = (long long)(c >> 32);
+  if (neg) {
+    c0 = -c0;
+    c1 = -c1;
+    c2 = -c2;
+  }
+#pragma unroll
+  for (int j = 0; j < kWin; ++j) L[j] += j == i ? c0 : (j == i + 1 ? c1 : (j == i + 2 ? c2 : 0ll));
+}
+
+// Exact sign (-1, 0, +1) of b + sum_{k<D} x[k] w[k]; called by all 32 lanes of
+// one warp with the same arguments.  `limbs` is this warp's kLimbs-entry
+// shared buffer (used only by the general routine).  Sets *nonfinite if an
+// operand is Inf/NaN (the result is then 0).
+template <typename Tx, typename Tw>
+__device__ int exact_sign_warp(const Tx* x, const Tw* w, int D, float b,
+                               unsigned long long* limbs, bool* nonfinite) {
+  const int lane = threadIdx.x & 31;
+  // pass 1: finiteness and the largest exponent
+  bool bad = false;
+  int fmax = INT_MIN;
+  for (int k = lane; k < D; k += 32) {
+    const FpParts px = fp_parts(to_f32(x[k]));
+    const FpParts pw = fp_parts(to_f32(w[k]));
+    bad |= !(px.finite && pw.finite);
+    if (px.m && pw.m) fmax = max(fmax, px.e + pw.e);
+  }
+  const FpParts pb = fp_parts(b);
+  bad |= !pb.finite;
+  if (pb.m) fmax = max(fmax, pb.e);
+  bad = __any_sync(kFull, bad);
+  fmax = __reduce_max_sync(kFull, fmax);
   if (bad) {
     *nonfinite = true;
     return 0;
   }
-  return sign;
+  if (fmax == INT_MIN) return 0;   // every product and b are zero
+  // pass 2: the window
+  const int base = fmax + 64 - 32 * kWin;
+  long long L[kWin];
+#pragma unroll
+  for (int j = 0; j < kWin; ++j) L[j] = 0;
+  bool below = false;
+  for (int k = lane; k < D; k += 32) {
+    const FpParts px = fp_parts(to_f32(x[k]));
+    const FpParts pw = fp_parts(to_f32(w[k]));
+    if (px.m && pw.m) {
+      const int o = px.e + pw.e - base;
+      if (o < 0) below = true;
+      else win_add(L, (unsigned long long)px.m * pw.m, o, px.neg != pw.neg);
+    }
+  }
+  if (lane == 0 && pb.m) {
+    const int o = pb.e - base;
+    if (o < 0) below = true;
+    else win_add(L, pb.m, o, pb.neg);
+  }
+  if (__any_sync(kFull, below)) return exact_sign_warp_limbs(x, w, D, b, limbs);
+#pragma unroll
+  for (int j = 0; j < kWin; ++j) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L[j] += __shfl_xor_sync(kFull, L[j], o);
+  }
+  long long carry = 0;
+  bool nz = false;
+#pragma unroll
+  for (int j = 0; j < kWin; ++j) {
+    const long long v = L[j] + carry;
+    nz |= (v & 0xffffffffll) != 0;
+    carry = v >> 32;   // arithmetic shift: floor division by 2^32
+  }
+  return carry < 0 ? -1 : ((carry > 0 || nz) ? 1 : 0);
 }
 
 // gamma_n = n u / (1 - n u) with u = 2^-24: the classical bound on the

@@ -17,9 +17,12 @@
 //            NormSiLU: subtract u, RMS over the d_e columns a thread holds,
 //            SiLU, times s_e * r_e            -> a (bf16, one row per pair)
 //   kDown    a rows of expert e x W_down[e]^T  -> v (fp16, one row per pair)
-//   kShared  hs x W_s_down^T, epilogue adds the token's routed rows v in
-//            ascending expert order (fixed order: deterministic) and the
-//            residual                          -> out (bf16)
+//   kShared  hs x W_s_down^T                   -> S (fp32)
+//
+// and two CUDA-core kernels around them: k_router (exact ReLU routing) and
+// k_combine, out = S + the token's routed rows v in ascending expert order
+// (a fixed order: deterministic) + the residual, one CTA per token with
+// coalesced row reads.
 //
 // Tiles are 128 rows x 256 columns x 64-element K blocks (128 B: one 128-byte
 // swizzle atom).  A 4-stage shared-memory ring feeds the tensor core: warp 5
@@ -96,6 +99,7 @@ struct Args {
   bf16* a_pairs;              // [pairs][d_e]
   __half* v_pairs;            // [pairs][D] fp16: 3 more significant bits than bf16
                               // for the only intermediate that is not an MMA operand
+  float* s_out;               // [T][D] shared-expert output (MoE layer; null: kShared writes out)
   bf16* out;                  // [T][D]
   int* err;
 };
@@ -361,22 +365,23 @@ __device__ __forceinline__ void epilogue(const Args& a, const Tile& t, uint32_t 
       if (ok) fin = store_f16x32(dst + col, v) && fin;
     }
     if (!fin) atomicOr(a.err, kErrRange);
-  } else {   // kShared: shared expert + routed rows in ascending expert order + residual
+  } else {   // kShared: the shared expert's output rows
     const int tok = t.arow + i;
     const bool ok = i < t.rows;
-    const int* po = a.pair_of + (size_t)(ok ? tok : 0) * a.E;
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       const int col = t.n0 + c0;
       if (col >= a.D) break;
       float v[32];
       tmem_ld32(trow + c0, v);
       if (!ok) continue;
-      for (int e = 0; e < a.E; ++e) {
-        const int q = __ldg(po + e);
-        if (q >= 0) add_f16x32(v, a.v_pairs + (size_t)q * a.D + col);
+      if (a.s_out) {   // MoE layer: fp32, the combine kernel adds the routed rows
+        float4* dst = reinterpret_cast<float4*>(a.s_out + (size_t)tok * a.D + col);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {         // dense FFN: the output itself
+        if (a.residual) add_bf16x32(v, a.x + (size_t)tok * a.D + col);
+        store_bf16x32(a.out + (size_t)tok * a.D + col, v);
       }
-      if (a.residual) add_bf16x32(v, a.x + (size_t)tok * a.D + col);
-      store_bf16x32(a.out + (size_t)tok * a.D + col, v);
     }
   }
 }
@@ -543,6 +548,280 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Router: z[t][e] = b_r[e] + x_t . W_r[e] on CUDA cores in fp32, with a
+// rigorous bound B on |z - exact| so that the sign, which decides whether e is
+// active for t (ReLU routing, "DECO ...", §2 Router design), is exact: pairs
+// with |z| <= B go to a list that k_router_exact settles with an exact integer
+// accumulation.
+//
+// A CTA computes 32 tokens x 64 experts; two groups of 128 threads take
+// alternate 32-element K chunks, every thread a 4 x 4 block of (token, expert)
+// sums.  Each chunk is summed from zero and then added to the running total,
+// and the two groups' totals are added at the end, so every value goes
+// through at most kRK + D/(2 kRK) + 2 roundings.  The product-magnitude sum S
+// in the bound is replaced by its Cauchy-Schwarz upper bound ||x_t|| ||W_r[e]||,
+// with both norms accumulated from the staged tiles.
+
+constexpr int kRT = 32;          // tokens per CTA
+constexpr int kRE = 64;          // experts per CTA
+constexpr int kRK = 32;          // K chunk
+constexpr int kRThreads = 256;   // two K groups of 128
+
+struct RouterArgs {
+  const bf16* x;
+  const bf16* W_r;
+  const float* b_r;
+  int T, D, E;
+  float* r;          // [T][E]
+  uint8_t* act;      // [T][E]
+  int2* fb;          // ambiguous pairs: {t * E + e, bits of z}
+  int* n_fb;
+  int* err;
+};
+
+__device__ __forceinline__ unsigned long long f2pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(unsigned long long v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+// d = a * b + d on both fp32 halves (each an IEEE fma, round to nearest)
+__device__ __forceinline__ void ffma2(unsigned long long& d, unsigned long long a, unsigned long long b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+
+__global__ void __launch_bounds__(kRThreads) k_router(const RouterArgs a) {
+  __shared__ __align__(16) float2 xs[2][kRK][kRT + 2];   // each x twice: {x, x}
+  __shared__ __align__(16) float ws[2][kRK][kRE + 4];
+  __shared__ float nx_s[2][kRT], nw_s[2][kRE];
+  __shared__ float tot_s[kRT][kRE + 1];
+  const int tid = threadIdx.x, g = tid >> 7, gt = tid & 127;
+  const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
+  // loading: x tile 32 rows x 32 k (one 8-element piece per thread), W tile
+  // 64 rows x 32 k (two pieces per thread)
+  const int xr = gt >> 2, kk = (gt & 3) * 8;
+  const bool xok = t0 + xr < a.T;
+  const bf16* xrow = a.x + (size_t)(xok ? t0 + xr : 0) * a.D;
+  const bool wok0 = e0 + xr < a.E, wok1 = e0 + xr + 32 < a.E;
+  const bf16* wrow0 = a.W_r + (size_t)(wok0 ? e0 + xr : 0) * a.D;
+  const bf16* wrow1 = a.W_r + (size_t)(wok1 ? e0 + xr + 32 : 0) * a.D;
+  float sx = 0.f, sw0 = 0.f, sw1 = 0.f;
+  // computing: tokens ty*4.., experts tx*4..
+  const int ty = gt >> 4, tx = gt & 15;
+  float tot[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tot[i][j] = 0.f;
+  const int iters = (a.D + 2 * kRK - 1) / (2 * kRK);   // the same in both groups (barriers)
+  const uint4 zero4 = make_uint4(0, 0, 0, 0);
+  // global loads run two chunks ahead of the math, in a 2-slot register ring
+  uint4 q[2][3];
+  auto fetch = [&](uint4 (&d)[3], int it) {
+    const int k0 = it * 2 * kRK + g * kRK;
+    const bool live = it < iters && k0 < a.D;
+    d[0] = (live && xok) ? *reinterpret_cast<const uint4*>(xrow + k0 + kk) : zero4;
+    d[1] = (live && wok0) ? *reinterpret_cast<const uint4*>(wrow0 + k0 + kk) : zero4;
+    d[2] = (live && wok1) ? *reinterpret_cast<const uint4*>(wrow1 + k0 + kk) : zero4;
+  };
+  fetch(q[0], 0);
+  fetch(q[1], 1);
+  auto step = [&](uint4 (&d)[3], int it) {
+    const int k0 = it * 2 * kRK + g * kRK;
+    float fx[8], fw0[8], fw1[8];
+    unpack16(d[0], fx);
+    unpack16(d[1], fw0);
+    unpack16(d[2], fw1);
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      xs[g][kk + j][xr] = make_float2(fx[j], fx[j]);
+      ws[g][kk + j][xr] = fw0[j];
+      ws[g][kk + j][xr + 32] = fw1[j];
+      sx = fmaf(fx[j], fx[j], sx);
+      sw0 = fmaf(fw0[j], fw0[j], sw0);
+      sw1 = fmaf(fw1[j], fw1[j], sw1);
+    }
+    __syncthreads();
+    fetch(d, it + 2);
+    if (k0 >= a.D) return;                                // this group is past the end
+    unsigned long long part[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) part[i][0] = part[i][1] = 0ull;
+#pragma unroll 8
+    for (int k = 0; k < kRK; ++k) {
+      const ulonglong2 x01 = *reinterpret_cast<const ulonglong2*>(&xs[g][k][ty * 4]);
+      const ulonglong2 x23 = *reinterpret_cast<const ulonglong2*>(&xs[g][k][ty * 4 + 2]);
+      const ulonglong2 w = *reinterpret_cast<const ulonglong2*>(&ws[g][k][tx * 4]);
+      const unsigned long long xa[4] = {x01.x, x01.y, x23.x, x23.y};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        ffma2(part[i][0], xa[i], w.x);
+        ffma2(part[i][1], xa[i], w.y);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 p0 = f2unpack(part[i][0]), p1 = f2unpack(part[i][1]);
+      tot[i][0] += p0.x;
+      tot[i][1] += p0.y;
+      tot[i][2] += p1.x;
+      tot[i][3] += p1.y;
+    }
+  };
+  for (int it = 0; it < iters; it += 2) {
+    step(q[0], it);
+    if (it + 1 < iters) step(q[1], it + 1);
+  }
+  // squared norms: the 4 threads of a row are adjacent lanes
+  sx += __shfl_xor_sync(kFull, sx, 1);
+  sx += __shfl_xor_sync(kFull, sx, 2);
+  sw0 += __shfl_xor_sync(kFull, sw0, 1);
+  sw0 += __shfl_xor_sync(kFull, sw0, 2);
+  sw1 += __shfl_xor_sync(kFull, sw1, 1);
+  sw1 += __shfl_xor_sync(kFull, sw1, 2);
+  if ((gt & 3) == 0) {
+    nx_s[g][xr] = sx;
+    nw_s[g][xr] = sw0;
+    nw_s[g][xr + 32] = sw1;
+  }
+  if (g == 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tot_s[ty * 4 + i][tx * 4 + j] = tot[i][j];
+  }
+  __syncthreads();
+  if (g == 1) return;
+  const int n = kRK + a.D / (2 * kRK) + 3;
+  const float gm = gamma_f32(n);
+  const float scale = 2.f * gm * (1.f + 2.f * gm);
+  const float tiny = float(n) * 2.8025969e-45f;                   // n * 2^-148
+  const float gD = gamma_f32(a.D);
+  const float sub = float(a.D) * 1.4012985e-45f;                  // D * 2^-149
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int tr = ty * 4 + i, t = t0 + tr;
+    if (t >= a.T) continue;
+    // upper bound of ||x_t||^2 from its fp32 sum (any order: error <= gamma_D)
+    const float nx = (nx_s[0][tr] + nx_s[1][tr] + sub) * (1.f + 3.f * gD);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int er = tx * 4 + j, e = e0 + er;
+      if (e >= a.E) continue;
+      const float nw = (nw_s[0][er] + nw_s[1][er] + sub) * (1.f + 3.f * gD);
+      const float S = sqrtf(nx) * sqrtf(nw) * (1.f + 1e-6f);
+      const float b = a.b_r[e];
+      const float z = (tot[i][j] + tot_s[tr][er]) + b;
+      const float B = scale * (S + fabsf(b)) + tiny;
+      const size_t o = (size_t)t * a.E + e;
+      if (fabsf(z) > B) {
+        a.r[o] = z > 0.f ? z : 0.f;
+        a.act[o] = z > 0.f ? 1 : 0;
+      } else {
+        const int slot = atomicAdd(a.n_fb, 1);
+        a.fb[slot] = make_int2((int)o, __float_as_int(z));   // NaN lands here too
+      }
+    }
+  }
+}
+
+// exact sign of every listed pair: one warp each, integer accumulation
+__global__ void __launch_bounds__(256) k_router_exact(const RouterArgs a) {
+  __shared__ unsigned long long limbs[8][kLimbs];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = *a.n_fb;
+  bool bad = false;
+  for (int i = blockIdx.x * 8 + warp; i < n; i += gridDim.x * 8) {
+    const int2 f = a.fb[i];
+    const int t = f.x / a.E, e = f.x - t * a.E;
+    const float z = __int_as_float(f.y);
+    const int sg = exact_sign_warp(a.x + (size_t)t * a.D, a.W_r + (size_t)e * a.D, a.D, a.b_r[e],
+                                   limbs[warp], &bad);
+    if (lane == 0) {
+      a.r[f.x] = sg > 0 ? fmaxf(z, 0.f) : 0.f;
+      a.act[f.x] = sg > 0 ? 1 : 0;
+    }
+  }
+  if (bad && lane == 0) atomicOr(a.err, 1);
+}
+
+// ---------------------------------------------------------------------------
+// out[t] = S[t] + sum over the token's active experts, ascending, of v[pair]
+// (+ x[t]): one CTA per token, 8 columns per thread, 16-byte coalesced loads.
+
+constexpr int kCThreads = 256;
+
+__global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__ S, const __half* __restrict__ v,
+                                                       const int* __restrict__ pair_of,
+                                                       const bf16* __restrict__ x, bf16* __restrict__ out,
+                                                       int D, int E, int residual) {
+  __shared__ int list[256];
+  __shared__ int n_list;
+  const int t = blockIdx.x, lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {   // the token's pairs in ascending expert order
+    int n = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int q = e < E ? pair_of[(size_t)t * E + e] : -1;
+      const unsigned m = __ballot_sync(kFull, q >= 0);
+      if (q >= 0) list[n + __popc(m & ((1u << lane) - 1u))] = q;
+      n += __popc(m);
+    }
+    if (lane == 0) n_list = n;
+  }
+  __syncthreads();
+  const int n = n_list;
+  for (int c = threadIdx.x * 8; c < D; c += kCThreads * 8) {
+    const float4* sp = reinterpret_cast<const float4*>(S + (size_t)t * D + c);
+    const float4 s0 = sp[0], s1 = sp[1];
+    float acc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    int i = 0;
+    for (; i + 4 <= n; i += 4) {
+      uint4 w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w[j] = __ldg(reinterpret_cast<const uint4*>(v + (size_t)list[i + j] * D + c));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t ws4[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws4[h]));
+          acc[2 * h] += f.x;
+          acc[2 * h + 1] += f.y;
+        }
+      }
+    }
+    for (; i < n; ++i) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(v + (size_t)list[i] * D + c));
+      const uint32_t ws4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws4[h]));
+        acc[2 * h] += f.x;
+        acc[2 * h + 1] += f.y;
+      }
+    }
+    if (residual) {
+      float f[8];
+      unpack16(*reinterpret_cast<const uint4*>(x + (size_t)t * D + c), f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += f[j];
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(out + (size_t)t * D + c) = o;
   }
 }
 

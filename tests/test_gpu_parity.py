@@ -245,3 +245,55 @@ def test_dense_ffn_tensor_core_path(lib):
     torch.cuda.synchronize()
     ref = O.dense_ffn(O.to_f64(Dn["x"]), O.to_f64(Dn["W1"]), O.to_f64(Dn["W2"]))
     check_close(out.double().cpu().numpy(), ref, "bf16", "dense bf16 T=300")
+
+
+@pytest.mark.parametrize("T,dtype", [(40, "bf16"), (300, "bf16"), (8, "bf16"), (40, "f32")])
+def test_routing_exact_on_cancelling_logits(lib, T, dtype):
+    """Router rows 0-2 see logits whose products cancel exactly (features come
+    in equal pairs, the weights in opposite pairs), so the exact logit is the
+    bias: +2^-30 (active), -2^-30 and 0 (inactive).  An fp32 evaluation lands
+    near zero with either sign; the decision must still be exact."""
+    shape = LayerShape(T, 256, 8, 64, 64, dtype)
+    L = make_layer(shape, 51)
+    x = L["x"].float()
+    x[:, 1::2] = x[:, 0::2]
+    W = L["W_r"].float()
+    W[:3, 1::2] = -W[:3, 0::2]
+    L["x"] = x.to(L["x"].dtype)
+    L["W_r"] = W.to(L["W_r"].dtype)
+    L["b_r"][0] = 2.0 ** -30
+    L["b_r"][1] = -(2.0 ** -30)
+    L["b_r"][2] = 0.0
+    G = to_gpu(L, lib)
+    act = _routing_check(lib, shape, L, G)
+    assert act[:, 0].all() and not act[:, 1].any() and not act[:, 2].any()
+    out = lib.forward(G["x"], G, eps=shape.eps)
+    torch.cuda.synchronize()
+    ref = O.layer_forward(O.to_f64(L["x"]), to_oracle(L, dtype), shape.eps)
+    check_close(out.double().cpu().numpy(), ref, dtype, f"cancelling logits T={T} {dtype}")
+
+
+@pytest.mark.parametrize("T,dtype", [(40, "bf16"), (8, "bf16"), (40, "f32")])
+def test_routing_exact_wide_exponent_range(lib, T, dtype):
+    """Even tokens carry two features of 2^120 that cancel in router rows 0-3
+    (rows 0-2 as in the cancelling test, row 3 with weights +1, -1), so the
+    exact logit of those rows is decided by products more than 128 bits below
+    the largest one: the general fixed-point accumulation, not the register
+    window.  Routing only (the other rows' logits are ~2^116)."""
+    shape = LayerShape(T, 256, 8, 64, 64, dtype)
+    L = make_layer(shape, 53)
+    x = L["x"].float()
+    x[:, 1::2] = x[:, 0::2]
+    x[0::2, 0] = 2.0 ** 120
+    x[0::2, 1] = 2.0 ** 120
+    W = L["W_r"].float()
+    W[:3, 1::2] = -W[:3, 0::2]
+    W[3, 0], W[3, 1] = 1.0, -1.0
+    L["x"] = x.to(L["x"].dtype)
+    L["W_r"] = W.to(L["W_r"].dtype)
+    L["b_r"][0] = 2.0 ** -30
+    L["b_r"][1] = -(2.0 ** -30)
+    L["b_r"][2] = 0.0
+    G = to_gpu(L, lib)
+    act = _routing_check(lib, shape, L, G)
+    assert act[:, 0].all() and not act[:, 1].any() and not act[:, 2].any()
