@@ -29,7 +29,7 @@ struct Plan {
   size_t cnt_bytes;
   // bf16, T > 16: ambiguous router pairs; prefill path: routed expert output
   // rows (one fp16 row per pair) and the shared expert's fp32 output
-  size_t fb, v_pairs, s_out;
+  size_t fb, blk, v_pairs, s_out;
   int tile_rows;
   int sms;
 };
@@ -79,7 +79,10 @@ Plan make_plan(const deco_moe_shape_t& s) {
   p.n_tiles = take(4);
   p.H = take(P * s.d_e * 4);       // NormSiLU activations (fp32; bf16 on the prefill path)
   p.sms = num_sms();
-  if (tiled_router(s)) p.fb = take(P * 8);
+  if (tiled_router(s)) {
+    p.fb = take(P * 8);
+    p.blk = take((size_t)((s.T + pf::kTabThreads - 1) / pf::kTabThreads) * E * 4);
+  }
   if (prefill_eligible(s)) {
     p.v_pairs = take(P * s.d_model * 2);
     p.s_out = take(T * s.d_model * 4);
@@ -234,7 +237,9 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
     rt.fb = reinterpret_cast<int2*>(ws + p.fb);
     rt.n_fb = reinterpret_cast<int*>(ws + p.err) + 1;   // zeroed with the error word
     rt.err = reinterpret_cast<int*>(ws + p.err);
-    pf::k_router<<<dim3((s.T + pf::kRT - 1) / pf::kRT, (s.E + pf::kRE - 1) / pf::kRE), pf::kRThreads, 0, st>>>(rt);
+    if ((err = allow_smem(pf::k_router, pf::kRouterSmem)) != cudaSuccess) return err;
+    pf::k_router<<<dim3((s.T + pf::kRT - 1) / pf::kRT, (s.E + pf::kRE - 1) / pf::kRE), pf::kRThreads,
+                   pf::kRouterSmem, st>>>(rt);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     pf::k_router_exact<<<p.sms, 256, 0, st>>>(rt);
   } else {
@@ -242,6 +247,21 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
   }
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   prof_mark(1, st);
+  if (!with_mean_shared && tiled_router(s)) {   // token-block tables
+    const int nb = (s.T + pf::kTabThreads - 1) / pf::kTabThreads;
+    int* blk = reinterpret_cast<int*>(ws + p.blk);
+    prof_mark(2, st);
+    pf::k_tab_count<<<nb, pf::kTabThreads, 0, st>>>(act, s.T, s.E, n_tok, blk);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    prof_mark(3, st);
+    prof_mark(4, st);
+    pf::k_tab_scatter<<<nb, pf::kTabThreads, 0, st>>>(act, s.T, s.E, blk, nb, counts, offsets, perm,
+                                                      reinterpret_cast<int*>(ws + p.pair_of),
+                                                      reinterpret_cast<int4*>(ws + p.tiles),
+                                                      reinterpret_cast<int*>(ws + p.n_tiles), tile_rows);
+    prof_mark(5, st);
+    return cudaGetLastError();
+  }
   prof_mark(2, st);
   k_count<<<s.E + (s.T + kThreads - 1) / kThreads, kThreads, 0, st>>>(act, s.T, s.E, counts, n_tok);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -365,29 +385,31 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Tensor map over a row-major bf16 matrix [rows][cols]: boxes of 64 columns
-// (128 B, one swizzle atom) x box_rows rows, 128-byte swizzle; rows past the
-// end read as zeros.
-cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+// Tensor map over a row-major matrix [rows][cols] of 2- or 4-byte elements:
+// boxes of 128 B of columns (one swizzle atom) x box_rows rows, 128-byte
+// swizzle; loads read zeros past the ends, stores are clipped there.
+cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                     CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
+  const uint64_t esz = type == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4 : 2;
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)pf::kBK, box_rows};
+  const cuuint64_t strides[1] = {cols * esz};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = fn(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int MODE>
-cudaError_t launch_pf(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2, const pf::Args& a,
-                      int grid, cudaStream_t st) {
+cudaError_t launch_pf(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2, const CUtensorMap& O,
+                      const CUtensorMap& O2, const pf::Args& a, int grid, cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
   cudaError_t err = allow_smem(pf::kp_gemm<MODE>, pf::kSmemBytes);
   if (err != cudaSuccess) return err;
-  pf::kp_gemm<MODE><<<grid, pf::kThreads, pf::kSmemBytes, st>>>(A, B, B2, a);
+  pf::kp_gemm<MODE><<<grid, pf::kThreads, pf::kSmemBytes, st>>>(A, B, B2, O, O2, a);
   return cudaGetLastError();
 }
 
@@ -425,7 +447,9 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   a.s_out = reinterpret_cast<float*>(ws + p.s_out);
   a.out = static_cast<bf16*>(out);
   a.err = reinterpret_cast<int*>(ws + p.err);
-  CUtensorMap mx, mbar, msup, mup, mapr, mdown, mhs, msdown;
+  // operand maps (tiles of 128 or 256 rows) and output maps (32-row boxes)
+  CUtensorMap mx, mbar, msup, mup, mapr, mdown, mhs, msdown, ou, ohs, oapr, ov, os;
+  constexpr CUtensorMapDataType F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32, F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   if ((err = make_map(&mx, x, D, T, pf::kBM)) != cudaSuccess ||
       (err = make_map(&mbar, w.W_bar_up, D, d_e, pf::kBN)) != cudaSuccess ||
       (err = make_map(&msup, w.W_s_up, D, d_s, pf::kBN)) != cudaSuccess ||
@@ -433,7 +457,12 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
       (err = make_map(&mapr, a.a_pairs, d_e, P, pf::kBM)) != cudaSuccess ||
       (err = make_map(&mdown, w.W_down, d_e, (uint64_t)E * D, pf::kBN)) != cudaSuccess ||
       (err = make_map(&mhs, a.hs, d_s, T, pf::kBM)) != cudaSuccess ||
-      (err = make_map(&msdown, w.W_s_down, d_s, D, pf::kBN)) != cudaSuccess)
+      (err = make_map(&msdown, w.W_s_down, d_s, D, pf::kBN)) != cudaSuccess ||
+      (err = make_map(&ou, a.u, d_e, T, 32, F32)) != cudaSuccess ||
+      (err = make_map(&ohs, a.hs, d_s, T, 32)) != cudaSuccess ||
+      (err = make_map(&oapr, a.a_pairs, d_e, P, 32)) != cudaSuccess ||
+      (err = make_map(&ov, a.v_pairs, D, P, 32, F16)) != cudaSuccess ||
+      (err = make_map(&os, a.s_out, D, T, 32, F32)) != cudaSuccess)
     return err;
   const int row_tiles_max = (int)std::min<uint64_t>(P / pf::kBM + E, 1u << 30);
   // u and SiLU(x W_s_up^T)
@@ -442,26 +471,26 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   a.n_tiles_n = a.nu + cdiv(d_s, pf::kBN);
   a.m_tiles = cdiv(T, pf::kBM);
   prof_mark(10, st);
-  err = launch_pf<pf::kProj>(mx, mbar, msup, a, std::min(a.m_tiles * a.n_tiles_n, p.sms), st);
+  err = launch_pf<pf::kProj>(mx, mbar, msup, ou, ohs, a, std::min(a.m_tiles * a.n_tiles_n, p.sms), st);
   if (err != cudaSuccess) return err;
   prof_mark(11, st);
   // routed up-projections with NormSiLU
   a.bn = d_e;
   prof_mark(6, st);
-  err = launch_pf<pf::kUp>(mx, mup, mup, a, std::min(row_tiles_max, p.sms), st);
+  err = launch_pf<pf::kUp>(mx, mup, mup, oapr, oapr, a, std::min(row_tiles_max, p.sms), st);
   if (err != cudaSuccess) return err;
   prof_mark(7, st);
   // routed down-projections, one output row per pair
   a.K = d_e;
   a.n_tiles_n = cdiv(D, pf::kBN);
   prof_mark(8, st);
-  err = launch_pf<pf::kDown>(mapr, mdown, mdown, a, p.sms, st);
+  err = launch_pf<pf::kDown>(mapr, mdown, mdown, ov, ov, a, p.sms, st);
   if (err != cudaSuccess) return err;
   prof_mark(9, st);
   // shared expert down-projection + combine + residual
   a.K = d_s;
   prof_mark(12, st);
-  err = launch_pf<pf::kShared>(mhs, msdown, msdown, a, std::min(a.m_tiles * a.n_tiles_n, p.sms), st);
+  err = launch_pf<pf::kShared>(mhs, msdown, msdown, os, os, a, std::min(a.m_tiles * a.n_tiles_n, p.sms), st);
   if (err != cudaSuccess) return err;
   prof_mark(13, st);
   // out = shared + routed rows in ascending expert order (+ x)
@@ -484,23 +513,24 @@ cudaError_t run_dense_tc(int T, int D, int d_ff, const void* x, const void* W1, 
   a.hs = reinterpret_cast<bf16*>(ws + 256);
   a.out = static_cast<bf16*>(out);
   a.err = reinterpret_cast<int*>(ws);
-  CUtensorMap mx, m1, mh, m2;
+  CUtensorMap mx, m1, mh, m2, oh;
   cudaError_t err;
   if ((err = make_map(&mx, x, D, T, pf::kBM)) != cudaSuccess ||
       (err = make_map(&m1, W1, D, d_ff, pf::kBN)) != cudaSuccess ||
       (err = make_map(&mh, a.hs, d_ff, T, pf::kBM)) != cudaSuccess ||
-      (err = make_map(&m2, W2, d_ff, D, pf::kBN)) != cudaSuccess)
+      (err = make_map(&m2, W2, d_ff, D, pf::kBN)) != cudaSuccess ||
+      (err = make_map(&oh, a.hs, d_ff, T, 32)) != cudaSuccess)
     return err;
   const int sms = num_sms();
   a.K = D;
   a.nu = 0;
   a.n_tiles_n = cdiv(d_ff, pf::kBN);
   a.m_tiles = cdiv(T, pf::kBM);
-  err = launch_pf<pf::kProj>(mx, m1, m1, a, std::min(a.m_tiles * a.n_tiles_n, sms), st);
+  err = launch_pf<pf::kProj>(mx, m1, m1, oh, oh, a, std::min(a.m_tiles * a.n_tiles_n, sms), st);
   if (err != cudaSuccess) return err;
   a.K = d_ff;
   a.n_tiles_n = cdiv(D, pf::kBN);
-  return launch_pf<pf::kShared>(mh, m2, m2, a, std::min(a.m_tiles * a.n_tiles_n, sms), st);
+  return launch_pf<pf::kShared>(mh, m2, m2, oh, oh, a, std::min(a.m_tiles * a.n_tiles_n, sms), st);
 }
 
 template <typename T>

@@ -126,6 +126,16 @@ __device__ __forceinline__ void limbs_add_scaled(unsigned long long* limbs, unsi
   limb_add(limbs, i + 2, c >> 32, neg);
 }
 
+// 8 consecutive elements (16-byte aligned) widened to fp32
+__device__ __forceinline__ void load8(const bf16* p, float (&v)[8]) {
+  unpack16(*reinterpret_cast<const uint4*>(p), v);
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 // Exact sign (-1, 0, +1) of b + sum_{k<D} x[k] w[k] in the full fixed-point
 // integer: the general routine, used when the register window below does not
 // hold every product.  Called by all 32 lanes of one warp with the same
@@ -201,14 +211,22 @@ template <typename Tx, typename Tw>
 __device__ int exact_sign_warp(const Tx* x, const Tw* w, int D, float b,
                                unsigned long long* limbs, bool* nonfinite) {
   const int lane = threadIdx.x & 31;
-  // pass 1: finiteness and the largest exponent
+  // pass 1: finiteness and the largest exponent (8 elements per lane per
+  // step, loaded as 16-byte vectors: D is a multiple of 64, rows 16-B aligned)
   bool bad = false;
   int fmax = INT_MIN;
-  for (int k = lane; k < D; k += 32) {
-    const FpParts px = fp_parts(to_f32(x[k]));
-    const FpParts pw = fp_parts(to_f32(w[k]));
-    bad |= !(px.finite && pw.finite);
-    if (px.m && pw.m) fmax = max(fmax, px.e + pw.e);
+#pragma unroll 2
+  for (int k0 = lane * 8; k0 < D; k0 += 256) {
+    float xv[8], wv[8];
+    load8(x + k0, xv);
+    load8(w + k0, wv);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const FpParts px = fp_parts(xv[q]);
+      const FpParts pw = fp_parts(wv[q]);
+      bad |= !(px.finite && pw.finite);
+      if (px.m && pw.m) fmax = max(fmax, px.e + pw.e);
+    }
   }
   const FpParts pb = fp_parts(b);
   bad |= !pb.finite;
@@ -226,13 +244,19 @@ __device__ int exact_sign_warp(const Tx* x, const Tw* w, int D, float b,
 #pragma unroll
   for (int j = 0; j < kWin; ++j) L[j] = 0;
   bool below = false;
-  for (int k = lane; k < D; k += 32) {
-    const FpParts px = fp_parts(to_f32(x[k]));
-    const FpParts pw = fp_parts(to_f32(w[k]));
-    if (px.m && pw.m) {
-      const int o = px.e + pw.e - base;
-      if (o < 0) below = true;
-      else win_add(L, (unsigned long long)px.m * pw.m, o, px.neg != pw.neg);
+  for (int k0 = lane * 8; k0 < D; k0 += 256) {
+    float xv[8], wv[8];
+    load8(x + k0, xv);
+    load8(w + k0, wv);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const FpParts px = fp_parts(xv[q]);
+      const FpParts pw = fp_parts(wv[q]);
+      if (px.m && pw.m) {
+        const int o = px.e + pw.e - base;
+        if (o < 0) below = true;
+        else win_add(L, (unsigned long long)px.m * pw.m, o, px.neg != pw.neg);
+      }
     }
   }
   if (lane == 0 && pb.m) {

@@ -34,7 +34,12 @@
 // finished accumulator to the epilogue.  Warps 0-3 read the accumulator with
 // tcgen05.ld (TMEM lane = tile row = thread), so every thread owns whole rows
 // and the RMS of kUp needs no cross-thread reduction; the epilogue of one tile
-// overlaps the main loop of the next through the second accumulator.
+// overlaps the main loop of the next through the second accumulator.  Results
+// leave through shared memory: each epilogue warp fills 32-row x 128-byte
+// boxes (128-byte swizzle) and stores each with one TMA tensor store, two
+// boxes in flight per warp.  kUp stages the u rows of its tokens through the
+// same boxes with coalesced loads and keeps c = g - u in TMEM between its two
+// passes (sum of squares, then SiLU).
 //
 // Waits are bounded (about 1 s), after which the kernel sets bit 2 of the
 // device error word, drains the copies it issued, frees tensor memory and
@@ -72,8 +77,10 @@ constexpr int kTmaWarp = 5;
 constexpr int kGatherWarp0 = 6;                // warps 6-7 (kUp only)
 constexpr int kGatherThreads = 64;
 constexpr uint32_t kTmemCols = 2 * kBN;
-constexpr uint32_t kBarOffset = kStages * (kABytes + kBBytes);
-constexpr size_t kSmemBytes = 1024 + kBarOffset + 256;   // 1 KB alignment slack + ring + barriers
+constexpr uint32_t kStageOut = 4096;                      // one output box: 32 rows x 128 B
+constexpr uint32_t kEpiOffset = kStages * (kABytes + kBBytes);
+constexpr uint32_t kBarOffset = kEpiOffset + 4 * 2 * kStageOut;   // two boxes per epilogue warp
+constexpr size_t kSmemBytes = 1024 + kBarOffset + 256;   // 1 KB alignment slack + ring + boxes + barriers
 
 enum : int { kProj = 0, kUp = 1, kDown = 2, kShared = 3 };
 constexpr int kErrRange = 4;   // device error bit: a routed expert output outside the fp16 range
@@ -178,6 +185,34 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// 32 consecutive fp32 TMEM columns of this thread's lane <- v
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+      "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
+      "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
+      "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// shared -> global 2-D TMA tensor store of one box at (col, row)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int col, int row) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(col), "r"(row)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N committed store groups may still read shared memory
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// SiLU with the fast exponential and division intrinsics (bf16 results)
+__device__ __forceinline__ float silu_fast(float h) { return __fdividef(h, 1.0f + __expf(-h)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -193,38 +228,6 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
     w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
     w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
     reinterpret_cast<uint4*>(dst)[q] = w;
-  }
-}
-// 32 fp32 values -> 32 fp16 (64 B) at a 16-byte aligned address; returns
-// false if a value is outside the fp16 range (or not finite)
-__device__ __forceinline__ bool store_f16x32(__half* dst, const float (&v)[32]) {
-  bool fin = true;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo = v[8 * q + 2 * j], hi = v[8 * q + 2 * j + 1];
-      fin = fin && fabsf(lo) <= 65504.f && fabsf(hi) <= 65504.f;
-      const __half2 h = __floats2half2_rn(lo, hi);
-      w[j] = *reinterpret_cast<const uint32_t*>(&h);
-    }
-    reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  return fin;
-}
-// v += 32 fp16 at a 16-byte aligned address
-__device__ __forceinline__ void add_f16x32(float (&v)[32], const __half* src) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src) + q);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[j]));
-      v[8 * q + 2 * j] += f.x;
-      v[8 * q + 2 * j + 1] += f.y;
-    }
   }
 }
 // v += 32 bf16 at a 16-byte aligned address
@@ -291,94 +294,219 @@ __device__ __forceinline__ Tile tile_at(const Args& a, int idx) {
 }
 
 // ---------------------------------------------------------------------------
-// epilogues: thread i (0..127) owns tile row i, TMEM lane i; `trow` is the
-// TMEM address of its lane at the accumulator's first column.  tcgen05.ld is
-// warp-collective, so every thread loads; only stores are predicated.
+// epilogue output boxes: 32 rows x 128 B, 16-byte chunk q of row r at
+// r * 128 + (q ^ (r & 7)) * 16 (the 128-byte swizzle of the output tensor maps)
+
+struct Out {
+  uint8_t* stg;      // this warp's two boxes
+  uint32_t stg_s;    // the same, shared-window address
+  int lane;
+  int n;             // boxes stored so far by this warp
+};
+
+__device__ __forceinline__ uint32_t box_off(int r, int q) {
+  return (uint32_t)r * 128u + ((uint32_t)(q ^ (r & 7)) << 4);
+}
+// the next box to fill, once the store that last read it is done
+__device__ __forceinline__ uint8_t* box_begin(Out& o) {
+  if (o.lane == 0 && o.n >= 2) bulk_wait_read<1>();
+  __syncwarp();
+  return o.stg + (o.n & 1) * kStageOut;
+}
+// hand the filled box to the async proxy and store it at (col, row)
+__device__ __forceinline__ void box_store(Out& o, const CUtensorMap* map, int col, int row) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (o.lane == 0) {
+    tma_store_2d(map, o.stg_s + (o.n & 1) * kStageOut, col, row);
+    bulk_commit();
+  }
+  ++o.n;
+}
+__device__ __forceinline__ void box_put_f32(uint8_t* box, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(box + box_off(r, q)) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+// 32 16-bit values: half h of the row
+__device__ __forceinline__ void box_put_16(uint8_t* box, int r, int h, const uint4 (&w)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(box + box_off(r, 4 * h + q)) = w[q];
+}
+__device__ __forceinline__ void pack_bf16x32(const float (&v)[32], uint4 (&w)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    w[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+// fp16; returns false if a value is outside the fp16 range (or not finite)
+__device__ __forceinline__ bool pack_f16x32(const float (&v)[32], uint4 (&w)[4]) {
+  bool fin = true;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = v[8 * q + 2 * j], hi = v[8 * q + 2 * j + 1];
+      fin = fin && fabsf(lo) <= 65504.f && fabsf(hi) <= 65504.f;
+      const __half2 x = __floats2half2_rn(lo, hi);
+      h[j] = *reinterpret_cast<const uint32_t*>(&x);
+    }
+    w[q] = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+  return fin;
+}
+
+// ---------------------------------------------------------------------------
+// epilogues: epilogue warp w (0..3) owns tile rows 32w..32w+31, lane r row
+// 32w + r, which is TMEM lane 32w + r; `trow` is that lane's TMEM address at
+// the accumulator's first column.  tcgen05.ld/st are warp-collective, so every
+// lane executes them; rows past the tile are dropped by the tensor map's
+// bounds (token rows) or written by direct stores of the valid rows only
+// (pair rows, whose next rows belong to another expert).
 
 template <int MODE>
-__device__ __forceinline__ void epilogue(const Args& a, const Tile& t, uint32_t trow, int i) {
+__device__ __forceinline__ void epilogue(const Args& a, const Tile& t, uint32_t trow, int warp, Out& o,
+                                         const CUtensorMap* tmO, const CUtensorMap* tmO2) {
+  const int r = o.lane, i = warp * 32 + r;
+  const int row0 = t.arow + warp * 32;
+  const bool ok = i < t.rows;
+  const bool full_warp = warp * 32 + 32 <= t.rows;
+  if ((MODE == kProj || (MODE == kShared && a.s_out)) && row0 >= a.T) return;   // no row of this warp exists
   if (MODE == kProj) {
-    const int tok = t.arow + i;
-    const bool ok = i < t.rows;
-    const int lim = t.bmap == 0 ? a.d_e : a.d_s;
-    for (int c0 = 0; c0 < kBN; c0 += 32) {
-      if (t.n0 + c0 >= lim) break;                       // uniform across the warp
-      float v[32];
-      tmem_ld32(trow + c0, v);
-      if (!ok) continue;
-      const int col = t.n0 + c0;                         // lim is a multiple of 64: all 32 valid
-      if (t.bmap == 0) {
-        float4* dst = reinterpret_cast<float4*>(a.u + (size_t)tok * a.d_e + col);
+    if (t.bmap == 0) {   // u, fp32: one box per 32 columns
+      for (int c0 = 0; c0 < kBN; c0 += 32) {
+        if (t.n0 + c0 >= a.d_e) break;                   // uniform across the warp
+        float v[32];
+        tmem_ld32(trow + c0, v);
+        uint8_t* box = box_begin(o);
+        box_put_f32(box, r, v);
+        box_store(o, tmO, t.n0 + c0, row0);
+      }
+    } else {             // SiLU(shared up-projection), bf16: one box per 64 columns
+      for (int c0 = 0; c0 < kBN; c0 += 64) {
+        if (t.brow + c0 >= a.d_s) break;                 // d_s is a multiple of 64
+        uint8_t* box = box_begin(o);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      } else {
+        for (int h = 0; h < 2; ++h) {
+          float v[32];
+          tmem_ld32(trow + c0 + 32 * h, v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = silu_f(v[j]);
-        store_bf16x32(a.hs + (size_t)tok * a.d_s + col, v);
+          for (int j = 0; j < 32; ++j) v[j] = silu_fast(v[j]);
+          uint4 w[4];
+          pack_bf16x32(v, w);
+          box_put_16(box, r, h, w);
+        }
+        box_store(o, tmO2, t.brow + c0, row0);
       }
     }
   } else if (MODE == kUp) {
-    const bool ok = i < t.rows;
     const int pair = t.arow + i;
     const int tok = ok ? a.perm[pair] : 0;
     const float coef = ok ? a.s[t.e] * a.r[(size_t)tok * a.E + t.e] : 0.f;
-    const float* ur = a.u + (size_t)tok * a.d_e;
+    // pass 1: c = g - u back into TMEM, sum of c^2.  The warp stages its 32
+    // rows' u through the two boxes, 32 columns (128 B per row) at a time: lane
+    // l loads 16 B of rows 4j + l/8 (j < 8), column chunk l % 8.
+    if (o.lane == 0) bulk_wait_read<0>();                // earlier stores done reading the boxes
+    __syncwarp();
+    int tk[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tk[j] = __shfl_sync(kFull, tok, 4 * j + (r >> 3));
+    const int cq = r & 7;
+    float4 q[8];
+    auto u_load = [&](int c0) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        q[j] = __ldg(reinterpret_cast<const float4*>(a.u + (size_t)tk[j] * a.d_e + c0) + cq);
+    };
+    auto u_put = [&](uint8_t* buf) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) *reinterpret_cast<float4*>(buf + box_off(4 * j + (r >> 3), cq)) = q[j];
+    };
+    const int nc = a.d_e / 32;
+    u_load(0);
+    u_put(o.stg);
+    __syncwarp();
     float ss = 0.f;
-    for (int c0 = 0; c0 < a.d_e; c0 += 32) {
+    for (int c = 0; c < nc; ++c) {
+      if (c + 1 < nc) u_load((c + 1) * 32);
       float v[32];
-      tmem_ld32(trow + c0, v);
+      tmem_ld32(trow + c * 32, v);
+      const uint8_t* ub = o.stg + (c & 1) * kStageOut;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 uq = __ldg(reinterpret_cast<const float4*>(ur + c0) + q);
-        const float c_0 = v[4 * q] - uq.x, c_1 = v[4 * q + 1] - uq.y;
-        const float c_2 = v[4 * q + 2] - uq.z, c_3 = v[4 * q + 3] - uq.w;
-        ss = fmaf(c_0, c_0, ss);
-        ss = fmaf(c_1, c_1, ss);
-        ss = fmaf(c_2, c_2, ss);
-        ss = fmaf(c_3, c_3, ss);
+      for (int qq = 0; qq < 8; ++qq) {
+        const float4 uq = *reinterpret_cast<const float4*>(ub + box_off(r, qq));
+        v[4 * qq] -= uq.x;
+        v[4 * qq + 1] -= uq.y;
+        v[4 * qq + 2] -= uq.z;
+        v[4 * qq + 3] -= uq.w;
       }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+      tmem_st32(trow + c * 32, v);
+      if (c + 1 < nc) u_put(o.stg + ((c + 1) & 1) * kStageOut);
+      __syncwarp();
     }
+    tmem_wait_st();
     const float inv = rsqrtf(ss / (float)a.d_e + a.eps);
+    // pass 2: a = SiLU(c / rms) * s_e * r_e, bf16, 64 columns per box
     bf16* dst = a.a_pairs + (size_t)pair * a.d_e;
-    for (int c0 = 0; c0 < a.d_e; c0 += 32) {
-      float v[32];
-      tmem_ld32(trow + c0, v);
+    for (int c0 = 0; c0 < a.d_e; c0 += 64) {
+      uint8_t* box = full_warp ? box_begin(o) : nullptr;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 uq = __ldg(reinterpret_cast<const float4*>(ur + c0) + q);
-        v[4 * q] = silu_f((v[4 * q] - uq.x) * inv) * coef;
-        v[4 * q + 1] = silu_f((v[4 * q + 1] - uq.y) * inv) * coef;
-        v[4 * q + 2] = silu_f((v[4 * q + 2] - uq.z) * inv) * coef;
-        v[4 * q + 3] = silu_f((v[4 * q + 3] - uq.w) * inv) * coef;
+      for (int h = 0; h < 2; ++h) {
+        float v[32];
+        tmem_ld32(trow + c0 + 32 * h, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = silu_fast(v[j] * inv) * coef;
+        uint4 w[4];
+        pack_bf16x32(v, w);
+        if (full_warp) {
+          box_put_16(box, r, h, w);
+        } else if (ok) {
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) reinterpret_cast<uint4*>(dst + c0 + 32 * h)[qq] = w[qq];
+        }
       }
-      if (ok) store_bf16x32(dst + c0, v);
+      if (full_warp) box_store(o, tmO, c0, row0);
     }
   } else if (MODE == kDown) {
-    const bool ok = i < t.rows;
     __half* dst = a.v_pairs + (size_t)(t.arow + i) * a.D;
     bool fin = true;
-    for (int c0 = 0; c0 < kBN; c0 += 32) {
+    for (int c0 = 0; c0 < kBN; c0 += 64) {
       const int col = t.n0 + c0;
       if (col >= a.D) break;                             // D is a multiple of 64
-      float v[32];
-      tmem_ld32(trow + c0, v);
-      if (ok) fin = store_f16x32(dst + col, v) && fin;
+      uint8_t* box = full_warp ? box_begin(o) : nullptr;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float v[32];
+        tmem_ld32(trow + c0 + 32 * h, v);
+        uint4 w[4];
+        const bool f = pack_f16x32(v, w);
+        if (full_warp) {
+          box_put_16(box, r, h, w);
+          fin = fin && f;
+        } else if (ok) {
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) reinterpret_cast<uint4*>(dst + col + 32 * h)[qq] = w[qq];
+          fin = fin && f;
+        }
+      }
+      if (full_warp) box_store(o, tmO, col, row0);
     }
     if (!fin) atomicOr(a.err, kErrRange);
   } else {   // kShared: the shared expert's output rows
     const int tok = t.arow + i;
-    const bool ok = i < t.rows;
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       const int col = t.n0 + c0;
       if (col >= a.D) break;
       float v[32];
       tmem_ld32(trow + c0, v);
-      if (!ok) continue;
-      if (a.s_out) {   // MoE layer: fp32, the combine kernel adds the routed rows
-        float4* dst = reinterpret_cast<float4*>(a.s_out + (size_t)tok * a.D + col);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      } else {         // dense FFN: the output itself
+      if (a.s_out) {   // MoE layer: fp32 boxes; the combine kernel adds the routed rows
+        uint8_t* box = box_begin(o);
+        box_put_f32(box, r, v);
+        box_store(o, tmO, col, row0);
+      } else if (ok) { // dense FFN: the output itself
         if (a.residual) add_bf16x32(v, a.x + (size_t)tok * a.D + col);
         store_bf16x32(a.out + (size_t)tok * a.D + col, v);
       }
@@ -391,7 +519,8 @@ __device__ __forceinline__ void epilogue(const Args& a, const Tile& t, uint32_t 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     kp_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const __grid_constant__ CUtensorMap tmB2, const Args a) {
+            const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmO,
+            const __grid_constant__ CUtensorMap tmO2, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;          // 128-byte swizzle needs 1 KB alignment
@@ -532,16 +661,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp < 4) {
+    Out o;
+    o.stg = sm + kEpiOffset + warp * 2 * kStageOut;
+    o.stg_s = base + kEpiOffset + warp * 2 * kStageOut;
+    o.lane = lane;
+    o.n = 0;
     int lt = 0;
     for (int idx = blockIdx.x; idx < total; idx += gridDim.x, ++lt) {
       const int b = lt & 1;
       if (!mbar_wait(&accf[b], (lt >> 1) & 1, abort_flag, a.err)) break;
       tc_fence_after();
       const Tile t = tile_at<MODE>(a, idx);
-      epilogue<MODE>(a, t, tmem + ((uint32_t)(warp * 32) << 16) + b * kBN, threadIdx.x);
+      epilogue<MODE>(a, t, tmem + ((uint32_t)(warp * 32) << 16) + b * kBN, warp, o, &tmO, &tmO2);
       tc_fence_before();
       mbar_arrive(&acce[b]);
     }
+    if (lane == 0) bulk_wait_all();   // every output store has landed
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -558,18 +694,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 // with |z| <= B go to a list that k_router_exact settles with an exact integer
 // accumulation.
 //
-// A CTA computes 32 tokens x 64 experts; two groups of 128 threads take
-// alternate 32-element K chunks, every thread a 4 x 4 block of (token, expert)
-// sums.  Each chunk is summed from zero and then added to the running total,
-// and the two groups' totals are added at the end, so every value goes
-// through at most kRK + D/(2 kRK) + 2 roundings.  The product-magnitude sum S
-// in the bound is replaced by its Cauchy-Schwarz upper bound ||x_t|| ||W_r[e]||,
-// with both norms accumulated from the staged tiles.
+// A CTA computes 32 tokens x 64 experts with 8 warps; warp g takes the
+// 16-element K chunks g, g+8, g+16, ... through its own shared-memory slice
+// (no block barrier in the main loop), each lane an 8 x 8 block of (token,
+// expert) sums.  Each chunk is summed from zero and added to the warp's running
+// total; the 8 warp totals are added in warp order at the end, so every value
+// goes through at most kRK + D/(8 kRK) + 8 roundings before the bias.  The
+// product-magnitude sum S in the bound is replaced by its Cauchy-Schwarz upper
+// bound ||x_t|| ||W_r[e]||, the norms accumulated from the staged tiles.
 
 constexpr int kRT = 32;          // tokens per CTA
 constexpr int kRE = 64;          // experts per CTA
-constexpr int kRK = 32;          // K chunk
-constexpr int kRThreads = 256;   // two K groups of 128
+constexpr int kRK = 16;          // K chunk
+constexpr int kRWarps = 8;
+constexpr int kRThreads = kRWarps * 32;
+constexpr size_t kRouterSmem =   // staging (aliased by the warp totals) + norms
+    (size_t)kRWarps * kRT * kRE * 4 + (size_t)kRWarps * (kRT + kRE) * 4;
 
 struct RouterArgs {
   const bf16* x;
@@ -598,138 +738,139 @@ __device__ __forceinline__ void ffma2(unsigned long long& d, unsigned long long 
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
 }
 
-__global__ void __launch_bounds__(kRThreads) k_router(const RouterArgs a) {
-  __shared__ __align__(16) float2 xs[2][kRK][kRT + 2];   // each x twice: {x, x}
-  __shared__ __align__(16) float ws[2][kRK][kRE + 4];
-  __shared__ float nx_s[2][kRT], nw_s[2][kRE];
-  __shared__ float tot_s[kRT][kRE + 1];
-  const int tid = threadIdx.x, g = tid >> 7, gt = tid & 127;
+__global__ void __launch_bounds__(kRThreads, 1) k_router(const RouterArgs a) {
+  extern __shared__ __align__(16) float rsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
-  // loading: x tile 32 rows x 32 k (one 8-element piece per thread), W tile
-  // 64 rows x 32 k (two pieces per thread)
-  const int xr = gt >> 2, kk = (gt & 3) * 8;
-  const bool xok = t0 + xr < a.T;
-  const bf16* xrow = a.x + (size_t)(xok ? t0 + xr : 0) * a.D;
-  const bool wok0 = e0 + xr < a.E, wok1 = e0 + xr + 32 < a.E;
-  const bf16* wrow0 = a.W_r + (size_t)(wok0 ? e0 + xr : 0) * a.D;
-  const bf16* wrow1 = a.W_r + (size_t)(wok1 ? e0 + xr + 32 : 0) * a.D;
+  // this warp's staging slice: xs[kRK][kRT], ws[kRK][kRE]
+  float* xs = rsm + (size_t)warp * kRK * (kRT + kRE);
+  float* ws = xs + kRK * kRT;
+  float* nx_w = rsm + (size_t)kRWarps * kRT * kRE + warp * (kRT + kRE);   // [kRT] then [kRE]
+  float* nw_w = nx_w + kRT;
+  // loading: lane = token row lane and expert rows lane, lane + 32; 16 k each
+  const bool xok = t0 + lane < a.T;
+  const bool wok0 = e0 + lane < a.E, wok1 = e0 + lane + 32 < a.E;
+  const bf16* xrow = a.x + (size_t)(xok ? t0 + lane : 0) * a.D;
+  const bf16* wrow0 = a.W_r + (size_t)(wok0 ? e0 + lane : 0) * a.D;
+  const bf16* wrow1 = a.W_r + (size_t)(wok1 ? e0 + lane + 32 : 0) * a.D;
   float sx = 0.f, sw0 = 0.f, sw1 = 0.f;
-  // computing: tokens ty*4.., experts tx*4..
-  const int ty = gt >> 4, tx = gt & 15;
-  float tot[4][4];
+  // computing: tokens ty*8 + i, experts tx*4 + {0..3} and 32 + tx*4 + {0..3}
+  const int ty = lane >> 3, tx = lane & 7;
+  unsigned long long tot[8][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tot[i][j] = 0.f;
-  const int iters = (a.D + 2 * kRK - 1) / (2 * kRK);   // the same in both groups (barriers)
+    for (int j = 0; j < 4; ++j) tot[i][j] = 0ull;
+  const int nchunks = a.D / kRK;
   const uint4 zero4 = make_uint4(0, 0, 0, 0);
-  // global loads run two chunks ahead of the math, in a 2-slot register ring
-  uint4 q[2][3];
-  auto fetch = [&](uint4 (&d)[3], int it) {
-    const int k0 = it * 2 * kRK + g * kRK;
-    const bool live = it < iters && k0 < a.D;
-    d[0] = (live && xok) ? *reinterpret_cast<const uint4*>(xrow + k0 + kk) : zero4;
-    d[1] = (live && wok0) ? *reinterpret_cast<const uint4*>(wrow0 + k0 + kk) : zero4;
-    d[2] = (live && wok1) ? *reinterpret_cast<const uint4*>(wrow1 + k0 + kk) : zero4;
-  };
-  fetch(q[0], 0);
-  fetch(q[1], 1);
-  auto step = [&](uint4 (&d)[3], int it) {
-    const int k0 = it * 2 * kRK + g * kRK;
-    float fx[8], fw0[8], fw1[8];
-    unpack16(d[0], fx);
-    unpack16(d[1], fw0);
-    unpack16(d[2], fw1);
-    __syncthreads();
+  uint4 q[6];   // next chunk: x (2), W rows (2 + 2)
+  auto fetch = [&](int c) {
+    const bool live = c < nchunks;
+    const int k0 = c * kRK;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      xs[g][kk + j][xr] = make_float2(fx[j], fx[j]);
-      ws[g][kk + j][xr] = fw0[j];
-      ws[g][kk + j][xr + 32] = fw1[j];
-      sx = fmaf(fx[j], fx[j], sx);
-      sw0 = fmaf(fw0[j], fw0[j], sw0);
-      sw1 = fmaf(fw1[j], fw1[j], sw1);
+    for (int h = 0; h < 2; ++h) {
+      q[h] = (live && xok) ? *reinterpret_cast<const uint4*>(xrow + k0 + 8 * h) : zero4;
+      q[2 + h] = (live && wok0) ? *reinterpret_cast<const uint4*>(wrow0 + k0 + 8 * h) : zero4;
+      q[4 + h] = (live && wok1) ? *reinterpret_cast<const uint4*>(wrow1 + k0 + 8 * h) : zero4;
     }
-    __syncthreads();
-    fetch(d, it + 2);
-    if (k0 >= a.D) return;                                // this group is past the end
-    unsigned long long part[4][2];
+  };
+  fetch(warp);
+  for (int c = warp; c < nchunks; c += kRWarps) {
+    float fx[16], fw0[16], fw1[16];
+    unpack16(q[0], *reinterpret_cast<float(*)[8]>(fx));
+    unpack16(q[1], *reinterpret_cast<float(*)[8]>(fx + 8));
+    unpack16(q[2], *reinterpret_cast<float(*)[8]>(fw0));
+    unpack16(q[3], *reinterpret_cast<float(*)[8]>(fw0 + 8));
+    unpack16(q[4], *reinterpret_cast<float(*)[8]>(fw1));
+    unpack16(q[5], *reinterpret_cast<float(*)[8]>(fw1 + 8));
+    __syncwarp();   // the previous chunk's reads are done
 #pragma unroll
-    for (int i = 0; i < 4; ++i) part[i][0] = part[i][1] = 0ull;
-#pragma unroll 8
     for (int k = 0; k < kRK; ++k) {
-      const ulonglong2 x01 = *reinterpret_cast<const ulonglong2*>(&xs[g][k][ty * 4]);
-      const ulonglong2 x23 = *reinterpret_cast<const ulonglong2*>(&xs[g][k][ty * 4 + 2]);
-      const ulonglong2 w = *reinterpret_cast<const ulonglong2*>(&ws[g][k][tx * 4]);
-      const unsigned long long xa[4] = {x01.x, x01.y, x23.x, x23.y};
+      xs[k * kRT + lane] = fx[k];
+      ws[k * kRE + lane] = fw0[k];
+      ws[k * kRE + lane + 32] = fw1[k];
+      sx = fmaf(fx[k], fx[k], sx);
+      sw0 = fmaf(fw0[k], fw0[k], sw0);
+      sw1 = fmaf(fw1[k], fw1[k], sw1);
+    }
+    __syncwarp();
+    fetch(c + kRWarps);
+    unsigned long long part[8][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        ffma2(part[i][0], xa[i], w.x);
-        ffma2(part[i][1], xa[i], w.y);
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0ull;
+#pragma unroll 4
+    for (int k = 0; k < kRK; ++k) {
+      const float4 xa = *reinterpret_cast<const float4*>(xs + k * kRT + ty * 8);
+      const float4 xb = *reinterpret_cast<const float4*>(xs + k * kRT + ty * 8 + 4);
+      const ulonglong2 wa = *reinterpret_cast<const ulonglong2*>(ws + k * kRE + tx * 4);
+      const ulonglong2 wb = *reinterpret_cast<const ulonglong2*>(ws + k * kRE + 32 + tx * 4);
+      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const unsigned long long xx = f2pack(xv[i], xv[i]);
+        ffma2(part[i][0], xx, wa.x);
+        ffma2(part[i][1], xx, wa.y);
+        ffma2(part[i][2], xx, wb.x);
+        ffma2(part[i][3], xx, wb.y);
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 p0 = f2unpack(part[i][0]), p1 = f2unpack(part[i][1]);
-      tot[i][0] += p0.x;
-      tot[i][1] += p0.y;
-      tot[i][2] += p1.x;
-      tot[i][3] += p1.y;
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 p = f2unpack(part[i][j]), t = f2unpack(tot[i][j]);
+        tot[i][j] = f2pack(t.x + p.x, t.y + p.y);
+      }
+  }
+  nx_w[lane] = sx;
+  nw_w[lane] = sw0;
+  nw_w[lane + 32] = sw1;
+  __syncthreads();   // every warp is past its staging slice
+  // warp totals: red[warp][t][e]
+  float* red = rsm + (size_t)warp * kRT * kRE;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 t = f2unpack(tot[i][j]);
+      const int e = (j < 2 ? tx * 4 : 32 + tx * 4) + 2 * (j & 1);
+      red[(ty * 8 + i) * kRE + e] = t.x;
+      red[(ty * 8 + i) * kRE + e + 1] = t.y;
     }
-  };
-  for (int it = 0; it < iters; it += 2) {
-    step(q[0], it);
-    if (it + 1 < iters) step(q[1], it + 1);
-  }
-  // squared norms: the 4 threads of a row are adjacent lanes
-  sx += __shfl_xor_sync(kFull, sx, 1);
-  sx += __shfl_xor_sync(kFull, sx, 2);
-  sw0 += __shfl_xor_sync(kFull, sw0, 1);
-  sw0 += __shfl_xor_sync(kFull, sw0, 2);
-  sw1 += __shfl_xor_sync(kFull, sw1, 1);
-  sw1 += __shfl_xor_sync(kFull, sw1, 2);
-  if ((gt & 3) == 0) {
-    nx_s[g][xr] = sx;
-    nw_s[g][xr] = sw0;
-    nw_s[g][xr + 32] = sw1;
-  }
-  if (g == 1) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) tot_s[ty * 4 + i][tx * 4 + j] = tot[i][j];
-  }
   __syncthreads();
-  if (g == 1) return;
-  const int n = kRK + a.D / (2 * kRK) + 3;
+  const int n = kRK + a.D / (kRWarps * kRK) + kRWarps + 3;
   const float gm = gamma_f32(n);
   const float scale = 2.f * gm * (1.f + 2.f * gm);
   const float tiny = float(n) * 2.8025969e-45f;                   // n * 2^-148
   const float gD = gamma_f32(a.D);
   const float sub = float(a.D) * 1.4012985e-45f;                  // D * 2^-149
+  const float* nrm = rsm + (size_t)kRWarps * kRT * kRE;
+  for (int p = threadIdx.x; p < kRT * kRE; p += kRThreads) {
+    const int tr = p / kRE, er = p - tr * kRE;
+    const int t = t0 + tr, e = e0 + er;
+    if (t >= a.T || e >= a.E) continue;
+    float zt = 0.f, nx = 0.f, nw = 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int tr = ty * 4 + i, t = t0 + tr;
-    if (t >= a.T) continue;
-    // upper bound of ||x_t||^2 from its fp32 sum (any order: error <= gamma_D)
-    const float nx = (nx_s[0][tr] + nx_s[1][tr] + sub) * (1.f + 3.f * gD);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int er = tx * 4 + j, e = e0 + er;
-      if (e >= a.E) continue;
-      const float nw = (nw_s[0][er] + nw_s[1][er] + sub) * (1.f + 3.f * gD);
-      const float S = sqrtf(nx) * sqrtf(nw) * (1.f + 1e-6f);
-      const float b = a.b_r[e];
-      const float z = (tot[i][j] + tot_s[tr][er]) + b;
-      const float B = scale * (S + fabsf(b)) + tiny;
-      const size_t o = (size_t)t * a.E + e;
-      if (fabsf(z) > B) {
-        a.r[o] = z > 0.f ? z : 0.f;
-        a.act[o] = z > 0.f ? 1 : 0;
-      } else {
-        const int slot = atomicAdd(a.n_fb, 1);
-        a.fb[slot] = make_int2((int)o, __float_as_int(z));   // NaN lands here too
-      }
+    for (int w = 0; w < kRWarps; ++w) {
+      zt += rsm[(size_t)w * kRT * kRE + p];
+      nx += nrm[w * (kRT + kRE) + tr];
+      nw += nrm[w * (kRT + kRE) + kRT + er];
+    }
+    // upper bounds of the squared norms from their fp32 sums (any order: error
+    // <= gamma_D), then S <= ||x_t|| ||W_r[e]||
+    const float S = sqrtf((nx + sub) * (1.f + 3.f * gD)) * sqrtf((nw + sub) * (1.f + 3.f * gD)) * (1.f + 1e-6f);
+    const float b = a.b_r[e];
+    const float z = zt + b;
+    const float B = scale * (S + fabsf(b)) + tiny;
+    const size_t o = (size_t)t * a.E + e;
+    if (fabsf(z) > B) {
+      a.r[o] = z > 0.f ? z : 0.f;
+      a.act[o] = z > 0.f ? 1 : 0;
+    } else {
+      const int slot = atomicAdd(a.n_fb, 1);
+      a.fb[slot] = make_int2((int)o, __float_as_int(z));   // NaN lands here too
     }
   }
 }
@@ -822,6 +963,143 @@ __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__
     o.z = pack_bf16x2(acc[4], acc[5]);
     o.w = pack_bf16x2(acc[6], acc[7]);
     *reinterpret_cast<uint4*>(out + (size_t)t * D + c) = o;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Token -> expert tables for large batches: a stable counting sort of the
+// active (token, expert) pairs by expert, tokens ascending within an expert.
+// The tokens are cut into blocks of 256; k_tab_count counts each block's
+// pairs per expert (and every token's pair count), k_tab_scatter gives every
+// block its first position per expert and places its pairs, warps in order
+// and lanes in order inside a warp.  Block 0 also writes counts, offsets and
+// the list of row tiles (<= tile_rows pairs of one expert each).
+
+constexpr int kTabThreads = 256;
+constexpr int kTabWarps = kTabThreads / 32;
+
+__global__ void __launch_bounds__(kTabThreads) k_tab_count(const uint8_t* __restrict__ act, int T, int E,
+                                                           int* __restrict__ n_tok, int* __restrict__ blk_counts) {
+  __shared__ int wc[kTabWarps][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTabThreads + threadIdx.x;
+  const bool ok = t < T;
+  const uint8_t* row = act + (size_t)(ok ? t : 0) * E;
+  int n = 0;
+  for (int e = 0; e < E; ++e) {
+    const bool f = ok && row[e];
+    const unsigned m = __ballot_sync(kFull, f);
+    if (lane == 0) wc[warp][e] = __popc(m);
+    n += f;
+  }
+  if (ok) n_tok[t] = n;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kTabThreads) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kTabWarps; ++w) c += wc[w][e];
+    blk_counts[(size_t)blockIdx.x * E + e] = c;
+  }
+}
+
+// exclusive prefix sum of v[0..n) (n <= 256) by one warp, in place; returns the total
+__device__ __forceinline__ int warp_exclusive_scan(int* v, int n) {
+  const int lane = threadIdx.x & 31;
+  int loc[8], sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane * 8 + i;
+    loc[i] = e < n ? v[e] : 0;
+    sum += loc[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - sum;
+  const int total = __shfl_sync(kFull, incl, 31);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane * 8 + i;
+    if (e < n) v[e] = run;
+    run += loc[i];
+  }
+  return total;
+}
+
+__global__ void __launch_bounds__(kTabThreads) k_tab_scatter(const uint8_t* __restrict__ act, int T, int E,
+                                                             const int* __restrict__ blk_counts, int nb,
+                                                             int* counts, int* offsets, int* perm, int* pair_of,
+                                                             int4* tiles, int* n_tiles, int tile_rows) {
+  __shared__ int cnt[256], off[256], base[256], ntl[256];
+  __shared__ int wc[kTabWarps][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // every block: counts per expert and the number of pairs in earlier blocks
+  for (int e = threadIdx.x; e < E; e += kTabThreads) {
+    int c = 0, before = 0;
+    for (int b = 0; b < nb; ++b) {
+      const int v = blk_counts[(size_t)b * E + e];
+      c += v;
+      if (b < (int)blockIdx.x) before += v;
+    }
+    cnt[e] = c;
+    off[e] = c;
+    base[e] = before;
+    ntl[e] = (c + tile_rows - 1) / tile_rows;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int P = warp_exclusive_scan(off, E);
+    if (blockIdx.x == 0 && lane == 0) offsets[E] = P;
+  } else if (warp == 1 && blockIdx.x == 0) {
+    const int nt = warp_exclusive_scan(ntl, E);
+    if (lane == 0) *n_tiles = nt;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < E; e += kTabThreads) {
+      counts[e] = cnt[e];
+      offsets[e] = off[e];
+    }
+    // row tiles: expert e's tiles start at ntl[e] (now its exclusive prefix)
+    for (int e = warp; e < E; e += kTabWarps) {
+      const int n = (cnt[e] + tile_rows - 1) / tile_rows;
+      for (int j = lane; j < n; j += 32)
+        tiles[ntl[e] + j] = make_int4(e, off[e] + j * tile_rows, min(tile_rows, cnt[e] - j * tile_rows), 0);
+    }
+  }
+  // this block's tokens: per-warp counts per expert, then positions
+  const int t = blockIdx.x * kTabThreads + threadIdx.x;
+  const bool ok = t < T;
+  const uint8_t* row = act + (size_t)(ok ? t : 0) * E;
+  for (int e = 0; e < E; ++e) {
+    const unsigned m = __ballot_sync(kFull, ok && row[e]);
+    if (lane == 0) wc[warp][e] = __popc(m);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kTabThreads) {
+    int run = off[e] + base[e];
+#pragma unroll
+    for (int w = 0; w < kTabWarps; ++w) {
+      const int v = wc[w][e];
+      wc[w][e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int e = 0; e < E; ++e) {
+    const bool f = ok && row[e];
+    const unsigned m = __ballot_sync(kFull, f);
+    if (f) {
+      const int pos = wc[warp][e] + __popc(m & lt);
+      perm[pos] = t;
+      pair_of[(size_t)t * E + e] = pos;
+    } else if (ok) {
+      pair_of[(size_t)t * E + e] = -1;
+    }
   }
 }
 
