@@ -37,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 DECODE_TS = (1, 4, 16)
+DECODE_KERNELS = ("route", "up", "down")     # the decode path's launches per forward
 METRIC = "MoE-layer tokens/s (decode)"
 
 
@@ -249,22 +250,14 @@ def main():
             step(G)
         graphs.append(g)
 
-    # instrumented graphs: events around every kernel of every forward
+    # events around every kernel of every forward (eager calls: the library
+    # records them with cudaEventRecord between its launches; PDL is off then)
     nk = len(deco.KERNELS)
     ev = {T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for T in DECODE_TS}
     for es in ev.values():          # torch creates CUDA events lazily, on first record
         for e in es:
             e.record(stream)
     torch.cuda.synchronize()
-    igraphs = []
-    for G in copies:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for T in DECODE_TS:
-                deco.set_profiling(ev[T])
-                deco.forward(xs[T], G, out=outs[T], workspace=wss[T], eps=base.eps)
-            deco.set_profiling(None)
-        igraphs.append(g)
 
     sampler = ClockSampler(local)
     with torch.cuda.stream(stream):
@@ -298,12 +291,18 @@ def main():
     tokens_per_step = sum(DECODE_TS)
     value = world * tokens_per_step * args.steps / (ms / 1000.0)
 
-    # live kernel durations from the instrumented graphs (one replay at a time)
+    # live kernel durations: eager forwards on the rotating weight copies
     kt = {T: {k: [] for k in deco.KERNELS} for T in DECODE_TS}
     with torch.cuda.stream(stream):
-        for i in range(min(args.steps, 60)):
-            igraphs[i % n_copies].replay()
+        for i in range(min(args.steps, 60) + 3):
+            G = copies[i % n_copies]
+            for T in DECODE_TS:
+                deco.set_profiling(ev[T])
+                deco.forward(xs[T], G, out=outs[T], workspace=wss[T], eps=base.eps)
+                deco.set_profiling(None)
             stream.synchronize()
+            if i < 3:
+                continue
             for T in DECODE_TS:
                 for j, k in enumerate(deco.KERNELS):
                     kt[T][k].append(ev[T][2 * j].elapsed_time(ev[T][2 * j + 1]))
@@ -317,7 +316,7 @@ def main():
     bytes_k = {T: layer_bytes(LayerShape(T, base.D, base.E, base.d_e, base.d_s, base.dtype), union[T])
                for T in DECODE_TS}
     mean_ms = {T: {k: statistics.mean(v) for k, v in kt[T].items()} for T in DECODE_TS}
-    tot_k = {k: sum(mean_ms[T][k] for T in DECODE_TS) for k in deco.KERNELS}
+    tot_k = {k: sum(mean_ms[T][k] for T in DECODE_TS) for k in DECODE_KERNELS}
     dom = max(tot_k, key=tot_k.get)
     dom_bytes = sum(bytes_k[T][dom] for T in DECODE_TS) / len(DECODE_TS)
     dom_ms = tot_k[dom] / len(DECODE_TS)
@@ -370,10 +369,11 @@ def main():
                      "unit": "GB/s", "frac": achieved / P["hbm"], "traffic": None,
                      "peak_source": P["src"], "layer_achieved_gbs": layer_gbs,
                      "layer_frac": layer_gbs / P["hbm"],
-                     "kernel_ms": {k: round(v / len(DECODE_TS), 5) for k, v in tot_k.items()}},
+                     "kernel_ms_by_T": {str(T): {k: round(mean_ms[T][k], 4) for k in DECODE_KERNELS}
+                                        for T in DECODE_TS}},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
                 "d2h_bytes_per_step": io_bytes},
-        "gpu_launches": args.steps * len(DECODE_TS) * nk,
+        "gpu_launches": args.steps * len(DECODE_TS) * len(DECODE_KERNELS),
         "clocks": clocks,
     }
     if rank == 0 and world == 1:
@@ -385,7 +385,7 @@ def main():
             line["extras"] = extras(deco, dev, stream, P)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for g in graphs + igraphs:
+    for g in graphs:
         del g
     if dist is not None:
         dist.destroy_process_group()
@@ -461,7 +461,12 @@ def extras(deco, dev, stream, P):
     pairs = float(n_t.sum())
     kflops = {"route": 2.0 * shape.T * D * E, "proj": 2.0 * shape.T * D * (de + ds), "up": 2.0 * pairs * D * de,
               "down": 2.0 * pairs * de * D, "shared": 2.0 * shape.T * ds * D}
+    dom = max(kflops, key=lambda k: kms[k])
+    dom_tf = kflops[dom] / (kms[dom] / 1e3) / 1e12
     out["prefill_t4096"] = {"ms": ms, "tokens_per_s": shape.T / (ms / 1e3),
+                            "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(dom_tf, 1),
+                                         "peak": P["bf16"], "unit": "TFLOP/s",
+                                         "frac": round(dom_tf / P["bf16"], 4), "peak_source": P["src"]},
                             "tflops": flops / (ms / 1e3) / 1e12,
                             "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / P["bf16"],
                             "mean_activation": float(act.float().mean()),

@@ -733,7 +733,7 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
   da.out = out;
   da.residual = 0;
   cudaError_t err;
-  if (dtype == DECO_BF16 && T > dec::kMaxT)
+  if (dtype == DECO_BF16)   // tensor cores at any batch size (a 128-row tile covers a small batch)
     return cuda_status(run_dense_tc(T, d_model, d_ff, x, W1, W2, out, ws, cs), "dense_ffn");
   const int tt = token_tile(d_model, dtype);
   if (dtype == DECO_F32) {

@@ -472,20 +472,16 @@ __global__ void __launch_bounds__(kThreads, 1) kd_route(const __grid_constant__ 
     if (w_ok && warp < ne) {
       const int e = e0 + warp;
       const bf16* wrow = reinterpret_cast<const bf16*>(ring.stage + (size_t)k * kStageBytes + (size_t)rs * rowbytes);
-      constexpr int kMaxChunks = 16;
-      uint4 w[kMaxChunks];
-#pragma unroll
-      for (int i = 0; i < kMaxChunks; ++i)
-        if (i < nc) w[i] = *reinterpret_cast<const uint4*>(wrow + (size_t)(lane + 32 * i) * 8);
       float v[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = 0.f;
-      // each lane: its D/32 products in chunk order (z in v[t], sum |x w| in v[16+t])
-#pragma unroll
-      for (int i = 0; i < kMaxChunks; ++i) {
-        if (i < nc) {
+      // each lane: its D/32 products in chunk order (z in v[t], sum |x w| in v[16+t]);
+      // the chunk loop stays rolled so the loop body fits the instruction cache
+#pragma unroll 1
+      for (int i = 0; i < nc; ++i) {
+        {
           float wv[8];
-          bf16x8_to_f32(w[i], wv);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(wrow + (size_t)(lane + 32 * i) * 8), wv);
 #pragma unroll
           for (int t = 0; t < kTok; ++t) {
             if (t < a.T) {

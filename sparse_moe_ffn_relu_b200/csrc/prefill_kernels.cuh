@@ -975,8 +975,17 @@ __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__
 // and lanes in order inside a warp.  Block 0 also writes counts, offsets and
 // the list of row tiles (<= tile_rows pairs of one expert each).
 
-constexpr int kTabThreads = 256;
+constexpr int kTabThreads = 128;
 constexpr int kTabWarps = kTabThreads / 32;
+
+// active flags of token t for experts e0..e0+31 as bits (independent loads)
+__device__ __forceinline__ uint32_t row_bits(const uint8_t* row, bool ok, int E, int e0) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (ok && e0 + j < E && row[e0 + j]) bits |= 1u << j;
+  return bits;
+}
 
 __global__ void __launch_bounds__(kTabThreads) k_tab_count(const uint8_t* __restrict__ act, int T, int E,
                                                            int* __restrict__ n_tok, int* __restrict__ blk_counts) {
@@ -986,11 +995,13 @@ __global__ void __launch_bounds__(kTabThreads) k_tab_count(const uint8_t* __rest
   const bool ok = t < T;
   const uint8_t* row = act + (size_t)(ok ? t : 0) * E;
   int n = 0;
-  for (int e = 0; e < E; ++e) {
-    const bool f = ok && row[e];
-    const unsigned m = __ballot_sync(kFull, f);
-    if (lane == 0) wc[warp][e] = __popc(m);
-    n += f;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const uint32_t bits = row_bits(row, ok, E, e0);
+    n += __popc(bits);
+    for (int j = 0; j < 32 && e0 + j < E; ++j) {
+      const unsigned m = __ballot_sync(kFull, (bits >> j) & 1u);
+      if (lane == 0) wc[warp][e0 + j] = __popc(m);
+    }
   }
   if (ok) n_tok[t] = n;
   __syncthreads();
@@ -1074,8 +1085,11 @@ __global__ void __launch_bounds__(kTabThreads) k_tab_scatter(const uint8_t* __re
   const int t = blockIdx.x * kTabThreads + threadIdx.x;
   const bool ok = t < T;
   const uint8_t* row = act + (size_t)(ok ? t : 0) * E;
+  uint32_t rb[8];   // this token's flags, 32 experts per word (E <= 256)
+#pragma unroll
+  for (int c = 0; c < 8; ++c) rb[c] = c * 32 < E ? row_bits(row, ok, E, c * 32) : 0u;
   for (int e = 0; e < E; ++e) {
-    const unsigned m = __ballot_sync(kFull, ok && row[e]);
+    const unsigned m = __ballot_sync(kFull, (rb[e >> 5] >> (e & 31)) & 1u);
     if (lane == 0) wc[warp][e] = __popc(m);
   }
   __syncthreads();
@@ -1091,7 +1105,7 @@ __global__ void __launch_bounds__(kTabThreads) k_tab_scatter(const uint8_t* __re
   __syncthreads();
   const unsigned lt = (1u << lane) - 1u;
   for (int e = 0; e < E; ++e) {
-    const bool f = ok && row[e];
+    const bool f = (rb[e >> 5] >> (e & 31)) & 1u;
     const unsigned m = __ballot_sync(kFull, f);
     if (f) {
       const int pos = wc[warp][e] + __popc(m & lt);
