@@ -38,6 +38,11 @@ sys.path.insert(0, ROOT)
 
 DECODE_TS = (1, 4, 16)
 DECODE_KERNELS = ("route", "up", "down")     # the decode path's launches per forward
+# DRAM bytes (read + write) per launch from an ncu capture of the current decode
+# kernels on the edge layer (profiles/decode_kernels_edge_decode_t16.md); a kernel
+# changed since its capture has no entry
+NCU_DRAM_BYTES = {("down", 16): 69_609_216 + 755_712, ("up", 16): 65_156_352 + 247_552,
+                  ("route", 16): 5_636_608}
 METRIC = "MoE-layer tokens/s (decode)"
 
 
@@ -317,9 +322,11 @@ def main():
                for T in DECODE_TS}
     mean_ms = {T: {k: statistics.mean(v) for k, v in kt[T].items()} for T in DECODE_TS}
     tot_k = {k: sum(mean_ms[T][k] for T in DECODE_TS) for k in DECODE_KERNELS}
+    # the dominant kernel (most time per step), at the largest decode batch
     dom = max(tot_k, key=tot_k.get)
-    dom_bytes = sum(bytes_k[T][dom] for T in DECODE_TS) / len(DECODE_TS)
-    dom_ms = tot_k[dom] / len(DECODE_TS)
+    T_r = max(DECODE_TS)
+    dom_bytes = bytes_k[T_r][dom]
+    dom_ms = mean_ms[T_r][dom]
     achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
     step_bytes = sum(sum(b.values()) for b in bytes_k.values())
     layer_gbs = step_bytes / (ms / args.steps / 1000.0) / 1e9
@@ -365,8 +372,9 @@ def main():
                    "union_experts": {str(T): union[T] for T in DECODE_TS},
                    "l2": f"rotating {n_copies} weight copies ({wbytes / 1e6:.0f} MB each) > 3x L2",
                    "cuda_graph": True, "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": P["hbm"],
-                     "unit": "GB/s", "frac": achieved / P["hbm"], "traffic": None,
+        "roofline": {"bound": "hbm", "kernel": dom, "T": T_r, "achieved": achieved, "peak": P["hbm"],
+                     "unit": "GB/s", "frac": achieved / P["hbm"], "traffic": NCU_DRAM_BYTES.get((dom, T_r)),
+                     "algorithmic_bytes": dom_bytes,
                      "peak_source": P["src"], "layer_achieved_gbs": layer_gbs,
                      "layer_frac": layer_gbs / P["hbm"],
                      "kernel_ms_by_T": {str(T): {k: round(mean_ms[T][k], 4) for k in DECODE_KERNELS}
