@@ -37,12 +37,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 DECODE_TS = (1, 4, 16)
-DECODE_KERNELS = ("route", "up", "down")     # the decode path's launches per forward
+DECODE_KERNELS = ("route", "up", "down", "combine")   # the decode path's launches per forward
 # DRAM bytes (read + write) per launch from an ncu capture of the current decode
 # kernels on the edge layer (profiles/decode_kernels_edge_decode_t16.md); a kernel
 # changed since its capture has no entry
-NCU_DRAM_BYTES = {("down", 16): 69_609_216 + 755_712, ("up", 16): 65_156_352 + 247_552,
-                  ("route", 16): 5_636_608}
+NCU_DRAM_BYTES = {("route", 16): 5_636_608}
 METRIC = "MoE-layer tokens/s (decode)"
 
 
@@ -185,7 +184,8 @@ def layer_bytes(shape, union_experts: int):
         "count": 0,
         "scatter": 0,
         "up": (union_experts * d_e * D + T * D) * es,
-        "down": (union_experts * D * d_e + D * d_s + T * D) * es,
+        "down": (union_experts * D * d_e + D * d_s) * es,
+        "combine": 2 * T * D * es,
     }
 
 
@@ -257,7 +257,7 @@ def main():
 
     # events around every kernel of every forward (eager calls: the library
     # records them with cudaEventRecord between its launches; PDL is off then)
-    nk = len(deco.KERNELS)
+    nk = len(deco.PREFILL_KERNELS)
     ev = {T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for T in DECODE_TS}
     for es in ev.values():          # torch creates CUDA events lazily, on first record
         for e in es:
@@ -297,7 +297,7 @@ def main():
     value = world * tokens_per_step * args.steps / (ms / 1000.0)
 
     # live kernel durations: eager forwards on the rotating weight copies
-    kt = {T: {k: [] for k in deco.KERNELS} for T in DECODE_TS}
+    kt = {T: {k: [] for k in deco.PREFILL_KERNELS} for T in DECODE_TS}
     with torch.cuda.stream(stream):
         for i in range(min(args.steps, 60) + 3):
             G = copies[i % n_copies]
@@ -309,7 +309,7 @@ def main():
             if i < 3:
                 continue
             for T in DECODE_TS:
-                for j, k in enumerate(deco.KERNELS):
+                for j, k in enumerate(deco.PREFILL_KERNELS):
                     kt[T][k].append(ev[T][2 * j].elapsed_time(ev[T][2 * j + 1]))
     # routing statistics -> union of active experts per batch
     union, ratio = {}, []

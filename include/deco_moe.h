@@ -171,8 +171,8 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
 deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
 
 /* Size of the library's built-in device scratch used by
- * deco_moe_forward_static: 32 MiB on every GPU that loads the library. */
-#define DECO_STATIC_SCRATCH_BYTES (32u << 20)
+ * deco_moe_forward_static: 64 MiB on every GPU that loads the library. */
+#define DECO_STATIC_SCRATCH_BYTES (64u << 20)
 
 /* deco_moe_forward without a caller-provided workspace.  The paper has no
  * counterpart for this; it exists for callers that cannot allocate device

@@ -133,12 +133,12 @@ def forward(x: torch.Tensor, L: dict, out=None, workspace=None, eps=1e-6, residu
     return out
 
 
-STATIC_SCRATCH_BYTES = 32 << 20
+STATIC_SCRATCH_BYTES = 64 << 20
 
 
 def forward_static(x: torch.Tensor, L: dict, out=None, eps=1e-6, residual=False,
                    stream=None) -> torch.Tensor:
-    """forward() on the library's built-in 32 MiB device scratch instead of a
+    """forward() on the library's built-in 64 MiB device scratch instead of a
     workspace, for callers that cannot allocate device memory while running
     layers.  Calls on one device share that scratch: do not let them overlap
     on the GPU.  The first call on a device should come before any stream
@@ -205,8 +205,8 @@ def dense_ffn(x, W1, W2, out=None, workspace=None, stream=None) -> torch.Tensor:
 
 
 # timing slots of deco_moe_set_profiling: slot i is bracketed by events 2i and
-# 2i+1.  The decode path (bf16, T <= 16) fills route, up and down; the general
-# path route..down; the prefill path (bf16, T > 16) all eight.
+# 2i+1.  The decode path (bf16, T <= 16) fills route, up, down and combine;
+# the general path route..down; the prefill path (bf16, T > 16) all eight.
 KERNELS = ("route", "count", "scatter", "up", "down")
 PREFILL_KERNELS = KERNELS + ("proj", "shared", "combine")
 

@@ -25,8 +25,7 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 struct Plan {
   size_t err, r, act, u, hs, counts, offsets, n_tok, perm, pair_of, tiles, n_tiles, H, total;
   // decode path (T <= 16)
-  size_t hs16, C16, a_cmp, cnt;
-  size_t cnt_bytes;
+  size_t hs16, C16, P16, Ps16;
   // bf16, T > 16: ambiguous router pairs; prefill path: routed expert output
   // rows (one fp16 row per pair) and the shared expert's fp32 output
   size_t fb, blk, v_pairs, s_out;
@@ -90,9 +89,8 @@ Plan make_plan(const deco_moe_shape_t& s) {
   if (s.T <= dec::kMaxT) {         // decode path buffers (see decode_kernels.cuh)
     p.hs16 = take((size_t)dec::kTok * s.d_s * 4);         // [16][hi d_s | lo d_s] bf16
     p.C16 = take(E * dec::kTok * s.d_e * 4);               // [E][16][d_e] fp32
-    p.a_cmp = take(E * dec::kTok * s.d_e * 4);             // [E][16][hi d_e | lo d_e] bf16
-    p.cnt_bytes = E * 4;
-    p.cnt = take(p.cnt_bytes);
+    p.P16 = take(E * dec::kTok * s.d_model * 4);           // [E][16][D] fp32
+    p.Ps16 = take((size_t)dec::down_nsq(s.d_s) * dec::kTok * s.d_model * 4);   // [nsq][16][D] fp32
   }
   p.total = off;
   return p;
@@ -278,99 +276,6 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
 // ---------------------------------------------------------------------------
 // decode path: bf16, T <= 16 (weight-streaming kernels, see decode_kernels.cuh)
 
-bool decode_eligible(const deco_moe_shape_t& s, int sms) {
-  if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT) return false;
-  if (s.d_model % 256 || s.d_model > 4096) return false;
-  if (s.E > 256 || s.d_e > 512 || s.d_e % 64 || s.d_s % 64 || s.d_s > 2048) return false;
-  if ((s.E + 7) / 8 >= sms) return false;                     // router CTAs leave room
-  const int R = dec::down_rows(s.d_model, sms);
-  if (R > 32) return false;                                    // two 16-row m-tiles per CTA
-  // one routed expert's slab plus its activation rows fit one stage
-  if (((uint32_t)R * s.d_e * 2 + 127u) / 128u * 128u + (uint32_t)s.T * s.d_e * 4 > dec::kStageBytes) return false;
-  const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
-  if (dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).nstages < 2) return false;
-  if (dec::smem_plan(xop, dec::kStageBytes).nstages < 2) return false;
-  if (dec::smem_plan((uint32_t)dec::kTok * s.d_s * 4 + 8 * 2048 + (uint32_t)s.d_e * 4, dec::kStageBytes).nstages < 2)
-    return false;
-  return true;
-}
-
-template <typename K>
-cudaError_t launch_dec(K kernel, const dec::Args& a, uint32_t smem_total, bool pdl, int grid, cudaStream_t st) {
-  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_total);
-  if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(dec::kThreads);
-  cfg.dynamicSmemBytes = smem_total;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, a);
-}
-
-cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
-                       void* out, unsigned char* ws, const Plan& p, cudaStream_t st) {
-  dec::Args a{};
-  a.T = s.T;
-  a.D = s.d_model;
-  a.E = s.E;
-  a.d_e = s.d_e;
-  a.d_s = s.d_s;
-  a.eps = s.rms_eps;
-  a.residual = s.residual;
-  a.x = static_cast<const bf16*>(x);
-  a.W_r = static_cast<const bf16*>(w.W_r);
-  a.b_r = w.b_r;
-  a.W_bar = static_cast<const bf16*>(w.W_bar_up);
-  a.W_up = static_cast<const bf16*>(w.W_up);
-  a.W_down = static_cast<const bf16*>(w.W_down);
-  a.s = w.s;
-  a.W_s_up = static_cast<const bf16*>(w.W_s_up);
-  a.W_s_down = static_cast<const bf16*>(w.W_s_down);
-  a.r = reinterpret_cast<float*>(ws + p.r);
-  a.act = reinterpret_cast<uint8_t*>(ws + p.act);
-  a.u = reinterpret_cast<float*>(ws + p.u);
-  a.hs = reinterpret_cast<bf16*>(ws + p.hs16);
-  a.C = reinterpret_cast<float*>(ws + p.C16);
-  a.a_cmp = reinterpret_cast<bf16*>(ws + p.a_cmp);
-  a.cnt_u = reinterpret_cast<int*>(ws + p.cnt);
-  a.err = reinterpret_cast<int*>(ws + p.err);
-  a.out = static_cast<bf16*>(out);
-  // completion counters start at zero every call
-  cudaError_t err = cudaMemsetAsync(ws + p.cnt, 0, p.cnt_bytes, st);
-  if (err != cudaSuccess) return err;
-  const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
-  const uint32_t route_smem = std::max(dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).total,
-                                       dec::smem_plan(xop, dec::kStageBytes).total);
-  const uint32_t down_smem =
-      dec::smem_plan((uint32_t)dec::kTok * s.d_s * 4 + 8 * 2048 + (uint32_t)s.d_e * 4, dec::kStageBytes).total;
-  // with timing events between the kernels each one is timed on its own
-  const bool pdl = g_prof_events == nullptr;
-  prof_mark(0, st);
-  err = launch_dec(dec::kd_route, a, route_smem, false, p.sms, st);
-  if (err != cudaSuccess) return err;
-  prof_mark(1, st);
-  prof_mark(2, st);
-  prof_mark(3, st);
-  prof_mark(4, st);
-  prof_mark(5, st);
-  prof_mark(6, st);
-  err = launch_dec(dec::kd_up, a, dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).total, pdl, p.sms, st);
-  if (err != cudaSuccess) return err;
-  prof_mark(7, st);
-  prof_mark(8, st);
-  err = launch_dec(dec::kd_down, a, down_smem, pdl, p.sms, st);
-  prof_mark(9, st);
-  return err;
-}
-
-// ---------------------------------------------------------------------------
-// prefill path: bf16, T > 16 (tcgen05 GEMMs, see prefill_kernels.cuh)
-
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -402,6 +307,106 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+
+// kd_down's resident operands: hidden rows, the NormSiLU tile, a zero row
+uint32_t dec_down_operand(const deco_moe_shape_t& s) {
+  return (uint32_t)dec::kTok * s.d_s * 4 + (uint32_t)dec::kTok * s.d_e * 4 + 1024;
+}
+
+bool decode_eligible(const deco_moe_shape_t& s, int sms) {
+  if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT) return false;
+  if (s.d_model % 256 || s.d_model > 4096) return false;
+  if (s.E > 256 || s.d_e > 256 || s.d_e % 64 || s.d_s % 64 || s.d_s > 2048) return false;
+  if ((s.E + 7) / 8 >= sms) return false;                     // router CTAs leave room
+  const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
+  if (dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).nstages < 2) return false;
+  if (dec::smem_plan(xop, dec::kStageBytes).nstages < 2) return false;
+  if (dec::smem_plan(dec_down_operand(s), dec::kStageBytes).nstages < 2) return false;
+  return true;
+}
+
+// launch with an optional programmatic-dependent-launch edge to the previous kernel
+template <typename K, typename... Ps>
+cudaError_t launch_dec(K kernel, dim3 grid, dim3 block, uint32_t smem_total, bool pdl, cudaStream_t st,
+                       const Ps&... params) {
+  if (smem_total > 48 * 1024) {
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_total);
+    if (err != cudaSuccess) return err;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem_total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, params...);
+}
+
+cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
+                       void* out, unsigned char* ws, const Plan& p, cudaStream_t st) {
+  dec::Args a{};
+  a.T = s.T;
+  a.D = s.d_model;
+  a.E = s.E;
+  a.d_e = s.d_e;
+  a.d_s = s.d_s;
+  a.eps = s.rms_eps;
+  a.residual = s.residual;
+  a.x = static_cast<const bf16*>(x);
+  a.W_r = static_cast<const bf16*>(w.W_r);
+  a.b_r = w.b_r;
+  a.W_bar = static_cast<const bf16*>(w.W_bar_up);
+  a.W_up = static_cast<const bf16*>(w.W_up);
+  a.W_down = static_cast<const bf16*>(w.W_down);
+  a.s = w.s;
+  a.W_s_up = static_cast<const bf16*>(w.W_s_up);
+  a.W_s_down = static_cast<const bf16*>(w.W_s_down);
+  a.r = reinterpret_cast<float*>(ws + p.r);
+  a.act = reinterpret_cast<uint8_t*>(ws + p.act);
+  a.u = reinterpret_cast<float*>(ws + p.u);
+  a.hs = reinterpret_cast<bf16*>(ws + p.hs16);
+  a.C = reinterpret_cast<float*>(ws + p.C16);
+  a.P = reinterpret_cast<float*>(ws + p.P16);
+  a.Ps = reinterpret_cast<float*>(ws + p.Ps16);
+  a.err = reinterpret_cast<int*>(ws + p.err);
+  a.out = static_cast<bf16*>(out);
+  // kd_down's weight tiles: 128 rows x 64 columns
+  CUtensorMap tmW, tmS;
+  cudaError_t err;
+  if ((err = make_map(&tmW, w.W_down, s.d_e, (uint64_t)s.E * s.d_model, dec::kDRows)) != cudaSuccess ||
+      (err = make_map(&tmS, w.W_s_down, s.d_s, s.d_model, dec::kDRows)) != cudaSuccess)
+    return err;
+  const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
+  const uint32_t route_smem = std::max(dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).total,
+                                       dec::smem_plan(xop, dec::kStageBytes).total);
+  const uint32_t down_smem = dec::smem_plan(dec_down_operand(s), dec::kStageBytes).total;
+  const dim3 grid(p.sms), block(dec::kThreads);
+  // with timing events between the kernels each one is timed on its own
+  const bool pdl = g_prof_events == nullptr;
+  prof_mark(0, st);
+  err = launch_dec(dec::kd_route, grid, block, route_smem, false, st, a);
+  if (err != cudaSuccess) return err;
+  prof_mark(1, st);
+  prof_mark(6, st);
+  err = launch_dec(dec::kd_up, grid, block, dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).total, pdl, st, a);
+  if (err != cudaSuccess) return err;
+  prof_mark(7, st);
+  prof_mark(8, st);
+  err = launch_dec(dec::kd_down, grid, block, down_smem, pdl, st, tmW, tmS, a);
+  if (err != cudaSuccess) return err;
+  prof_mark(9, st);
+  prof_mark(14, st);
+  err = launch_dec(dec::kd_combine, dim3((s.d_model + 255) / 256, s.T), dim3(256), 0, pdl, st, a);
+  prof_mark(15, st);
+  return err;
+}
+
+// ---------------------------------------------------------------------------
+// prefill path: bf16, T > 16 (tcgen05 GEMMs, see prefill_kernels.cuh)
 
 template <int MODE>
 cudaError_t launch_pf(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2, const CUtensorMap& O,

@@ -9,11 +9,13 @@
 //   kd_route  router rows W_r (exact activation decisions, CUDA cores), and
 //             the mean up-projection W_bar_up and shared up-projection W_s_up
 //             (tensor cores) -> r, active, u = x W_bar_up^T, SiLU(x W_s_up^T)
-//   kd_up     W_up[e] of the union of active experts (tensor cores); the CTA
-//             that completes an expert applies NormSiLU (subtract u, RMS over
-//             d_e, SiLU) and writes s_e * r_e * a for its tokens
-//   kd_down   each CTA owns a block of output rows and accumulates the shared
-//             expert and every active expert's down-projection for them
+//   kd_up     W_up[e] of the union of active experts (tensor cores) -> g
+//   kd_down   units of 128 output rows of one active expert's W_down (or of a
+//             256-column part of W_s_down) arrive as TMA boxes; the CTA computes
+//             the expert's NormSiLU (subtract u, RMS over d_e, SiLU, times
+//             s_e r_e) when the expert changes and writes fp32 partials
+//   kd_combine adds the shared-expert parts and the active experts' partials
+//             in ascending expert order (+ the residual)
 //
 // Data movement: one CTA per SM, 8 consumer warps and 1 producer warp.  The
 // producer streams contiguous weight rows with bulk copies of >= 4 KB each
@@ -23,12 +25,12 @@
 // kd_route / kd_up give each CTA a contiguous range of weight rows at full
 // width and copy each row into a 16-byte padded shared-memory row, so that
 // ldmatrix reads of 8 rows hit 8 different bank groups; the 8 consumer warps
-// split the columns and add their partial sums in warp order.  kd_down gives
-// each CTA a block of output rows; each active expert's slab of those rows is
-// one contiguous copy, which a warp re-lays into a swizzled tile before use.
-// Activations a later kernel consumes are written in a layout its copies and
-// ldmatrix reads can use directly (an XOR swizzle of the 16-byte chunks inside
-// each row).
+// split the columns and add their partial sums in warp order.  kd_down loads
+// 128-row x 64-column tiles with TMA in the 128-byte swizzle, which ldmatrix
+// reads directly; each consumer warp owns 16 of the 128 rows.
+// Activations a later kernel consumes are written in a layout its ldmatrix
+// reads can use directly (an XOR swizzle of the 16-byte chunks inside each
+// row).
 //
 // Arithmetic: the projections are tiny dense contractions (16 tokens x 8..64
 // weight rows x K) done with mma.sync m16n8k16 (bf16 in, fp32 accumulate): a
@@ -270,9 +272,9 @@ struct Args {
   float* u;          // [T][d_e]
   bf16* hs;          // [16 tok][hi d_s | lo d_s], chunk-swizzled rows: SiLU(x W_s_up^T)
   float* C;          // [E][16 tok][d_e] up-projection g = x W_up[e]^T (active experts)
-  bf16* a_cmp;       // [E][16 slots][hi d_e | lo d_e], chunk-swizzled rows: s_e r_e NormSiLU,
-                     // slot i = the i-th active token of expert e (ascending)
-  int* cnt_u;        // [E] finished rows per expert (zero at entry)
+  float* P;          // [E][16 slots][D] routed down-projection partials, slot i = the i-th
+                     // active token of expert e (ascending)
+  float* Ps;         // [ceil(d_s / 256)][16 tok][D] shared down-projection partials
   int* err;
   bf16* out;
 };
@@ -575,16 +577,13 @@ __global__ void __launch_bounds__(kThreads, 1) kd_route(const __grid_constant__ 
 
 // ---------------------------------------------------------------------------
 // kd_up: the rows of W_up[e] for the active experts e (in union order), split
-// evenly over the CTAs; writes g = x W_up[e]^T; the CTA that completes an
-// expert applies NormSiLU to its active tokens and writes the compact,
-// scaled activations for kd_down.
+// evenly over the CTAs; writes g = x W_up[e]^T (NormSiLU runs in kd_down).
 
 __global__ void __launch_bounds__(kThreads, 1) kd_up(const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint16_t emask[256];
   __shared__ uint8_t ulist[256];
   __shared__ int s_U;
-  __shared__ int fin_u[16], n_fin;
   const uint32_t pitch = x_pitch(a.D);
   const SmemPlan sp = smem_plan(kTok * pitch + 4096, row_stage_bytes(a.D));
   Ring ring;
@@ -639,307 +638,259 @@ __global__ void __launch_bounds__(kThreads, 1) kd_up(const __grid_constant__ Arg
       }
     }
   }
-  // publish; the CTA that completes an expert runs its NormSiLU
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    n_fin = 0;
-    if (!*abort_flag) {
-      for (int g = ra; g < rb;) {
-        const int ue = g / a.d_e;
-        const int n = min(rb, (ue + 1) * a.d_e) - g;
-        const int old = atomicAdd(a.cnt_u + ulist[ue], n);
-        if (old + n == a.d_e && n_fin < 16) fin_u[n_fin++] = ue;
-        g += n;
-      }
-    }
-  }
-  __syncthreads();
-  if (warp >= kConsumerWarps || n_fin == 0) return;
-  __threadfence();
-  const float inv_de = 1.f / float(a.d_e);
-  int item = 0;
-  for (int f = 0; f < n_fin; ++f) {
-    const int e = ulist[fin_u[f]];
-    const float se = a.s[e];
-    int slot = 0;
-    for (uint32_t m = emask[e]; m; m &= m - 1, ++slot, ++item) {
-      if (item % kConsumerWarps != warp) continue;
-      const int t = __ffs(m) - 1;
-      float cv[16];   // d_e <= 512: 16 values per lane
-      float ss = 0.f;
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const int j = lane + 32 * q;
-        cv[q] = 0.f;
-        if (j < a.d_e) {
-          cv[q] = __ldcg(a.C + ((size_t)e * kTok + t) * a.d_e + j) - __ldcg(a.u + (size_t)t * a.d_e + j);
-          ss = fmaf(cv[q], cv[q], ss);
-        }
-      }
-      ss = warp_sum(ss);
-      const float rinv = 1.f / sqrtf(ss * inv_de + a.eps);
-      const float coef = se * __ldcg(a.r + (size_t)t * a.E + e);
-      bf16* row = a.a_cmp + ((size_t)e * kTok + slot) * 2 * a.d_e;
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const int j = lane + 32 * q;
-        if (j < a.d_e) store_row_hi_lo(row, slot, a.d_e, j, coef * silu_f(cv[q] * rinv));
-      }
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
-// kd_down: CTA c owns output rows [n0, n1), at most 32.  Its units, packed
-// greedily into 32 KB stages, are the shared expert's row pieces
-// W_s_down[m0:m1][:] and then, per active expert e ascending, the slab
-// W_down[e][n0:n1][:] followed by the expert's compact activation rows.  Unit
-// u is multiplied by consumer warp u % 8: for each 64-column tile the warp
-// re-lays the slab's rows into a swizzled 16 x 64 scratch tile and runs
-// m16n8k16 steps with the weights as A (rows) and the token activations as B.
-// B rows of tokens that do not use the expert point at a zero row, so every
-// warp accumulates token-indexed results in registers; the 8 warps' sums are
-// added in warp order at the end (deterministic).
+// kd_down: the routed and the shared down-projections as fp32 partial sums.
+//
+// Units are (expert e of the union, block of 128 output rows), with all of d_e
+// as K, and (K part q of 256 columns of W_s_down, block of 128 output rows)
+// for the shared expert.  CTA c takes a contiguous range of the units (shared
+// ones first, then experts ascending), so consecutive units mostly share an
+// expert.  A unit's weights arrive as TMA boxes of 128 rows x 64 columns
+// (16 KB, 128-byte swizzle, the layout ldmatrix reads without bank
+// conflicts), two boxes per 32 KB stage; consumer warp w multiplies the unit's
+// rows 16w..16w+15 (m16n8k16, weights as A, tokens as B).  B rows are the
+// shared expert's hidden activations (hi/lo, resident in shared memory) or the
+// expert's NormSiLU activations, which the CTA computes when the expert
+// changes: c = g - u, h = c / sqrt(mean c^2 + eps), a = s_e r_e SiLU(h), stored
+// as hi/lo in compact slots (slot i = the i-th active token of e).  Results go
+// to P[e][slot][row] and Ps[q][token][row]; kd_combine adds them.
 
-__host__ __device__ inline int down_rows(int D, int G) { return (D + G - 1) / G; }
+constexpr int kDRows = 128;                  // output rows per unit
+constexpr uint32_t kBoxBytes = kDRows * 128; // 128 rows x 64 bf16 columns
+constexpr int kSq = 256;                     // K columns per shared-expert unit
 
-struct DownUnits {
-  int n0, n1, srows, nshared, nunits;
+__host__ __device__ inline int down_nsq(int d_s) { return (d_s + kSq - 1) / kSq; }
+
+struct DUnit {
+  bool shared;
+  int e, q, rb, K, kb0;   // kb0: first K column of the unit within its matrix row
 };
 
-__device__ __forceinline__ uint32_t down_unit_bytes(const Args& a, const DownUnits& du, const uint16_t* emask,
-                                                    const uint8_t* ulist, int u) {
-  if (u < du.nshared) {
-    const int m0 = du.n0 + u * du.srows, m1 = min(du.n1, m0 + du.srows);
-    return (uint32_t)(m1 - m0) * a.d_s * 2;
+__device__ __forceinline__ DUnit down_unit(const Args& a, const uint8_t* ulist, int nrb, int u) {
+  DUnit d;
+  const int ns = down_nsq(a.d_s) * nrb;
+  d.shared = u < ns;
+  if (d.shared) {
+    d.q = u / nrb;
+    d.rb = u - d.q * nrb;
+    d.kb0 = d.q * kSq;
+    d.K = min(kSq, a.d_s - d.kb0);
+    d.e = -1;
+  } else {
+    const int v = u - ns, ui = v / nrb;
+    d.rb = v - ui * nrb;
+    d.e = ulist[ui];
+    d.q = 0;
+    d.kb0 = 0;
+    d.K = a.d_e;
   }
-  const uint32_t w = (uint32_t)(du.n1 - du.n0) * a.d_e * 2;
-  const uint32_t act = (uint32_t)__popc(emask[ulist[u - du.nshared]]) * a.d_e * 4;
-  return ((w + 127u) & ~127u) + act;
+  return d;
 }
 
-__device__ __forceinline__ int down_stage_end(const Args& a, const DownUnits& du, const uint16_t* emask,
-                                              const uint8_t* ulist, int u, uint32_t cap) {
-  uint32_t used = (down_unit_bytes(a, du, emask, ulist, u) + 127u) & ~127u;
-  int v = u + 1;
-  while (v < du.nunits) {
-    const uint32_t b = (down_unit_bytes(a, du, emask, ulist, v) + 127u) & ~127u;
-    if (used + b > cap) break;
-    used += b;
-    ++v;
-  }
-  return v;
-}
-
-// re-lay columns [64c, 64c+64) of a row-major slab (nr rows, pitch bytes per
-// row) into a swizzled 16 x 64 tile at `tile`: tile row r takes slab row
-// sr0 + r, or zeros where that is outside [0, nr); one warp
-__device__ __forceinline__ void relayout_tile(const unsigned char* slab, uint32_t pitch, int sr0, int nr, int c,
-                                              unsigned char* tile, int lane) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int r = q * 4 + (lane >> 3), k = lane & 7;
-    const int sr = sr0 + r;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (sr >= 0 && sr < nr) v = *reinterpret_cast<const uint4*>(slab + (size_t)sr * pitch + (size_t)(c * 8 + k) * 16);
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((k ^ (r & 7)) << 4)) = v;
-  }
-  __syncwarp();
-}
-
-__global__ void __launch_bounds__(kThreads, 1) kd_down(const __grid_constant__ Args a) {
+__global__ void __launch_bounds__(kThreads, 1)
+    kd_down(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
+            const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint16_t emask[256];
   __shared__ uint8_t ulist[256];
   __shared__ int s_U;
-  // operand: hs rows (16 x 4 d_s bytes), per-warp scratch tiles (8 x 2 KB),
-  // a zero activation row (4 d_e bytes)
+  // operand: hs rows (16 x 4 d_s bytes), the NormSiLU tile (16 x 4 d_e bytes),
+  // a zero row for slots past the expert's tokens (4 d_e <= 1 KB)
   const uint32_t hbytes = (uint32_t)kTok * a.d_s * 4;
-  const SmemPlan sp = smem_plan(hbytes + 8 * 2048 + (uint32_t)a.d_e * 4, kStageBytes);
+  const uint32_t tbytes = (uint32_t)kTok * a.d_e * 4;
+  const SmemPlan sp = smem_plan(hbytes + tbytes + 1024, kStageBytes);
   Ring ring;
   uint64_t* hbar;
   volatile int* abort_flag;
   unsigned char* smem = ring_setup(smem_raw, sp, ring, hbar, abort_flag);
   unsigned char* hsm = smem + sp.op_off;
-  unsigned char* scratch = hsm + hbytes;
-  unsigned char* zrow = scratch + 8 * 2048;
+  unsigned char* tile = hsm + hbytes;
+  unsigned char* zrow = tile + tbytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < a.d_e / 4; i += blockDim.x) reinterpret_cast<uint4*>(zrow)[i] = make_uint4(0, 0, 0, 0);
+  pdl_trigger();
+  for (int i = threadIdx.x; i < 1024 / 16; i += blockDim.x) reinterpret_cast<uint4*>(zrow)[i] = make_uint4(0, 0, 0, 0);
   // The router's outputs are complete: this grid starts only after every CTA
   // of kd_up passed its own wait on the router.
   build_union(a, emask, ulist, &s_U);
-  DownUnits du;
-  du.n0 = (int)(((long long)blockIdx.x * a.D) / gridDim.x);
-  du.n1 = (int)(((long long)(blockIdx.x + 1) * a.D) / gridDim.x);
-  const int R = du.n1 - du.n0;
-  // shared pieces: a power of two >= 8 rows (so a piece never straddles two
-  // 16-row m-tiles), at most one stage
-  du.srows = 8;
-  while (du.srows * 2 * a.d_s * 2 <= (int)kStageBytes && du.srows < 32) du.srows *= 2;
-  du.nshared = (R + du.srows - 1) / du.srows;
-  du.nunits = du.nshared + s_U;
-  const uint32_t wbytes = (uint32_t)R * a.d_e * 2;
-  const uint32_t wpad = (wbytes + 127u) & ~127u;
+  const int nrb = a.D / kDRows;
+  const int NU = (down_nsq(a.d_s) + s_U) * nrb;
+  const int u0 = (int)((long long)blockIdx.x * NU / gridDim.x);
+  const int u1 = (int)((long long)(blockIdx.x + 1) * NU / gridDim.x);
 
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       const uint64_t pol = evict_first_policy();
       mbar_expect_tx(hbar, hbytes);
       bulk_g2s(hsm, a.hs, hbytes, hbar);
-      auto issue_w = [&](int v0, int v1, int s) {
-        unsigned char* st = ring.stage + (size_t)s * ring.stage_bytes;
-        uint32_t total = 0;
-        for (int u = v0; u < v1; ++u) total += down_unit_bytes(a, du, emask, ulist, u) - (u < du.nshared ? 0 : wpad - wbytes);
-        mbar_expect_tx(&ring.full[s], total);
-        uint32_t off = 0;
-        for (int u = v0; u < v1; ++u) {
-          if (u < du.nshared) {
-            const int m0 = du.n0 + u * du.srows, m1 = min(du.n1, m0 + du.srows);
-            bulk_g2s(st + off, a.W_s_down + (size_t)m0 * a.d_s, (uint32_t)(m1 - m0) * a.d_s * 2, &ring.full[s], pol);
-          } else {
-            const int e = ulist[u - du.nshared];
-            bulk_g2s(st + off, a.W_down + ((size_t)e * a.D + du.n0) * a.d_e, wbytes, &ring.full[s], pol);
-          }
-          off += (down_unit_bytes(a, du, emask, ulist, u) + 127u) & ~127u;
+      // weights do not depend on kd_up: they stream while it finishes
+      int k = 0;
+      for (int u = u0; u < u1; ++u) {
+        const DUnit d = down_unit(a, ulist, nrb, u);
+        const int row = d.shared ? d.rb * kDRows : d.e * a.D + d.rb * kDRows;
+        for (int c0 = 0; c0 < d.K; c0 += 128, ++k) {
+          const int s = k % ring.nstages;
+          if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
+          const int nb = min(2, (d.K - c0) / 64);
+          mbar_expect_tx(&ring.full[s], (uint32_t)nb * kBoxBytes);
+          for (int b = 0; b < nb; ++b)
+            tma_2d(ring.stage + (size_t)s * ring.stage_bytes + b * kBoxBytes, d.shared ? &tmS : &tmW,
+                   d.kb0 + c0 + 64 * b, row, &ring.full[s], pol);
         }
-      };
-      auto issue_a = [&](int v0, int v1, int s) {   // activations written by kd_up
-        unsigned char* st = ring.stage + (size_t)s * ring.stage_bytes;
-        uint32_t off = 0;
-        for (int u = v0; u < v1; ++u) {
-          if (u >= du.nshared) {
-            const int e = ulist[u - du.nshared];
-            const uint32_t n = (uint32_t)__popc(emask[e]) * a.d_e * 4;
-            bulk_g2s(st + off + wpad, a.a_cmp + (size_t)e * kTok * 2 * a.d_e, n, &ring.full[s]);
-          }
-          off += (down_unit_bytes(a, du, emask, ulist, u) + 127u) & ~127u;
-        }
-      };
-      // weights of the first stages go out before kd_up has finished ...
-      int u = 0, k = 0;
-      int first_u[kMaxStages + 1];
-      for (; u < du.nunits && k < ring.nstages; ++k) {
-        const int v = down_stage_end(a, du, emask, ulist, u, ring.stage_bytes);
-        first_u[k] = u;
-        issue_w(u, v, k);
-        u = v;
-      }
-      first_u[k] = u;
-      pdl_wait();
-      // ... their activations only once it has
-      for (int q = 0; q < k; ++q) issue_a(first_u[q], first_u[q + 1], q);
-      for (; u < du.nunits; ++k) {
-        const int v = down_stage_end(a, du, emask, ulist, u, ring.stage_bytes);
-        const int s = k % ring.nstages;
-        if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
-        issue_w(u, v, s);
-        issue_a(u, v, s);
-        u = v;
+        if (*abort_flag) break;
       }
     }
     return;
   }
 
-  // acc[m][n]: rows n0 + 16m .. +16, tokens 8n .. 8n+8 (C fragment layout)
-  float acc[2][2][4] = {};
-  unsigned char* my_tile = scratch + warp * 2048;
-  const uint32_t tile_u32 = smem_u32(my_tile);
-  const int ntiles = (a.T + 7) / 8;
+  pdl_wait();   // g (kd_up), u, r (kd_route)
   bool ok = mbar_wait(hbar, 0, abort_flag, a.err);
-  int k = 0;
-  for (int v0 = 0; ok && v0 < du.nunits; ++k) {
-    const int v1 = down_stage_end(a, du, emask, ulist, v0, ring.stage_bytes);
-    const int s = k % ring.nstages;
-    if (!mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err)) break;
-    const unsigned char* st = ring.stage + (size_t)s * ring.stage_bytes;
-    uint32_t off = 0;
-    for (int u = v0; u < v1; ++u) {
-      if (u % kConsumerWarps == warp) {
-        const bool shared = u < du.nshared;
-        const int m0 = shared ? du.n0 + u * du.srows : du.n0;
-        const int nr = shared ? min(du.n1, m0 + du.srows) - m0 : R;
-        const int K = shared ? a.d_s : a.d_e;
-        const uint32_t pitch = (uint32_t)K * 2;
-        // B rows: token t's activation row (hi part; lo is K columns later)
-        // and the row index its chunks are swizzled with (token or slot)
-        uint32_t brow[2];
-        int bsw[2];
-        uint32_t m_e = 0;
-        if (!shared) m_e = emask[ulist[u - du.nshared]];
+  const uint32_t hs_u32 = smem_u32(hsm), tile_u32 = smem_u32(tile), z_u32 = smem_u32(zrow);
+  int cur_e = -1, n_cur = 0, k = 0;
+  for (int u = u0; u < u1; ++u) {
+    const DUnit d = down_unit(a, ulist, nrb, u);
+    if (!d.shared && d.e != cur_e) {
+      // NormSiLU rows of expert e, one warp per active token
+      consumer_sync();   // every warp is done with the previous tile
+      const int e = d.e;
+      const uint32_t m_e = emask[e];
+      n_cur = __popc(m_e);
+      if (ok && !*abort_flag) {
+        const float se = a.s[e];
+        for (int slot = warp; slot < n_cur; slot += kConsumerWarps) {
+          uint32_t m = m_e;
+          for (int i = 0; i < slot; ++i) m &= m - 1;
+          const int t = __ffs(m) - 1;
+          float cv[8];   // d_e <= 256: 8 values per lane
+          float ss = 0.f;
 #pragma unroll
-        for (int n = 0; n < 2; ++n) {
-          const int t = 8 * n + (lane & 7);
-          if (shared) {
-            brow[n] = smem_u32(hsm) + (uint32_t)t * 4 * a.d_s;
-            bsw[n] = t;
-          } else {
-            const bool on = t < a.T && ((m_e >> t) & 1u);
-            const int slot = __popc(m_e & ((1u << t) - 1u));
-            brow[n] = on ? smem_u32(st + off + wpad) + (uint32_t)slot * 4 * a.d_e : smem_u32(zrow);
-            bsw[n] = on ? slot : 0;
-          }
-        }
-        // output rows [rr0, rr0 + nr) relative to n0, in 16-row m-tiles
-        const int rr0 = m0 - du.n0;
-        for (int ms = rr0 / 16; ms <= (rr0 + nr - 1) / 16; ++ms) {
-          for (int c = 0; c < K / kKB; ++c) {
-            relayout_tile(st + off, pitch, 16 * ms - rr0, nr, c, my_tile, lane);
-#pragma unroll
-            for (int ks = 0; ks < kKB / 16; ++ks) {
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4(a_addr(tile_u32, lane, ks), a0, a1, a2, a3);
-              const int kc = c * 8 + 2 * ks + ((lane >> 3) & 1);   // logical 16-byte chunk of this lane's row
-#pragma unroll
-              for (int n = 0; n < 2; ++n) {
-                if (n < ntiles) {
-                  uint32_t bh0, bh1, bl0, bl1;
-                  ldsm_x2(brow[n] + (uint32_t)row_chunk(bsw[n], kc) * 16u, bh0, bh1);
-                  ldsm_x2(brow[n] + (uint32_t)row_chunk(bsw[n], kc + K / 8) * 16u, bl0, bl1);
-                  if (ms == 0) {
-                    mma16816(acc[0][n], a0, a1, a2, a3, bh0, bh1);
-                    mma16816(acc[0][n], a0, a1, a2, a3, bl0, bl1);
-                  } else {
-                    mma16816(acc[1][n], a0, a1, a2, a3, bh0, bh1);
-                    mma16816(acc[1][n], a0, a1, a2, a3, bl0, bl1);
-                  }
-                }
-              }
+          for (int q = 0; q < 8; ++q) {
+            const int j = lane + 32 * q;
+            cv[q] = 0.f;
+            if (j < a.d_e) {
+              cv[q] = __ldcg(a.C + ((size_t)e * kTok + t) * a.d_e + j) - __ldcg(a.u + (size_t)t * a.d_e + j);
+              ss = fmaf(cv[q], cv[q], ss);
             }
-            __syncwarp();
+          }
+          ss = warp_sum(ss);
+          const float rinv = 1.f / sqrtf(ss / float(a.d_e) + a.eps);
+          const float coef = se * __ldcg(a.r + (size_t)t * a.E + e);
+          bf16* row = reinterpret_cast<bf16*>(tile + (size_t)slot * 4 * a.d_e);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int j = lane + 32 * q;
+            if (j < a.d_e) store_row_hi_lo(row, slot, a.d_e, j, coef * silu_f(cv[q] * rinv));
           }
         }
       }
-      off += (down_unit_bytes(a, du, emask, ulist, u) + 127u) & ~127u;
+      consumer_sync();
+      cur_e = e;
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&ring.empty[s]);
-    v0 = v1;
-  }
-  // add the 8 warps' accumulators in warp order; the scratch reuses stage 0,
-  // whose last copy every consumer warp has awaited
-  consumer_sync();
-  float* red = reinterpret_cast<float*>(ring.stage);   // [8 warps][16 values][32 lanes]
+    // B rows of this unit: tokens (shared) or slots (routed); rows past n read zeros
+    const int n = d.shared ? a.T : n_cur;
+    const int ntiles = (n + 7) / 8;
+    const int L = d.shared ? a.d_s : a.d_e;            // hi half length of a B row
+    uint32_t brow[2];
+    int bsw[2];
 #pragma unroll
-  for (int m = 0; m < 2; ++m)
+    for (int nt = 0; nt < 2; ++nt) {
+      const int r = 8 * nt + (lane & 7);
+      // hidden rows of tokens >= T are zeros (kd_route writes all 16 rows)
+      const bool on = d.shared || r < n;
+      brow[nt] = on ? (d.shared ? hs_u32 : tile_u32) + (uint32_t)r * 4u * (uint32_t)L : z_u32;
+      bsw[nt] = on ? r : 0;
+    }
+    const int kcb = d.kb0 / 8;                          // first 16-byte chunk of the unit in a B row
+    float acc[2][4] = {};
+    for (int c0 = 0; c0 < d.K; c0 += 128, ++k) {
+      const int s = k % ring.nstages;
+      ok = ok && mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err);
+      const int nb = min(2, (d.K - c0) / 64);
+      if (ok) {
+        const uint32_t st = smem_u32(ring.stage + (size_t)s * ring.stage_bytes);
+        for (int b = 0; b < nb; ++b) {
+          const uint32_t box = st + b * kBoxBytes;
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
+          for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1, a2,
+                    a3);
+            const int kc = kcb + (c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) red[(warp * 16 + (m * 2 + n) * 4 + i) * 32 + lane] = acc[m][n][i];
-  consumer_sync();
-  if (*abort_flag || !ok) return;
-  for (int o = threadIdx.x; o < 16 * 32; o += kConsumerWarps * 32) {
-    const int q = o / 128, i = (o / 32) % 4, l = o % 32;
-    const int m = q >> 1, n = q & 1;
-    float v = 0.f;
-    for (int w = 0; w < kConsumerWarps; ++w) v += red[(w * 16 + q * 4 + i) * 32 + l];
-    const int row = du.n0 + 16 * m + (l >> 2) + 8 * (i >> 1);
-    const int t = 8 * n + 2 * (l & 3) + (i & 1);
-    if (t < a.T && row < du.n1) {
-      if (a.residual) v += __bfloat162float(a.x[(size_t)t * a.D + row]);
-      a.out[(size_t)t * a.D + row] = __float2bfloat16_rn(v);
+            for (int nt = 0; nt < 2; ++nt) {
+              if (nt < ntiles) {
+                uint32_t bh0, bh1, bl0, bl1;
+                ldsm_x2(brow[nt] + (uint32_t)row_chunk(bsw[nt], kc) * 16u, bh0, bh1);
+                ldsm_x2(brow[nt] + (uint32_t)row_chunk(bsw[nt], kc + L / 8) * 16u, bl0, bl1);
+                mma16816(acc[nt], a0, a1, a2, a3, bh0, bh1);
+                mma16816(acc[nt], a0, a1, a2, a3, bl0, bl1);
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ring.empty[s]);
+    }
+    if (!ok) continue;
+    // acc[nt][i]: row 16 warp + lane/4 + 8 (i >> 1), column 8 nt + 2 (lane & 3) + (i & 1)
+    const int r0 = d.rb * kDRows + 16 * warp + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = 8 * nt + 2 * (lane & 3) + (i & 1);
+        const int row = r0 + 8 * (i >> 1);
+        if (col < n) {
+          float* dst = d.shared ? a.Ps + ((size_t)d.q * kTok + col) * a.D
+                                : a.P + ((size_t)d.e * kTok + col) * a.D;
+          dst[row] = acc[nt][i];
+        }
+      }
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// kd_combine: out[t][row] = sum over the shared-expert K parts q of Ps[q][t][row]
+// + sum over t's active experts e, ascending, of P[e][slot][row] (+ x[t][row]);
+// a fixed order, so the result is bitwise reproducible.
+
+__global__ void __launch_bounds__(256) kd_combine(const __grid_constant__ Args a) {
+  __shared__ int list_e[256], list_s[256], n_list;
+  const int t = blockIdx.y, lane = threadIdx.x & 31;
+  pdl_wait();   // partials (kd_down), act (kd_route)
+  if (threadIdx.x < 32) {
+    int n = 0;
+    for (int e0 = 0; e0 < a.E; e0 += 32) {
+      const int e = e0 + lane;
+      bool f = false;
+      int slot = 0;
+      if (e < a.E) {
+        f = __ldcg(a.act + (size_t)t * a.E + e) != 0;
+        for (int tp = 0; tp < t; ++tp) slot += __ldcg(a.act + (size_t)tp * a.E + e) != 0;
+      }
+      const unsigned m = __ballot_sync(kFull, f);
+      if (f) {
+        const int i = n + __popc(m & ((1u << lane) - 1u));
+        list_e[i] = e;
+        list_s[i] = slot;
+      }
+      n += __popc(m);
+    }
+    if (lane == 0) n_list = n;
+  }
+  __syncthreads();
+  const int row = blockIdx.x * 256 + threadIdx.x;
+  if (row >= a.D) return;
+  float v = 0.f;
+  const int nsq = down_nsq(a.d_s);
+  for (int q = 0; q < nsq; ++q) v += __ldcg(a.Ps + ((size_t)q * kTok + t) * a.D + row);
+  const int n = n_list;
+  for (int i = 0; i < n; ++i) v += __ldcg(a.P + ((size_t)list_e[i] * kTok + list_s[i]) * a.D + row);
+  if (a.residual) v += __bfloat162float(a.x[(size_t)t * a.D + row]);
+  a.out[(size_t)t * a.D + row] = __float2bfloat16_rn(v);
 }
 
 }  // namespace dec
