@@ -88,7 +88,7 @@ Plan make_plan(const deco_moe_shape_t& s) {
   }
   if (s.T <= dec::kMaxT) {         // decode path buffers (see decode_kernels.cuh)
     p.hs16 = take((size_t)dec::kTok * s.d_s * 4);         // [16][hi d_s | lo d_s] bf16
-    p.C16 = take(E * dec::kTok * s.d_e * 4);               // [E][16][d_e] fp32
+    p.C16 = take(8 * E * dec::kTok * s.d_e * 4);           // [kp <= 8][E][16][d_e] fp32
     p.P16 = take(E * dec::kTok * s.d_model * 4);           // [E][16][D] fp32
     p.Ps16 = take((size_t)dec::down_nsq(s.d_s) * dec::kTok * s.d_model * 4);   // [nsq][16][D] fp32
   }
@@ -317,7 +317,7 @@ bool decode_eligible(const deco_moe_shape_t& s, int sms) {
   if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT) return false;
   if (s.d_model % 256 || s.d_model > 4096) return false;
   if (s.E > 256 || s.d_e > 256 || s.d_e % 64 || s.d_s % 64 || s.d_s > 2048) return false;
-  if ((s.E + 7) / 8 >= sms) return false;                     // router CTAs leave room
+  if (dec::router_ctas(s.E) + 16 > sms) return false;         // router CTAs leave room
   const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
   if (dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).nstages < 2) return false;
   if (dec::smem_plan(xop, dec::kStageBytes).nstages < 2) return false;
@@ -375,9 +375,10 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
   a.err = reinterpret_cast<int*>(ws + p.err);
   a.out = static_cast<bf16*>(out);
   // kd_down's weight tiles: 128 rows x 64 columns
-  CUtensorMap tmW, tmS;
+  CUtensorMap tmU, tmW, tmS;
   cudaError_t err;
-  if ((err = make_map(&tmW, w.W_down, s.d_e, (uint64_t)s.E * s.d_model, dec::kDRows)) != cudaSuccess ||
+  if ((err = make_map(&tmU, w.W_up, s.d_model, (uint64_t)s.E * s.d_e, dec::kDRows)) != cudaSuccess ||
+      (err = make_map(&tmW, w.W_down, s.d_e, (uint64_t)s.E * s.d_model, dec::kDRows)) != cudaSuccess ||
       (err = make_map(&tmS, w.W_s_down, s.d_s, s.d_model, dec::kDRows)) != cudaSuccess)
     return err;
   const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
@@ -392,7 +393,8 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
   if (err != cudaSuccess) return err;
   prof_mark(1, st);
   prof_mark(6, st);
-  err = launch_dec(dec::kd_up, grid, block, dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).total, pdl, st, a);
+  err = launch_dec(dec::kd_up, grid, block, dec::smem_plan(dec::kTok * dec::x_pitch(s.d_model), dec::kStageBytes).total,
+                   pdl, st, tmU, a);
   if (err != cudaSuccess) return err;
   prof_mark(7, st);
   prof_mark(8, st);

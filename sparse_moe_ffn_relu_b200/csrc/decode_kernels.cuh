@@ -271,7 +271,8 @@ struct Args {
   uint8_t* act;      // [T][E]
   float* u;          // [T][d_e]
   bf16* hs;          // [16 tok][hi d_s | lo d_s], chunk-swizzled rows: SiLU(x W_s_up^T)
-  float* C;          // [E][16 tok][d_e] up-projection g = x W_up[e]^T (active experts)
+  float* C;          // [kp <= 8][E][16 tok][d_e] up-projection g = x W_up[e]^T (active experts),
+                     // partial sums over K parts
   float* P;          // [E][16 slots][D] routed down-projection partials, slot i = the i-th
                      // active token of expert e (ascending)
   float* Ps;         // [ceil(d_s / 256)][16 tok][D] shared down-projection partials
@@ -419,15 +420,18 @@ __device__ __forceinline__ float chunk_gemv(uint32_t xs, uint32_t ws, uint32_t p
 // ---------------------------------------------------------------------------
 // kd_route
 //
-// CTAs [0, Cr) with Cr = ceil(E / 8): router rows, 8 per CTA, one warp each,
-// on CUDA cores with an exact sign decision (see common.cuh).  The remaining
-// CTAs split the rows of [W_bar_up ; W_s_up] evenly and write
-// u = x W_bar_up^T and SiLU(x W_s_up^T) (as hi/lo pairs) for them.
+// CTAs [0, Cr) with Cr = min(E, 64): router rows on CUDA cores with an exact
+// sign decision (see common.cuh), the 8 warps of a CTA splitting each row's
+// columns.  The remaining CTAs split the rows of [W_bar_up ; W_s_up] evenly
+// and write u = x W_bar_up^T and SiLU(x W_s_up^T) (as hi/lo pairs) for them.
+
+// router CTAs of kd_route: one router row each (E <= 64), else several
+__host__ __device__ inline int router_ctas(int E) { return E < 64 ? E : 64; }
 
 __global__ void __launch_bounds__(kThreads, 1) kd_route(const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  __shared__ unsigned long long limbs[kConsumerWarps][kLimbs];   // 1280 B
-  const int Cr = (a.E + 7) / 8;
+  __shared__ unsigned long long limbs[1][kLimbs];
+  const int Cr = router_ctas(a.E);
   const bool router_cta = (int)blockIdx.x < Cr;
   const uint32_t pitch = x_pitch(a.D);
   // operand: x rows, then the 4 KB cross-warp reduction scratch
@@ -442,54 +446,56 @@ __global__ void __launch_bounds__(kThreads, 1) kd_route(const __grid_constant__ 
   pdl_trigger();
 
   if (router_cta) {
-    const int e0 = blockIdx.x * 8, ne = min(8, a.E - e0);
+    // router rows e = blockIdx.x + Cr i; for each row the 8 consumer warps
+    // split the D columns (16-byte chunks), and their partial sums are added
+    // in warp order
+    const int nrow = (a.E - (int)blockIdx.x + Cr - 1) / Cr;
     const uint32_t rowbytes = (uint32_t)a.D * 2;
     const int per = (int)(kStageBytes / rowbytes);   // router rows per stage
+    const int nst = (nrow + per - 1) / per;
     if (warp == kConsumerWarps) {
       if (lane == 0) {
         const uint64_t pol = evict_first_policy();
         stage_x(a, xsm, xbar);
-        for (int k = 0, done = 0; done < ne; ++k) {
-          const int n = min(per, ne - done);
+        for (int k = 0; k < nst; ++k) {
+          const int n = min(per, nrow - k * per);
           mbar_expect_tx(&ring.full[k], n * rowbytes);
-          bulk_g2s(ring.stage + (size_t)k * kStageBytes, a.W_r + (size_t)(e0 + done) * a.D, n * rowbytes,
-                   &ring.full[k], pol);
-          done += n;
+          for (int j = 0; j < n; ++j)
+            bulk_g2s(ring.stage + (size_t)k * kStageBytes + (size_t)j * rowbytes,
+                     a.W_r + (size_t)(blockIdx.x + Cr * (k * per + j)) * a.D, rowbytes, &ring.full[k], pol);
         }
       }
       return;
     }
-    const int nc = a.D / 256;
-    const int n_terms = a.D / 32 + 6;
+    // a value goes through <= 8 ceil(D / 2048) products in its lane, 5
+    // butterfly levels, 7 cross-warp additions and the bias
+    const int n_terms = 8 * ((a.D + 2047) / 2048) + 16;
     const float gm = gamma_f32(n_terms);
     const float bscale = 2.f * gm * (1.f + 2.f * gm);
     const float tiny = float(n_terms) * 2.8025969e-45f;
     bool bad = false;
-    // every consumer warp waits for x and for the stage of the rows of warp
-    // min(warp, ne - 1), so every issued copy is awaited before the CTA exits
-    const bool x_ok = mbar_wait(xbar, 0, abort_flag, a.err);
-    const int myrow = min(warp, ne - 1);
-    const int k = myrow / per, rs = myrow % per;
-    const bool w_ok = x_ok && mbar_wait(&ring.full[k], 0, abort_flag, a.err);
-    if (w_ok && warp < ne) {
-      const int e = e0 + warp;
-      const bf16* wrow = reinterpret_cast<const bf16*>(ring.stage + (size_t)k * kStageBytes + (size_t)rs * rowbytes);
+    // every consumer warp waits for x and for every stage, so every issued
+    // copy is awaited before the CTA exits
+    bool ok = mbar_wait(xbar, 0, abort_flag, a.err);
+    for (int k = 0; k < nst; ++k) ok = ok && mbar_wait(&ring.full[k], 0, abort_flag, a.err);
+    for (int i = 0; i < nrow; ++i) {
+      const int e = blockIdx.x + Cr * i;
+      const bf16* wrow =
+          reinterpret_cast<const bf16*>(ring.stage + (size_t)(i / per) * kStageBytes + (size_t)(i % per) * rowbytes);
       float v[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.f;
-      // each lane: its D/32 products in chunk order (z in v[t], sum |x w| in v[16+t]);
-      // the chunk loop stays rolled so the loop body fits the instruction cache
+      for (int q = 0; q < 32; ++q) v[q] = 0.f;
+      // z partials in v[t], sum |x w| partials in v[16 + t]
+      if (ok) {
 #pragma unroll 1
-      for (int i = 0; i < nc; ++i) {
-        {
+        for (int ch = warp * 32 + lane; ch < a.D / 8; ch += kConsumerWarps * 32) {
           float wv[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(wrow + (size_t)(lane + 32 * i) * 8), wv);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(wrow + (size_t)ch * 8), wv);
 #pragma unroll
           for (int t = 0; t < kTok; ++t) {
             if (t < a.T) {
               float xv[8];
-              bf16x8_to_f32(*reinterpret_cast<const uint4*>(xsm + (size_t)t * pitch + (size_t)(lane + 32 * i) * 16),
-                            xv);
+              bf16x8_to_f32(*reinterpret_cast<const uint4*>(xsm + (size_t)t * pitch + (size_t)ch * 16), xv);
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
                 v[t] = fmaf(xv[q], wv[q], v[t]);
@@ -499,28 +505,35 @@ __global__ void __launch_bounds__(kThreads, 1) kd_route(const __grid_constant__ 
           }
         }
       }
-      const float tot = warp_reduce_scatter<32>(v, lane);   // lane l: value l
-      const float S = __shfl_sync(kFull, tot, (lane + 16) & 31);
-      const float b = a.b_r[e];
-      const int t = lane;
-      const bool mine = t < a.T;
-      const float z = tot + b;
-      const float B = bscale * (S + fabsf(b)) + tiny;
-      const bool sure = fabsf(z) > B;
-      bool on = sure && z > 0.f;
-      // guard band: exact re-evaluation of the sign, one whole warp per score
-      unsigned need = __ballot_sync(kFull, mine && !sure);
-      while (need) {
-        const int tt = __ffs(need) - 1;
-        need &= need - 1;
-        const int sg = exact_sign_warp(reinterpret_cast<const bf16*>(xsm + (size_t)tt * pitch), wrow, a.D, b,
-                                       limbs[warp], &bad);
-        if (lane == tt) on = sg > 0;
+      red[warp * 32 + lane] = warp_reduce_scatter<32>(v, lane);   // lane l: this warp's value l
+      consumer_sync();
+      if (warp == 0 && ok) {
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) tot += red[w * 32 + lane];
+        const float S = __shfl_sync(kFull, tot, (lane + 16) & 31);
+        const float b = a.b_r[e];
+        const int t = lane;
+        const bool mine = t < a.T;
+        const float z = tot + b;
+        const float B = bscale * (S + fabsf(b)) + tiny;
+        const bool sure = fabsf(z) > B;
+        bool on = sure && z > 0.f;
+        // guard band: exact re-evaluation of the sign, the whole warp per score
+        unsigned need = __ballot_sync(kFull, mine && !sure);
+        while (need) {
+          const int tt = __ffs(need) - 1;
+          need &= need - 1;
+          const int sg = exact_sign_warp(reinterpret_cast<const bf16*>(xsm + (size_t)tt * pitch), wrow, a.D, b,
+                                         limbs[0], &bad);
+          if (lane == tt) on = sg > 0;
+        }
+        if (mine) {
+          a.r[(size_t)t * a.E + e] = on ? fmaxf(z, 0.f) : 0.f;
+          a.act[(size_t)t * a.E + e] = on ? 1 : 0;
+        }
       }
-      if (mine) {
-        a.r[(size_t)t * a.E + e] = on ? fmaxf(z, 0.f) : 0.f;
-        a.act[(size_t)t * a.E + e] = on ? 1 : 0;
-      }
+      consumer_sync();   // red is reused by the next row
     }
     if (bad && lane == 0) atomicOr(a.err, 1);
     return;
@@ -576,65 +589,119 @@ __global__ void __launch_bounds__(kThreads, 1) kd_route(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------
-// kd_up: the rows of W_up[e] for the active experts e (in union order), split
-// evenly over the CTAs; writes g = x W_up[e]^T (NormSiLU runs in kd_down).
+// kd_up: g = x W_up[e]^T for the experts some token uses, as fp32 partial
+// sums over K parts.  Units are (expert e of the union, block of 128 rows of
+// W_up[e], K part p of D / kp columns), with kp <= 8 the smallest power of
+// two that gives every CTA at least two units; CTA c takes a contiguous range
+// of them.  Weights arrive as 128 x 64 TMA boxes (two per 32 KB stage, the
+// 128-byte swizzle ldmatrix reads directly), x stays resident in padded
+// shared-memory rows, and consumer warp w multiplies rows 16w..16w+15 of the
+// unit by the 16 token rows.  Results go to C[p][e][t][j]; kd_down adds the
+// K parts in order.  (NormSiLU runs in kd_down.)
 
-__global__ void __launch_bounds__(kThreads, 1) kd_up(const __grid_constant__ Args a) {
+constexpr int kDRows = 128;                  // weight rows per unit (kd_up, kd_down)
+constexpr uint32_t kBoxBytes = kDRows * 128; // 128 rows x 64 bf16 columns
+
+__host__ __device__ inline int up_kparts(int U, int d_e, int D, int G) {
+  const int units = U * ((d_e + kDRows - 1) / kDRows);
+  int kp = 1;
+  while (kp < 8 && D / (2 * kp) >= 256 && units * kp < 2 * G) kp *= 2;
+  return kp;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    kd_up(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint16_t emask[256];
   __shared__ uint8_t ulist[256];
   __shared__ int s_U;
   const uint32_t pitch = x_pitch(a.D);
-  const SmemPlan sp = smem_plan(kTok * pitch + 4096, row_stage_bytes(a.D));
+  const SmemPlan sp = smem_plan(kTok * pitch, kStageBytes);
   Ring ring;
   uint64_t* xbar;
   volatile int* abort_flag;
   unsigned char* smem = ring_setup(smem_raw, sp, ring, xbar, abort_flag);
   unsigned char* xsm = smem + sp.op_off;
-  float* red = reinterpret_cast<float*>(xsm + kTok * pitch);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // x does not depend on the router: stage it before waiting for it
   if (threadIdx.x == 0) stage_x(a, xsm, xbar);
   if (warp < kConsumerWarps) zero_x_tail(a, xsm, threadIdx.x, kConsumerWarps * 32);
-  pdl_wait();          // router outputs and the completion counters
+  pdl_wait();          // router outputs
   pdl_trigger();
   build_union(a, emask, ulist, &s_U);
-  const int nrows = s_U * a.d_e;
-  const int c = blockIdx.x, G = gridDim.x;
-  const int ra = (int)((long long)c * nrows / G), rb = (int)((long long)(c + 1) * nrows / G);
-  const int rc = rows_per_chunk(a.D);
-  const int nchunks = (rb - ra + rc - 1) / rc;
+  const int nrb = (a.d_e + kDRows - 1) / kDRows;
+  const int kp = up_kparts(s_U, a.d_e, a.D, gridDim.x);
+  const int Kp = a.D / kp;
+  const int NU = s_U * nrb * kp;
+  const int u0 = (int)((long long)blockIdx.x * NU / gridDim.x);
+  const int u1 = (int)((long long)(blockIdx.x + 1) * NU / gridDim.x);
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       const uint64_t pol = evict_first_policy();
-      for (int k = 0; k < nchunks; ++k) {
-        const int s = k % ring.nstages;
-        if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
-        const int g0 = ra + k * rc, n = min(rc, rb - g0);
-        mbar_expect_tx(&ring.full[s], (uint32_t)n * a.D * 2);
-        for (int i = 0; i < n; ++i) {
-          const int g = g0 + i;
-          bulk_g2s(ring.stage + (size_t)s * ring.stage_bytes + (size_t)i * pitch,
-                   a.W_up + ((size_t)ulist[g / a.d_e] * a.d_e + g % a.d_e) * a.D, (uint32_t)a.D * 2,
+      int k = 0;
+      for (int u = u0; u < u1; ++u) {
+        const int p = u % kp, rb = (u / kp) % nrb, e = ulist[u / (kp * nrb)];
+        const int row = e * a.d_e + rb * kDRows;
+        for (int c0 = 0; c0 < Kp; c0 += 128, ++k) {
+          const int s = k % ring.nstages;
+          if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
+          const int nb = min(2, (Kp - c0) / 64);
+          mbar_expect_tx(&ring.full[s], (uint32_t)nb * kBoxBytes);
+          for (int b = 0; b < nb; ++b)
+            tma_2d(ring.stage + (size_t)s * ring.stage_bytes + b * kBoxBytes, &tmU, p * Kp + c0 + 64 * b, row,
                    &ring.full[s], pol);
         }
+        if (*abort_flag) break;
       }
     }
-  } else {
-    // the x copies were issued unconditionally: always await them
-    bool ok = mbar_wait(xbar, 0, abort_flag, a.err);
-    for (int k = 0; k < nchunks; ++k) {
+    return;
+  }
+  // the x copies were issued unconditionally: always await them
+  bool ok = mbar_wait(xbar, 0, abort_flag, a.err);
+  const uint32_t x_u32 = smem_u32(xsm);
+  const int ntiles = (a.T + 7) / 8;
+  int k = 0;
+  for (int u = u0; u < u1; ++u) {
+    const int p = u % kp, rb = (u / kp) % nrb, e = ulist[u / (kp * nrb)];
+    float acc[2][4] = {};
+    for (int c0 = 0; c0 < Kp; c0 += 128, ++k) {
       const int s = k % ring.nstages;
       ok = ok && mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err);
-      const float v = chunk_gemv(smem_u32(xsm), smem_u32(ring.stage + (size_t)s * ring.stage_bytes), pitch, a.D,
-                                 warp, lane, red, ok);
-      if (ok && lane == 0) mbar_arrive(&ring.empty[s]);
-      const int o = threadIdx.x;
-      const int t = o >> 3, i = o & 7;
-      const int g = ra + k * rc + i;
-      if (ok && o < 128 && i < rc && g < rb && t < a.T) {
-        const int e = ulist[g / a.d_e];
-        a.C[((size_t)e * kTok + t) * a.d_e + g % a.d_e] = v;
+      const int nb = min(2, (Kp - c0) / 64);
+      if (ok) {
+        const uint32_t st = smem_u32(ring.stage + (size_t)s * ring.stage_bytes);
+        for (int b = 0; b < nb; ++b) {
+          const uint32_t box = st + b * kBoxBytes;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1, a2,
+                    a3);
+            const int kc = (p * Kp + c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              if (nt < ntiles) {
+                uint32_t b0, b1;
+                ldsm_x2(x_u32 + (uint32_t)(8 * nt + (lane & 7)) * pitch + (uint32_t)kc * 16u, b0, b1);
+                mma16816(acc[nt], a0, a1, a2, a3, b0, b1);
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ring.empty[s]);
+    }
+    if (!ok) continue;
+    // acc[nt][i]: row 16 warp + lane/4 + 8 (i >> 1), token 8 nt + 2 (lane & 3) + (i & 1)
+    const int j0 = rb * kDRows + 16 * warp + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 8 * nt + 2 * (lane & 3) + (i & 1);
+        const int j = j0 + 8 * (i >> 1);
+        if (t < a.T && j < a.d_e) a.C[(((size_t)p * a.E + e) * kTok + t) * a.d_e + j] = acc[nt][i];
       }
     }
   }
@@ -657,8 +724,6 @@ __global__ void __launch_bounds__(kThreads, 1) kd_up(const __grid_constant__ Arg
 // as hi/lo in compact slots (slot i = the i-th active token of e).  Results go
 // to P[e][slot][row] and Ps[q][token][row]; kd_combine adds them.
 
-constexpr int kDRows = 128;                  // output rows per unit
-constexpr uint32_t kBoxBytes = kDRows * 128; // 128 rows x 64 bf16 columns
 constexpr int kSq = 256;                     // K columns per shared-expert unit
 
 __host__ __device__ inline int down_nsq(int d_s) { return (d_s + kSq - 1) / kSq; }
@@ -716,6 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   build_union(a, emask, ulist, &s_U);
   const int nrb = a.D / kDRows;
   const int NU = (down_nsq(a.d_s) + s_U) * nrb;
+  const int kp_up = up_kparts(s_U, a.d_e, a.D, gridDim.x);   // kd_up runs on the same grid
   const int u0 = (int)((long long)blockIdx.x * NU / gridDim.x);
   const int u1 = (int)((long long)(blockIdx.x + 1) * NU / gridDim.x);
 
@@ -762,16 +828,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t m = m_e;
           for (int i = 0; i < slot; ++i) m &= m - 1;
           const int t = __ffs(m) - 1;
-          float cv[8];   // d_e <= 256: 8 values per lane
-          float ss = 0.f;
+          // every load of the token's row is issued before the first is used
+          float gp[8][8], uq[8];   // [K part][value], d_e <= 256: 8 values per lane
+#pragma unroll
+          for (int pp = 0; pp < 8; ++pp)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int j = lane + 32 * q;
+              gp[pp][q] = (pp < kp_up && j < a.d_e)
+                              ? __ldcg(a.C + (((size_t)pp * a.E + e) * kTok + t) * a.d_e + j) : 0.f;
+            }
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const int j = lane + 32 * q;
-            cv[q] = 0.f;
-            if (j < a.d_e) {
-              cv[q] = __ldcg(a.C + ((size_t)e * kTok + t) * a.d_e + j) - __ldcg(a.u + (size_t)t * a.d_e + j);
-              ss = fmaf(cv[q], cv[q], ss);
-            }
+            uq[q] = j < a.d_e ? __ldcg(a.u + (size_t)t * a.d_e + j) : 0.f;
+          }
+          float cv[8];
+          float ss = 0.f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float g = 0.f;   // kd_up's K parts, in order (absent parts add an exact 0)
+#pragma unroll
+            for (int pp = 0; pp < 8; ++pp) g += gp[pp][q];
+            cv[q] = g - uq[q];
+            ss = fmaf(cv[q], cv[q], ss);
           }
           ss = warp_sum(ss);
           const float rinv = 1.f / sqrtf(ss / float(a.d_e) + a.eps);
@@ -865,12 +945,16 @@ __global__ void __launch_bounds__(256) kd_combine(const __grid_constant__ Args a
     int n = 0;
     for (int e0 = 0; e0 < a.E; e0 += 32) {
       const int e = e0 + lane;
-      bool f = false;
-      int slot = 0;
+      uint32_t m = 0;   // tokens using e (all flags loaded before any is used)
       if (e < a.E) {
-        f = __ldcg(a.act + (size_t)t * a.E + e) != 0;
-        for (int tp = 0; tp < t; ++tp) slot += __ldcg(a.act + (size_t)tp * a.E + e) != 0;
+        uint8_t fl[kTok];
+#pragma unroll
+        for (int tp = 0; tp < kTok; ++tp) fl[tp] = tp < a.T ? __ldcg(a.act + (size_t)tp * a.E + e) : 0;
+#pragma unroll
+        for (int tp = 0; tp < kTok; ++tp) m |= (fl[tp] ? 1u : 0u) << tp;
       }
+      const bool f = (m >> t) & 1u;
+      const int slot = __popc(m & ((1u << t) - 1u));
       const unsigned m = __ballot_sync(kFull, f);
       if (f) {
         const int i = n + __popc(m & ((1u << lane) - 1u));
