@@ -945,16 +945,16 @@ __global__ void __launch_bounds__(256) kd_combine(const __grid_constant__ Args a
     int n = 0;
     for (int e0 = 0; e0 < a.E; e0 += 32) {
       const int e = e0 + lane;
-      uint32_t m = 0;   // tokens using e (all flags loaded before any is used)
+      uint32_t toks = 0;   // tokens using e (all flags loaded before any is used)
       if (e < a.E) {
         uint8_t fl[kTok];
 #pragma unroll
         for (int tp = 0; tp < kTok; ++tp) fl[tp] = tp < a.T ? __ldcg(a.act + (size_t)tp * a.E + e) : 0;
 #pragma unroll
-        for (int tp = 0; tp < kTok; ++tp) m |= (fl[tp] ? 1u : 0u) << tp;
+        for (int tp = 0; tp < kTok; ++tp) toks |= (fl[tp] ? 1u : 0u) << tp;
       }
-      const bool f = (m >> t) & 1u;
-      const int slot = __popc(m & ((1u << t) - 1u));
+      const bool f = (toks >> t) & 1u;
+      const int slot = __popc(toks & ((1u << t) - 1u));
       const unsigned m = __ballot_sync(kFull, f);
       if (f) {
         const int i = n + __popc(m & ((1u << lane) - 1u));
