@@ -823,12 +823,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t m_e = emask[e];
       n_cur = __popc(m_e);
       if (ok && !*abort_flag) {
-        const float se = a.s[e];
         for (int slot = warp; slot < n_cur; slot += kConsumerWarps) {
           uint32_t m = m_e;
           for (int i = 0; i < slot; ++i) m &= m - 1;
           const int t = __ffs(m) - 1;
           // every load of the token's row is issued before the first is used
+          const float rte = __ldcg(a.r + (size_t)t * a.E + e);
+          const float se = __ldg(a.s + e);
           float gp[8][8], uq[8];   // [K part][value], d_e <= 256: 8 values per lane
 #pragma unroll
           for (int pp = 0; pp < 8; ++pp)
@@ -855,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ss = warp_sum(ss);
           const float rinv = 1.f / sqrtf(ss / float(a.d_e) + a.eps);
-          const float coef = se * __ldcg(a.r + (size_t)t * a.E + e);
+          const float coef = se * rte;
           bf16* row = reinterpret_cast<bf16*>(tile + (size_t)slot * 4 * a.d_e);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
