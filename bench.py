@@ -70,6 +70,26 @@ def peaks():
 
 
 # --------------------------------------------------------------------------
+# ranks: one process per GPU, independent replicas (tokens never interact in
+# an FFN layer); the only cross-rank traffic is the barrier and the max of the
+# timed durations
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's duration (every rank calls this, in the same order)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank processed `steps` steps in at most `ms`."""
+    return world * tokens_per_step * steps / (ms / 1000.0)
+
+
+# --------------------------------------------------------------------------
 # CPU oracle timing (the baseline arm and cpu_baseline)
 
 def oracle_tokens_per_s(budget_s: float, max_steps: int | None = None):
@@ -289,13 +309,9 @@ def main():
         torch.cuda.synchronize()
         barrier()
         clocks = sampler.stop()
-    ms = start.elapsed_time(end)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dist, dev)
     tokens_per_step = sum(DECODE_TS)
-    value = world * tokens_per_step * args.steps / (ms / 1000.0)
+    value = job_tokens_per_s(world, tokens_per_step, args.steps, ms)
 
     # live kernel durations: eager forwards on the rotating weight copies
     kt = {T: {k: [] for k in deco.PREFILL_KERNELS} for T in DECODE_TS}
@@ -354,12 +370,8 @@ def main():
         e2.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms2 = s2.elapsed_time(e2)
-    if dist is not None:
-        t = torch.tensor([ms2], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms2 = float(t.item())
-    e2e_value = world * tokens_per_step * e2e_steps / (ms2 / 1000.0)
+    ms2 = max_over_ranks(s2.elapsed_time(e2), dist, dev)
+    e2e_value = job_tokens_per_s(world, tokens_per_step, e2e_steps, ms2)
     io_bytes = sum(T * base.D * 2 for T in DECODE_TS)
 
     line = {
