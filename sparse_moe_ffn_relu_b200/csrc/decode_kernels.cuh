@@ -941,7 +941,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(256) kd_combine(const __grid_constant__ Args a) {
   __shared__ int list_e[256], list_s[256], n_list;
   const int t = blockIdx.y, lane = threadIdx.x & 31;
-  pdl_wait();   // partials (kd_down), act (kd_route)
+  // The router's outputs are complete: this grid starts only after every CTA
+  // of kd_down started, and kd_down starts only after kd_up passed its wait on
+  // the router.  The token's expert list is built while kd_down finishes.
   if (threadIdx.x < 32) {
     int n = 0;
     for (int e0 = 0; e0 < a.E; e0 += 32) {
@@ -967,6 +969,7 @@ __global__ void __launch_bounds__(256) kd_combine(const __grid_constant__ Args a
     if (lane == 0) n_list = n;
   }
   __syncthreads();
+  pdl_wait();   // the partials (kd_down)
   const int row = blockIdx.x * 256 + threadIdx.x;
   if (row >= a.D) return;
   float v = 0.f;

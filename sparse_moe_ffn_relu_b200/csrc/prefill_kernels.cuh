@@ -925,13 +925,15 @@ __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__
     const float4* sp = reinterpret_cast<const float4*>(S + (size_t)t * D + c);
     const float4 s0 = sp[0], s1 = sp[1];
     float acc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-    int i = 0;
-    for (; i + 4 <= n; i += 4) {
-      uint4 w[4];
+    for (int i = 0; i < n; i += 8) {   // up to 8 rows in flight, added in list order
+      uint4 w[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) w[j] = __ldg(reinterpret_cast<const uint4*>(v + (size_t)list[i + j] * D + c));
+      for (int j = 0; j < 8; ++j)
+        w[j] = i + j < n ? __ldg(reinterpret_cast<const uint4*>(v + (size_t)list[i + j] * D + c))
+                         : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
+        if (i + j >= n) break;
         const uint32_t ws4[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
@@ -939,16 +941,6 @@ __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__
           acc[2 * h] += f.x;
           acc[2 * h + 1] += f.y;
         }
-      }
-    }
-    for (; i < n; ++i) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(v + (size_t)list[i] * D + c));
-      const uint32_t ws4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws4[h]));
-        acc[2 * h] += f.x;
-        acc[2 * h + 1] += f.y;
       }
     }
     if (residual) {
@@ -977,6 +969,7 @@ __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__
 
 constexpr int kTabThreads = 128;
 constexpr int kTabWarps = kTabThreads / 32;
+constexpr int kTabStage = 8192;   // block counts staged in shared memory (32 KB) up to this size
 
 // active flags of token t for experts e0..e0+31 as bits (independent loads)
 __device__ __forceinline__ uint32_t row_bits(const uint8_t* row, bool ok, int E, int e0) {
@@ -1046,12 +1039,19 @@ __global__ void __launch_bounds__(kTabThreads) k_tab_scatter(const uint8_t* __re
                                                              int4* tiles, int* n_tiles, int tile_rows) {
   __shared__ int cnt[256], off[256], base[256], ntl[256];
   __shared__ int wc[kTabWarps][256];
+  __shared__ int bc[kTabStage];   // the block counts, when they fit
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // every block: counts per expert and the number of pairs in earlier blocks
+  // (the [nb][E] block counts are staged with coalesced loads when they fit)
+  const bool staged = nb * E <= kTabStage;
+  if (staged) {
+    for (int i = threadIdx.x; i < nb * E; i += kTabThreads) bc[i] = blk_counts[i];
+    __syncthreads();
+  }
   for (int e = threadIdx.x; e < E; e += kTabThreads) {
     int c = 0, before = 0;
     for (int b = 0; b < nb; ++b) {
-      const int v = blk_counts[(size_t)b * E + e];
+      const int v = staged ? bc[b * E + e] : blk_counts[(size_t)b * E + e];
       c += v;
       if (b < (int)blockIdx.x) before += v;
     }
