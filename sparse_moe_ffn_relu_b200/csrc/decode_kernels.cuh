@@ -32,11 +32,11 @@
 // reads can use directly (an XOR swizzle of the 16-byte chunks inside each
 // row).
 //
-// Arithmetic: the projections are tiny dense contractions (16 tokens x 8..64
-// weight rows x K) done with mma.sync m16n8k16 (bf16 in, fp32 accumulate): a
-// tensor-core instruction per 16x8x16 tile keeps the instruction count far
-// below the memory time.  (tcgen05's smallest tile, M = 64, would make the
-// tensor core read several times the shared memory these tiles occupy.)
+// Arithmetic: the projections are thin dense contractions (up to 16 tokens
+// against 8-row chunks or 128-row units of weights) done with mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate) with the weights as A: a tensor-core
+// instruction per 16x8x16 tile keeps the instruction count far below the
+// memory time, which is the bound at these batch sizes.
 // Intermediates fed back into a contraction (the shared expert's hidden
 // activations and the scaled NormSiLU outputs) are stored as a bf16 pair
 // hi + lo with lo = bf16(v - hi), and both halves are multiplied, so they
@@ -63,7 +63,6 @@ constexpr int kMaxStages = 8;
 constexpr size_t kSmemLimit = 232448;          // 227 KB opt-in per CTA on sm_100
 constexpr long long kWaitCycles = 2000000000ll;  // ~1 s at 1.9 GHz
 constexpr int kErrTimeout = 2;
-constexpr int kKB = 64;                        // columns per weight tile (128 B of bf16)
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -178,19 +177,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // different bank groups.
 __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk) {
   return base + (uint32_t)row * 128u + ((uint32_t)(chunk ^ (row & 7)) << 4);
-}
-__host__ __device__ constexpr uint32_t tile_bytes(int rows) {   // rows x 128 B, 1024-B multiple
-  return (uint32_t)((rows * 128 + 1023) / 1024 * 1024);
-}
-
-// ldmatrix address of this lane for the A operand (16 token rows x 16 columns
-// at k-step ks of a 64-column tile)
-__device__ __forceinline__ uint32_t a_addr(uint32_t tile, int lane, int ks) {
-  return swz(tile, (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4));
-}
-// ... for the B operand, rows r0..r0+15 (x4: two n-tiles) or r0..r0+7 (x2)
-__device__ __forceinline__ uint32_t b_addr(uint32_t tile, int lane, int ks, int r0) {
-  return swz(tile, r0 + (lane & 7) + (lane >> 4) * 8, 2 * ks + ((lane >> 3) & 1));
 }
 
 // ---------------------------------------------------------------------------
