@@ -42,7 +42,7 @@ DECODE_KERNELS = ("route", "up", "down", "combine")   # the decode path's launch
 # kernels on the edge layer (profiles/decode_kernels_edge_decode_t16.md); a kernel
 # changed since its capture has no entry
 NCU_DRAM_BYTES = {("route", 16): 5_638_144, ("up", 16): 65_105_152 + 562_432,
-                  ("down", 16): 70_251_520 + 1_234_944, ("combine", 16): 2_366_208}
+                  ("down", 16): 70_251_520 + 1_234_944}
 METRIC = "MoE-layer tokens/s (decode)"
 
 
