@@ -414,8 +414,9 @@ def main():
 
 def profile_only(args):
     """Eager forward passes of the edge layer at one batch size, for ncu:
-    warmup forwards first, then `steps` more; kernels in launch order
-    route, up, down (decode path) or route, count, scatter, up, down."""
+    warmup forwards first, then `steps` more.  Kernels in launch order:
+    kd_route, kd_up, kd_down, kd_combine (T <= 16); k_router, k_router_exact,
+    k_tab_count, k_tab_scatter, kp_gemm<0..3>, k_combine (T > 16)."""
     import torch
 
     import sparse_moe_ffn_relu_b200 as deco
