@@ -123,3 +123,29 @@ def test_routing_mean_dense_reject_bad_arguments(deco):
                                       0x5000, 8, None) == 3
     code = ctypes.c_int(0)
     assert lib.deco_moe_device_error(None, ctypes.byref(code), None) == 1
+
+
+def test_workspace_follows_the_kernel_path(deco):
+    """Host-side path choice seen through the workspace plan: a bf16 batch of
+    more than 16 tokens with d_e <= 256 takes the tensor-core path, whose
+    workspace holds an fp16 row of D values per possible (token, expert) pair;
+    fp32 batches and d_e = 512 take the general kernels, which do not."""
+    T, D, E = 32, 2048, 64
+    rc, n_bf16 = _ws(deco, _shape(deco, T=T))
+    rc2, n_f32 = _ws(deco, _shape(deco, T=T, dtype=deco.DECO_F32))
+    rc3, n_wide = _ws(deco, _shape(deco, T=T, d_e=512))
+    assert rc == rc2 == rc3 == 0
+    assert n_bf16 >= T * E * D * 2
+    assert n_f32 < T * E * D * 2 and n_wide < T * E * D * 2 + T * E * 512 * 4
+
+
+def test_decode_workspaces_fit_the_static_scratch(deco):
+    """Every decode batch of the two bench layers fits the built-in scratch of
+    deco_moe_forward_static, whose size the header and the binding agree on."""
+    text = open(os.path.join(ROOT, "include", "deco_moe.h")).read()
+    m = re.search(r"#define DECO_STATIC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == deco.STATIC_SCRATCH_BYTES
+    for T in (1, 4, 16):
+        for D, E, d_s in ((2048, 64, 1024), (4096, 128, 2048)):
+            rc, n = _ws(deco, _shape(deco, T=T, D=D, E=E, d_s=d_s))
+            assert rc == 0 and n <= deco.STATIC_SCRATCH_BYTES, (T, D, E, n)
