@@ -4,7 +4,8 @@
 // most 16 tokens, and only the routed experts that some token activates need
 // to be read (the paper's point about sparse activation saving memory access,
 // "DECO: Sparse Mixture-of-Experts with Dense-Comparable Performance on
-// End-Side Devices", §1 and §5).  Three kernels stream the weights once:
+// End-Side Devices", §1 and §5).  Three kernels stream the weights once and
+// a fourth adds the partial results:
 //
 //   kd_route  router rows W_r (exact activation decisions, CUDA cores), and
 //             the mean up-projection W_bar_up and shared up-projection W_s_up
@@ -180,7 +181,7 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk) {
 }
 
 // ---------------------------------------------------------------------------
-// Ring of weight stages shared by the three kernels.
+// Ring of weight stages shared by the three streaming kernels.
 
 struct Ring {
   uint64_t* full;    // [kMaxStages]
