@@ -54,5 +54,5 @@ shared expert's activation and the router bias.
 from .deco import (  # noqa: F401
     to_f64, round_bf16, round_storage, silu, router_logits, route, routing_tables,
     mean_up, norm_silu, expert_output, shared_expert, layer_forward,
-    layer_forward_tokens, dense_ffn, stack_forward, topk_route,
+    layer_forward_tokens, dense_ffn, stack_forward, topk_route, exact_logit,
 )

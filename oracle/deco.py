@@ -92,20 +92,51 @@ def route(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray):
     return z, active, r
 
 
+def exact_logit(x_t: np.ndarray, w: np.ndarray, b: float):
+    """The exact rational value of b + sum_k x_t[k] w[k] (a Fraction)."""
+    from fractions import Fraction
+    total = Fraction(float(b))
+    for xv, wv in zip(x_t.tolist(), w.tolist()):
+        total += Fraction(xv) * Fraction(wv)
+    return total
+
+
 def topk_route(x: np.ndarray, W_r: np.ndarray, b_r: np.ndarray, k: int):
     """TopK routing baseline at a fixed k: the k largest logits per token
     (ties to the lower expert index), weights ReLU(z) of the chosen ones.
 
     The comparison point of [arXiv] §5 ("TopK ... conventional TopK" at the
     same average activation ratio).  Returns (z, active, r) like `route`.
+
+    Ranking is by the exact logit.  The correctly rounded sums of
+    `router_logits` keep the order of distinct exact values except that two
+    of them may round to the same fp64 number; such ties are settled on the
+    exact rational values, and only exactly equal logits go to the lower
+    index.
     """
+    from functools import cmp_to_key
     T = x.shape[0]
     E = W_r.shape[0]
     z = np.stack([router_logits(x[t], W_r, b_r) for t in range(T)]) if T else \
         np.zeros((0, E))
     active = np.zeros((T, E), dtype=bool)
     for t in range(T):
-        order = sorted(range(E), key=lambda e: (-z[t, e], e))
+        exact = {}
+
+        def value(e):
+            if e not in exact:
+                exact[e] = exact_logit(x[t], W_r[e], b_r[e])
+            return exact[e]
+
+        def cmp(e, f):   # negative: e ranks above f
+            if z[t, e] != z[t, f]:
+                return -1 if z[t, e] > z[t, f] else 1
+            ve, vf = value(e), value(f)
+            if ve != vf:
+                return -1 if ve > vf else 1
+            return -1 if e < f else (1 if e > f else 0)
+
+        order = sorted(range(E), key=cmp_to_key(cmp))
         for e in order[:k]:
             active[t, e] = True
     r = np.where(active, np.maximum(z, 0.0), 0.0)

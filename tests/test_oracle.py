@@ -308,3 +308,43 @@ def test_topk_route_picks_k_largest():
     for t in range(9):
         chosen = np.sort(np.nonzero(active[t])[0])
         np.testing.assert_array_equal(chosen, np.sort(np.argsort(-z[t], kind="stable")[:3]))
+
+
+def test_topk_route_ranks_by_exact_value():
+    # logits 1 and 1 + 2^-60 round to the same fp64 number; the exact order
+    # decides (expert 1 is larger although its index is higher), and an exact
+    # tie (experts 2 and 3) goes to the lower index
+    x = np.zeros((1, 4))
+    x[0, 0], x[0, 1] = 1.0, 2.0 ** -30
+    W = np.zeros((4, 4))
+    W[0, 0] = 1.0
+    W[1, 0], W[1, 1] = 1.0, 2.0 ** -30
+    W[2, 0], W[2, 2] = 0.5, 1.0
+    W[3, 0], W[3, 3] = 0.5, 2.0
+    x[0, 2], x[0, 3] = 0.25, 0.125
+    b = np.zeros(4)
+    z, act, r = O.topk_route(x, W, b, 1)
+    assert z[0, 0] == z[0, 1] == 1.0                     # tie in fp64
+    assert act[0].tolist() == [False, True, False, False]
+    z, act, r = O.topk_route(x, W, b, 3)
+    assert z[0, 2] == z[0, 3] == 0.75                    # an exact tie
+    assert act[0].tolist() == [True, True, True, False]
+    assert r[0, 1] == 1.0 and r[0, 3] == 0.0
+
+
+def test_topk_route_matches_brute_force_exact_ranking():
+    # small-integer operands: every logit is an exact integer, many tie
+    from fractions import Fraction
+    rng = np.random.default_rng(3)
+    x = rng.integers(-3, 4, size=(12, 6)).astype(float)
+    W = rng.integers(-2, 3, size=(9, 6)).astype(float)
+    b = rng.integers(-2, 3, size=9).astype(float)
+    for k in (1, 3, 9):
+        _, act, r = O.topk_route(x, W, b, k)
+        for t in range(12):
+            vals = [sum(Fraction(a) * Fraction(c) for a, c in zip(x[t], W[e])) + Fraction(b[e])
+                    for e in range(9)]
+            want = sorted(range(9), key=lambda e: (-vals[e], e))[:k]
+            assert sorted(np.nonzero(act[t])[0].tolist()) == sorted(want)
+            for e in range(9):
+                assert r[t, e] == (max(float(vals[e]), 0.0) if e in want else 0.0)
