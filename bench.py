@@ -16,9 +16,11 @@ replicas (the layer shards by token with no exchange): value = all ranks'
 tokens / max time ("weak" scaling).
 
 Extra keys: roofline of the dominant kernel (live CUDA-event kernel times
-from an instrumented replay of the same graphs), e2e through the public API
-with pinned host buffers, clocks sampled during the run, the CPU oracle as
-the baseline, and (rank 0, one GPU) prefill and dense-FFN comparisons.
+from eager forwards on the rotating copies), e2e through the public API with
+pinned host buffers, clocks sampled during the run, the CPU oracle as the
+baseline (one thread, and all host cores), and (rank 0, one GPU) prefill,
+the activation-ratio sweep against the equal-parameter dense FFN, TopK vs
+ReLU routing, and the 8-layer d_model-4096 stack.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -37,13 +39,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 DECODE_TS = (1, 4, 16)
-DECODE_KERNELS = ("route", "up", "down", "combine")   # the decode path's launches per forward
-# DRAM bytes (read + write) per launch from an ncu capture of the current decode
-# kernels on the edge layer (profiles/decode_kernels_edge_decode_t16.md); a kernel
-# changed since its capture has no entry
-NCU_DRAM_BYTES = {("route", 16): 5_638_144, ("up", 16): 65_105_152 + 562_432,
-                  ("down", 16): 70_251_520 + 1_234_944}
 METRIC = "MoE-layer tokens/s (decode)"
+# DRAM bytes (read + write) per launch of the decode kernel at T = 16 from an
+# ncu capture of the current kernel (None until one is taken; a kernel changed
+# since its capture has no entry)
+NCU_DRAM_BYTES = {}
 
 
 def parse():
@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--profile-tokens", type=int, default=0,
                     help="profiling mode: only run eager forward passes of the edge layer at this "
                          "batch size (warmup + steps), print nothing; for ncu captures")
+    ap.add_argument("--profile-dense", action="store_true",
+                    help="with --profile-tokens: the equal-parameter dense FFN instead")
     return ap.parse_args()
 
 
@@ -92,32 +94,90 @@ def job_tokens_per_s(world: int, tokens_per_step: int, steps: int, ms: float) ->
 # --------------------------------------------------------------------------
 # CPU oracle timing (the baseline arm and cpu_baseline)
 
-def oracle_tokens_per_s(budget_s: float, max_steps: int | None = None):
-    """Time the fp64 oracle on whole steps of the decode workload (21 tokens),
-    single-threaded, until `budget_s` of CPU work (or max_steps) is done."""
-    import numpy as np
-    from threadpoolctl import threadpool_limits
-
+def _oracle_layer():
     import oracle as O
     from synth import CONFIGS, make_layer
-
     cfg = CONFIGS["edge_decode_t16"]
     L = make_layer(cfg["shape"], cfg["seed"])
     L64 = {k: O.to_f64(v) for k, v in L.items()}
     L64["W_bar_up"] = O.mean_up(L64["W_up"], "bf16")
     x = L64.pop("x")
+    return x, L64, cfg["shape"].eps
+
+
+def oracle_tokens_per_s(budget_s: float, max_steps: int | None = None):
+    """Time the fp64 oracle on whole steps of the decode workload (21 tokens),
+    single-threaded, until `budget_s` of CPU work (or max_steps) is done."""
+    from threadpoolctl import threadpool_limits
+
+    import oracle as O
+    x, L64, eps = _oracle_layer()
     steps = tokens = 0
     with threadpool_limits(limits=1):
         t0 = time.perf_counter()
         while True:
             for T in DECODE_TS:
-                O.layer_forward_tokens(x[:T], L64, cfg["shape"].eps)
+                O.layer_forward_tokens(x[:T], L64, eps)
                 tokens += T
             steps += 1
             el = time.perf_counter() - t0
             if el >= budget_s or (max_steps and steps >= max_steps):
                 break
     return tokens / el, steps, tokens, el
+
+
+_POOL_LAYER = None
+
+
+def _pool_init():
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(limits=1)
+
+
+def _pool_tokens(args):
+    import oracle as O
+    x, L64, eps = _POOL_LAYER
+    toks, reps = args
+    for _ in range(reps):
+        O.layer_forward_tokens(x, L64, eps, toks)
+    return len(toks) * reps
+
+
+def oracle_all_cores(budget_s: float = 10.0):
+    """The same oracle on every host core: worker processes (forked before any
+    CUDA call, sharing the fp64 layer copy-on-write) each evaluate tokens of
+    the T = 16 batch, one thread each.  Returns tokens/s, workers, sample."""
+    import multiprocessing as mp
+    global _POOL_LAYER
+    _POOL_LAYER = _oracle_layer()
+    n = max(1, min(os.cpu_count() or 1, 64))
+    # calibrate: one token's cost on one core
+    import oracle as O
+    x, L64, eps = _POOL_LAYER
+    t0 = time.perf_counter()
+    O.layer_forward_tokens(x, L64, eps, [0])
+    per_tok = max(time.perf_counter() - t0, 1e-3)
+    reps = max(1, int(budget_s / per_tok / 16))
+    work = [([i % 16 for i in range(w, w + 16)], reps) for w in range(n)]
+    ctx = mp.get_context("fork")
+    with ctx.Pool(n, initializer=_pool_init) as pool:
+        pool.map(_pool_tokens, [([0], 1)] * n)          # warm the workers
+        t0 = time.perf_counter()
+        done = sum(pool.map(_pool_tokens, work))
+        el = time.perf_counter() - t0
+    _POOL_LAYER = None
+    return done / el, n, f"{n} processes x {reps} x 16 tokens of the edge_decode layer, {el:.1f} s"
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args, rank, world):
@@ -195,19 +255,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(busy)}
 
 
-def layer_bytes(shape, union_experts: int):
-    """Algorithmic HBM bytes per kernel for one decode forward: the weights
-    each kernel must read (only the union of active experts) plus x in / out."""
-    D, E, d_e, d_s, T = shape.D, shape.E, shape.d_e, shape.d_s, shape.T
-    es = 2 if shape.dtype == "bf16" else 4
-    return {
-        "route": ((E + d_e + d_s) * D + T * D) * es,
-        "count": 0,
-        "scatter": 0,
-        "up": (union_experts * d_e * D + T * D) * es,
-        "down": (union_experts * D * d_e + D * d_s) * es,
-        "combine": 2 * T * D * es,
-    }
+def layer_bytes(T, D, E, d_e, d_s, union_experts: int, es: int = 2) -> int:
+    """Algorithmic HBM bytes of one decode forward: every weight it must read
+    (W_r, W_bar_up, W_s_up, W_s_down, and W_up / W_down of the union of the
+    batch's active experts only), x in and out, b_r and s."""
+    return (((E + d_e + d_s) * D + union_experts * 2 * d_e * D + D * d_s + 2 * T * D) * es
+            + 8 * E)
+
+
+def dense_bytes(T, D, d_ff, es: int = 2) -> int:
+    return (2 * d_ff * D + 2 * T * D) * es
+
+
+def layer_flops(n_t, D, E, d_e, d_s) -> float:
+    """Algorithmic FLOPs of a prefill forward: router, mean and shared
+    up-projections for every token, routed up and down per active pair, the
+    shared down-projection (no padding counted)."""
+    T = len(n_t)
+    return float(T * (2 * D * E + 2 * D * d_e + 4 * D * d_s) + 4 * D * d_e * sum(n_t))
 
 
 def main():
@@ -221,12 +286,15 @@ def main():
     if args.profile_tokens:
         profile_only(args)
         return
+    # the all-core oracle timing forks worker processes: before any CUDA call
+    cpu_all = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        cpu_all = oracle_all_cores()
 
-    import numpy as np
     import torch
 
     import sparse_moe_ffn_relu_b200 as deco
-    from synth import CONFIGS, LayerShape, make_layer
+    from synth import CONFIGS, make_layer
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -276,15 +344,6 @@ def main():
             step(G)
         graphs.append(g)
 
-    # events around every kernel of every forward (eager calls: the library
-    # records them with cudaEventRecord between its launches; PDL is off then)
-    nk = len(deco.PREFILL_KERNELS)
-    ev = {T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for T in DECODE_TS}
-    for es in ev.values():          # torch creates CUDA events lazily, on first record
-        for e in es:
-            e.record(stream)
-    torch.cuda.synchronize()
-
     sampler = ClockSampler(local)
     with torch.cuda.stream(stream):
         for i in range(max(3, args.warmup)):
@@ -313,8 +372,17 @@ def main():
     tokens_per_step = sum(DECODE_TS)
     value = job_tokens_per_s(world, tokens_per_step, args.steps, ms)
 
-    # live kernel durations: eager forwards on the rotating weight copies
-    kt = {T: {k: [] for k in deco.PREFILL_KERNELS} for T in DECODE_TS}
+    # live kernel durations: eager forwards on the rotating weight copies; the
+    # decode path is one kernel (timing slot "layer")
+    names = deco.ALL_SLOTS
+    ev = {T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))] for T in DECODE_TS}
+    with torch.cuda.stream(stream):
+        for es in ev.values():          # torch creates CUDA events lazily, on first record
+            for e in es:
+                e.record(stream)
+    torch.cuda.synchronize()
+    kt = {T: [] for T in DECODE_TS}
+    slot = names.index("layer")
     with torch.cuda.stream(stream):
         for i in range(min(args.steps, 60) + 3):
             G = copies[i % n_copies]
@@ -326,26 +394,21 @@ def main():
             if i < 3:
                 continue
             for T in DECODE_TS:
-                for j, k in enumerate(deco.PREFILL_KERNELS):
-                    kt[T][k].append(ev[T][2 * j].elapsed_time(ev[T][2 * j + 1]))
+                kt[T].append(ev[T][2 * slot].elapsed_time(ev[T][2 * slot + 1]))
     # routing statistics -> union of active experts per batch
-    union, ratio = {}, []
+    union, ratio, per_tok = {}, [], []
     for T in DECODE_TS:
         rt = deco.routing(xs[T], G0)
         act = rt["active"].bool()
         union[T] = int(act.any(dim=0).sum().item())
         ratio.append(float(act.float().mean().item()))
-    bytes_k = {T: layer_bytes(LayerShape(T, base.D, base.E, base.d_e, base.d_s, base.dtype), union[T])
-               for T in DECODE_TS}
-    mean_ms = {T: {k: statistics.mean(v) for k, v in kt[T].items()} for T in DECODE_TS}
-    tot_k = {k: sum(mean_ms[T][k] for T in DECODE_TS) for k in DECODE_KERNELS}
-    # the dominant kernel (most time per step), at the largest decode batch
-    dom = max(tot_k, key=tot_k.get)
+        per_tok += act.float().mean(dim=1).tolist()
+    D, E, d_e, d_s = base.D, base.E, base.d_e, base.d_s
+    bytes_T = {T: layer_bytes(T, D, E, d_e, d_s, union[T]) for T in DECODE_TS}
+    kms = {T: statistics.mean(kt[T]) for T in DECODE_TS}
     T_r = max(DECODE_TS)
-    dom_bytes = bytes_k[T_r][dom]
-    dom_ms = mean_ms[T_r][dom]
-    achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
-    step_bytes = sum(sum(b.values()) for b in bytes_k.values())
+    achieved = bytes_T[T_r] / (kms[T_r] / 1000.0) / 1e9
+    step_bytes = sum(bytes_T.values())
     layer_gbs = step_bytes / (ms / args.steps / 1000.0) / 1e9
 
     # end to end through the public API: pinned host x -> device -> layer -> host
@@ -379,22 +442,26 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "edge_decode", "T": list(DECODE_TS), "d_model": base.D, "E": base.E,
-                   "d_e": base.d_e, "d_s": base.d_s, "storage": "bf16", "accumulate": "fp32",
+        "config": {"workload": "edge_decode", "T": list(DECODE_TS), "d_model": D, "E": E,
+                   "d_e": d_e, "d_s": d_s, "storage": "bf16", "accumulate": "fp32",
                    "mean_activation": round(statistics.mean(ratio), 4),
+                   "min_token_activation": round(min(per_tok), 4),
+                   "max_token_activation": round(max(per_tok), 4),
+                   "zero_expert_tokens": int(sum(1 for v in per_tok if v == 0.0)),
                    "union_experts": {str(T): union[T] for T in DECODE_TS},
                    "l2": f"rotating {n_copies} weight copies ({wbytes / 1e6:.0f} MB each) > 3x L2",
                    "cuda_graph": True, "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": dom, "T": T_r, "achieved": achieved, "peak": P["hbm"],
-                     "unit": "GB/s", "frac": achieved / P["hbm"], "traffic": NCU_DRAM_BYTES.get((dom, T_r)),
-                     "algorithmic_bytes": dom_bytes,
+        "roofline": {"bound": "hbm", "kernel": "kd_layer", "T": T_r, "achieved": achieved, "peak": P["hbm"],
+                     "unit": "GB/s", "frac": achieved / P["hbm"], "traffic": NCU_DRAM_BYTES.get(("layer", T_r)),
+                     "algorithmic_bytes": bytes_T[T_r],
                      "peak_source": P["src"], "layer_achieved_gbs": layer_gbs,
                      "layer_frac": layer_gbs / P["hbm"],
-                     "kernel_ms_by_T": {str(T): {k: round(mean_ms[T][k], 4) for k in DECODE_KERNELS}
-                                        for T in DECODE_TS}},
+                     "kernel_us_by_T": {str(T): round(1000 * kms[T], 2) for T in DECODE_TS},
+                     "frac_by_T": {str(T): round(bytes_T[T] / (kms[T] / 1e3) / 1e9 / P["hbm"], 4)
+                                   for T in DECODE_TS}},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
                 "d2h_bytes_per_step": io_bytes},
-        "gpu_launches": args.steps * len(DECODE_TS) * len(DECODE_KERNELS),
+        "gpu_launches": args.steps * len(DECODE_TS),
         "clocks": clocks,
     }
     if rank == 0 and world == 1:
@@ -402,6 +469,9 @@ def main():
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{st} steps ({tok} tokens) of the edge_decode workload, "
                                           f"{el:.1f} s, numpy fp64, one thread"}
+        if cpu_all is not None:
+            line["cpu_baseline_all_cores"] = {"value": cpu_all[0], "unit": "tokens/s", "cores": cpu_all[1],
+                                              "kind": "oracle", "cpu": cpu_model(), "sample": cpu_all[2]}
         if not args.no_extras:
             line["extras"] = extras(deco, dev, stream, P)
     if rank == 0:
@@ -415,13 +485,21 @@ def main():
 def profile_only(args):
     """Eager forward passes of the edge layer at one batch size, for ncu:
     warmup forwards first, then `steps` more.  Kernels in launch order:
-    kd_route, kd_up, kd_down, kd_combine (T <= 16); k_router, k_router_exact,
-    k_tab_count, k_tab_scatter, kp_gemm<0..3>, k_combine (T > 16)."""
+    kd_layer (T <= 16); k_router, k_router_exact, k_tab_count, k_tab_scatter,
+    kp_gemm<0..3>, k_combine (T > 16).  --profile-dense: the dense FFN."""
     import torch
 
     import sparse_moe_ffn_relu_b200 as deco
-    from synth import CONFIGS, LayerShape, make_layer
+    from synth import CONFIGS, LayerShape, make_dense, make_layer
     base = CONFIGS["edge_decode_t16"]["shape"]
+    if args.profile_dense:
+        Dn = make_dense(args.profile_tokens, base.D, base.d_s + base.E * base.d_e, "bf16", 7)
+        x, W1, W2 = Dn["x"].cuda(), Dn["W1"].cuda(), Dn["W2"].cuda()
+        out = torch.empty_like(x)
+        for _ in range(args.warmup + args.steps):
+            deco.dense_ffn(x, W1, W2, out=out)
+        torch.cuda.synchronize()
+        return
     shape = LayerShape(args.profile_tokens, base.D, base.E, base.d_e, base.d_s, base.dtype)
     L = make_layer(shape, CONFIGS["edge_decode_t16"]["seed"])
     G = {k: v.cuda() for k, v in L.items()}
@@ -433,12 +511,71 @@ def profile_only(args):
     torch.cuda.synchronize()
 
 
-def extras(deco, dev, stream, P):
-    """Prefill (T=4096) and dense-FFN comparisons on one GPU."""
-    import torch
+# --------------------------------------------------------------------------
+# extras (rank 0, one GPU)
 
-    from synth import CONFIGS, make_dense, make_layer
+def _time_graphs(torch, stream, fns, reps=100):
+    """Mean ms of one call of each fn in `fns` (one per weight copy), captured
+    in CUDA graphs and replayed in rotation, so consecutive calls read
+    different copies."""
+    graphs = []
+    with torch.cuda.stream(stream):
+        for fn in fns:
+            fn()
+        torch.cuda.synchronize()
+        for fn in fns:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs.append(g)
+        for i in range(3 * len(graphs)):
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for i in range(reps):
+            graphs[i % len(graphs)].replay()
+        e.record(stream)
+        torch.cuda.synchronize()
+    for g in graphs:
+        del g
+    return s.elapsed_time(e) / reps
+
+
+def _time_eager(torch, stream, fn, n=10):
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(n):
+            fn()
+        e.record(stream)
+        torch.cuda.synchronize()
+    return s.elapsed_time(e) / n
+
+
+def _copies(torch, G, n):
+    return [G] + [{k: v.clone() for k, v in G.items()} for _ in range(n - 1)]
+
+
+def extras(deco, dev, stream, P):
+    import torch
     out = {}
+    out["prefill_t4096"] = extra_prefill(deco, dev, stream, P, torch)
+    out["ratio_sweep"] = extra_sweep(deco, dev, stream, P, torch)
+    out["topk_vs_relu"] = extra_topk(deco, dev, stream, P, torch)
+    out["stack_8_layers_d4096"] = extra_stack(deco, dev, stream, P, torch)
+    out["context"] = ("the pages report model-level decode speedups of DECO's kernel over dense "
+                      "inference of 3.00x (Jetson AGX Orin) and 2.58x (RTX 4090), through FR-Spec on "
+                      "Spec-Bench; other hardware and a whole model, not this layer")
+    return out
+
+
+def extra_prefill(deco, dev, stream, P, torch):
+    """Config 3: the edge layer at T = 4096 with per-token activation jitter."""
+    from synth import CONFIGS, make_layer
     cfg = CONFIGS["edge_prefill_t4096"]
     shape = cfg["shape"]
     L = make_layer(shape, cfg["seed"], jitter=cfg["jitter"], zero_every=cfg["zero_every"])
@@ -446,29 +583,15 @@ def extras(deco, dev, stream, P):
     G["W_bar_up"] = deco.mean_up(G["W_up"])
     ws = deco.alloc_workspace(deco.layer_shape(G["x"], G), dev)
     o = torch.empty_like(G["x"])
-
-    def timeit(fn, n=10):
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                fn()
-            torch.cuda.synchronize()
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record(stream)
-            for _ in range(n):
-                fn()
-            e.record(stream)
-            torch.cuda.synchronize()
-        return s.elapsed_time(e) / n
-
-    ms = timeit(lambda: deco.forward(G["x"], G, out=o, workspace=ws))
+    ms = _time_eager(torch, stream, lambda: deco.forward(G["x"], G, out=o, workspace=ws))
     act = deco.routing(G["x"], G)["active"].bool()
-    n_t = act.sum(dim=1).double()
+    n_t = act.sum(dim=1).tolist()
     D, E, de, ds = shape.D, shape.E, shape.d_e, shape.d_s
-    flops = float((2 * D * E + 2 * D * de + n_t * 4 * D * de + 4 * D * ds).sum())
+    flops = layer_flops(n_t, D, E, de, ds)
     # per-kernel device time, eager calls with events between the kernels
-    names = deco.PREFILL_KERNELS
+    names = deco.ALL_SLOTS
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]
-    kt = {k: [] for k in names}
+    kt = {k: [] for k in deco.PREFILL_KERNELS}
     with torch.cuda.stream(stream):
         for e in ev:
             e.record(stream)
@@ -476,39 +599,197 @@ def extras(deco, dev, stream, P):
         for _ in range(6):
             deco.forward(G["x"], G, out=o, workspace=ws)
             stream.synchronize()
-            for j, k in enumerate(names):
+            for j, k in enumerate(deco.PREFILL_KERNELS):
                 kt[k].append(ev[2 * j].elapsed_time(ev[2 * j + 1]))
         deco.set_profiling(None)
     kms = {k: statistics.mean(v[1:]) for k, v in kt.items()}
-    pairs = float(n_t.sum())
+    pairs = float(sum(n_t))
     kflops = {"route": 2.0 * shape.T * D * E, "proj": 2.0 * shape.T * D * (de + ds), "up": 2.0 * pairs * D * de,
               "down": 2.0 * pairs * de * D, "shared": 2.0 * shape.T * ds * D}
     dom = max(kflops, key=lambda k: kms[k])
     dom_tf = kflops[dom] / (kms[dom] / 1e3) / 1e12
-    out["prefill_t4096"] = {"ms": ms, "tokens_per_s": shape.T / (ms / 1e3),
-                            "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(dom_tf, 1),
-                                         "peak": P["bf16"], "unit": "TFLOP/s",
-                                         "frac": round(dom_tf / P["bf16"], 4), "peak_source": P["src"]},
-                            "tflops": flops / (ms / 1e3) / 1e12,
-                            "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / P["bf16"],
-                            "mean_activation": float(act.float().mean()),
-                            "kernel_ms": {k: round(v, 4) for k, v in kms.items()},
-                            "kernel_tflops": {k: round(f / (kms[k] / 1e3) / 1e12, 1)
-                                              for k, f in kflops.items()}}
+    per_tok = act.float().mean(dim=1)
+    return {"ms": ms, "tokens_per_s": shape.T / (ms / 1e3),
+            "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(dom_tf, 1),
+                         "peak": P["bf16"], "unit": "TFLOP/s",
+                         "frac": round(dom_tf / P["bf16"], 4), "peak_source": P["src"]},
+            "tflops": flops / (ms / 1e3) / 1e12,
+            "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / P["bf16"],
+            "mean_activation": float(per_tok.mean()), "min_token_activation": float(per_tok.min()),
+            "max_token_activation": float(per_tok.max()),
+            "zero_expert_tokens": int((per_tok == 0).sum()),
+            "kernel_ms": {k: round(v, 4) for k, v in kms.items()},
+            "kernel_tflops": {k: round(f / (kms[k] / 1e3) / 1e12, 1) for k, f in kflops.items()}}
+
+
+def extra_sweep(deco, dev, stream, P, torch):
+    """Config 5: the edge layer at 5/10/20/40/100 % mean activation, T = 1, 4,
+    16 (CUDA graphs over rotating weight copies, L2 defeated) and T = 4096
+    (eager), each next to the equal-parameter dense FFN (d_ff = d_s + E d_e)."""
+    from synth import CONFIGS, LayerShape, make_dense, make_layer
+    base = CONFIGS["edge_decode_t16"]["shape"]
+    D, E, de, ds = base.D, base.E, base.d_e, base.d_s
     d_ff = ds + E * de
-    for T in (16, 4096):
-        Dn = make_dense(T, D, d_ff, "bf16", 7)
-        x, W1, W2 = Dn["x"].to(dev), Dn["W1"].to(dev), Dn["W2"].to(dev)
-        od = torch.empty_like(x)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    res = {"d_ff": d_ff, "dense": {}, "sparse": {}}
+    # dense FFN
+    Dn = make_dense(4096, D, d_ff, "bf16", 7)
+    W = {"W1": Dn["W1"].to(dev), "W2": Dn["W2"].to(dev)}
+    nd = max(2, math.ceil(3 * l2 / (2 * d_ff * D * 2)) + 1)
+    Wc = _copies(torch, W, nd)
+    xd_all = Dn["x"].to(dev)
+    for T in (1, 4, 16, 4096):
+        x = xd_all[:T]
+        o = torch.empty_like(x)
         wsd = torch.empty(deco.dense_workspace_size(T, D, d_ff, x.dtype), dtype=torch.uint8, device=dev)
-        dms = timeit(lambda: deco.dense_ffn(x, W1, W2, out=od, workspace=wsd))
-        xs_ = G["x"][:T]
-        os_ = torch.empty_like(xs_)
-        ws_ = deco.alloc_workspace(deco.layer_shape(xs_, G), dev)
-        sms = timeit(lambda: deco.forward(xs_, G, out=os_, workspace=ws_))
-        out[f"dense_vs_sparse_t{T}"] = {"dense_ms": dms, "sparse_ms": sms, "speedup": dms / sms}
-        del W1, W2
-    return out
+        if T <= 16:
+            ms = _time_graphs(torch, stream, [lambda c=c: deco.dense_ffn(x, c["W1"], c["W2"], out=o, workspace=wsd)
+                                              for c in Wc])
+            res["dense"][str(T)] = {"us": round(1000 * ms, 2),
+                                    "hbm_frac": round(dense_bytes(T, D, d_ff) / (ms / 1e3) / 1e9 / P["hbm"], 4)}
+        else:
+            ms = _time_eager(torch, stream, lambda: deco.dense_ffn(x, W["W1"], W["W2"], out=o, workspace=wsd))
+            tf = 4.0 * T * D * d_ff / (ms / 1e3) / 1e12
+            res["dense"][str(T)] = {"us": round(1000 * ms, 2), "tflops": round(tf, 1),
+                                    "tensor_frac": round(tf / P["bf16"], 4)}
+    del Wc, W
+    torch.cuda.empty_cache()
+    for ratio in (0.05, 0.1, 0.2, 0.4, 1.0):
+        shape = LayerShape(4096, D, E, de, ds, "bf16")
+        L = make_layer(shape, 1, ratio=ratio)
+        x_all = L.pop("x").to(dev)
+        G = {k: v.to(dev) for k, v in L.items()}
+        G["W_bar_up"] = deco.mean_up(G["W_up"])
+        wb = sum(t.numel() * t.element_size() for t in G.values())
+        Gc = _copies(torch, G, max(2, math.ceil(3 * l2 / wb) + 1))
+        row = {}
+        for T in (1, 4, 16, 4096):
+            x = x_all[:T]
+            o = torch.empty_like(x)
+            ws = deco.alloc_workspace(deco.layer_shape(x, G), dev)
+            act = deco.routing(x, G)["active"].bool()
+            if T <= 16:
+                ms = _time_graphs(torch, stream, [lambda c=c: deco.forward(x, c, out=o, workspace=ws) for c in Gc])
+                nb = layer_bytes(T, D, E, de, ds, int(act.any(dim=0).sum()))
+                row[str(T)] = {"us": round(1000 * ms, 2), "hbm_frac": round(nb / (ms / 1e3) / 1e9 / P["hbm"], 4),
+                               "activation": round(float(act.float().mean()), 4),
+                               "speedup_vs_dense": round(res["dense"][str(T)]["us"] / (1000 * ms), 3)}
+            else:
+                ms = _time_eager(torch, stream, lambda: deco.forward(x, G, out=o, workspace=ws))
+                tf = layer_flops(act.sum(dim=1).tolist(), D, E, de, ds) / (ms / 1e3) / 1e12
+                row[str(T)] = {"us": round(1000 * ms, 2), "tflops": round(tf, 1),
+                               "tensor_frac": round(tf / P["bf16"], 4),
+                               "activation": round(float(act.float().mean()), 4),
+                               "speedup_vs_dense": round(res["dense"][str(T)]["us"] / (1000 * ms), 3)}
+            del ws
+        res["sparse"][f"{int(round(100 * ratio))}%"] = row
+        del Gc, G
+        torch.cuda.empty_cache()
+    return res
+
+
+def extra_topk(deco, dev, stream, P, torch):
+    """TopK routing at k = round(0.2 E) against DECO's ReLU routing at ~20 %
+    on the edge layer (the paper's §5 comparison), T = 1, 16 (graphs over
+    rotating copies) and 4096 (eager)."""
+    from synth import CONFIGS, LayerShape, make_layer
+    base = CONFIGS["edge_decode_t16"]["shape"]
+    D, E, de, ds = base.D, base.E, base.d_e, base.d_s
+    k = int(round(0.2 * E))
+    shape = LayerShape(4096, D, E, de, ds, "bf16")
+    L = make_layer(shape, 1)
+    x_all = L.pop("x").to(dev)
+    G = {kk: v.to(dev) for kk, v in L.items()}
+    G["W_bar_up"] = deco.mean_up(G["W_up"])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    wb = sum(t.numel() * t.element_size() for t in G.values())
+    Gc = _copies(torch, G, max(2, math.ceil(3 * l2 / wb) + 1))
+    res = {"k": k}
+    for T in (1, 16, 4096):
+        x = x_all[:T]
+        o = torch.empty_like(x)
+        row = {}
+        for name, tk in (("relu", 0), ("topk", k)):
+            ws = deco.alloc_workspace(deco.layer_shape(x, G, topk=tk), dev)
+            if T <= 16:
+                ms = _time_graphs(torch, stream,
+                                  [lambda c=c: deco.forward(x, c, out=o, workspace=ws, topk=tk) for c in Gc])
+            else:
+                ms = _time_eager(torch, stream, lambda: deco.forward(x, G, out=o, workspace=ws, topk=tk))
+            act = deco.routing(x, G, topk=tk)["active"].bool()
+            row[name] = {"us": round(1000 * ms, 2), "activation": round(float(act.float().mean()), 4),
+                         "union_experts": int(act.any(dim=0).sum())}
+        res[str(T)] = row
+    del Gc, G
+    torch.cuda.empty_cache()
+    return res
+
+
+def extra_stack(deco, dev, stream, P, torch):
+    """Config 4: 8 stacked layers (d_model 4096, 128 routed experts of width
+    256, shared width 2048, bf16, ~20 %), residual adds, T = 16 (decode
+    kernel; the 4.6 GB of weights exceed L2) and T = 16384 (tensor-core
+    kernels); tokens/s of the stack and per layer."""
+    from synth import CONFIGS, make_layer
+    base = CONFIGS["large_t16384"]["shape"]
+    D, E, de, ds = base.D, base.E, base.d_e, base.d_s
+    layers = []
+    for l in range(8):
+        L = make_layer(base, 3, layer=l, with_x=(l == 0))
+        x0 = L.pop("x") if l == 0 else None
+        G = {k: v.to(dev) for k, v in L.items()}
+        G["W_bar_up"] = deco.mean_up(G["W_up"])
+        layers.append(G)
+        if l == 0:
+            x_all = x0.to(dev)
+        del L
+    res = {}
+    for T in (16, 16384):
+        x = x_all[:T].contiguous()
+        bufs = [torch.empty_like(x), torch.empty_like(x)]
+        ws = deco.alloc_workspace(deco.layer_shape(x, layers[0], residual=True), dev)
+
+        def stack():
+            cur = x
+            for i, G in enumerate(layers):
+                nxt = bufs[i & 1]
+                deco.forward(cur, G, out=nxt, workspace=ws, eps=base.eps, residual=True)
+                cur = nxt
+        if T <= 16:
+            ms = _time_graphs(torch, stream, [stack], reps=50)
+            acts = []
+            cur = x
+            for i, G in enumerate(layers):
+                acts.append(deco.routing(cur, G)["active"].bool())
+                nxt = torch.empty_like(x)
+                deco.forward(cur, G, out=nxt, eps=base.eps, residual=True)
+                cur = nxt
+            nb = sum(layer_bytes(T, D, E, de, ds, int(a.any(dim=0).sum())) for a in acts)
+            res[str(T)] = {"ms": round(ms, 4), "tokens_per_s": T / (ms / 1e3),
+                           "hbm_frac": round(nb / (ms / 1e3) / 1e9 / P["hbm"], 4),
+                           "mean_activation": round(float(torch.stack(acts).float().mean()), 4)}
+        else:
+            ms = _time_eager(torch, stream, stack, n=3)
+            flops = 0.0
+            cur = x
+            acts = []
+            for G in layers:
+                a = deco.routing(cur, G)["active"].bool()
+                acts.append(float(a.float().mean()))
+                flops += layer_flops(a.sum(dim=1).tolist(), D, E, de, ds)
+                nxt = torch.empty_like(x)
+                deco.forward(cur, G, out=nxt, workspace=ws, eps=base.eps, residual=True)
+                cur = nxt
+                del a
+            tf = flops / (ms / 1e3) / 1e12
+            res[str(T)] = {"ms": round(ms, 3), "tokens_per_s": T / (ms / 1e3), "tflops": round(tf, 1),
+                           "tensor_frac": round(tf / P["bf16"], 4),
+                           "mean_activation": round(statistics.mean(acts), 4)}
+        del ws
+        torch.cuda.empty_cache()
+    del layers
+    torch.cuda.empty_cache()
+    return res
 
 
 if __name__ == "__main__":

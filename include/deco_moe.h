@@ -29,8 +29,9 @@
  *    keep them in fp32; bf16 batches of up to 16 tokens keep the hidden
  *    activations as bf16 hi/lo pairs (~16 significant bits); larger bf16
  *    batches (tensor-core path) round the hidden activations to bf16 and each
- *    (token, expert) output to fp16 before the fixed-order sum, which costs
- *    about 1 % of the output RMS at the largest element on the test layers.
+ *    (token, expert) output W_down[e] a, before its s_e r_e scaling, to fp16
+ *    ahead of the fixed-order sum, which costs about 1 % of the output RMS at
+ *    the largest element on the test layers.
  *  - All calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL is the legacy default stream) and never synchronise, except
  *    deco_moe_device_error.  They do not allocate, so a sequence of calls can
@@ -76,7 +77,12 @@ typedef enum { DECO_F32 = 0, DECO_BF16 = 1 } deco_dtype_t;
  *   d_s      shared expert width: multiple of 64, 64..16384
  *   dtype    storage dtype of x, out and every weight matrix
  *   rms_eps  epsilon added to the mean square inside NormSiLU's square root
- *   residual 0: out = layer(x); 1: out = x + layer(x), rounded once        */
+ *   residual 0: out = layer(x); 1: out = x + layer(x), rounded once
+ *   topk     routing rule.  0: DECO's ReLU routing (active iff z_e > 0).
+ *            k in 1..E: the TopK baseline of [arXiv] §5 -- each token keeps
+ *            its k largest logits (ranked on their exact values, exact ties
+ *            to the lower expert index) with weights ReLU(z_e), not
+ *            renormalised; everything after the router is unchanged      */
 typedef struct {
   int T;
   int d_model;
@@ -86,6 +92,7 @@ typedef struct {
   int dtype;      /* deco_dtype_t */
   float rms_eps;
   int residual;
+  int topk;
 } deco_moe_shape_t;
 
 /* The layer's weights (device pointers, storage dtype unless noted).
@@ -174,10 +181,13 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
 /* Synchronises `stream`, then reads the device error word a kernel may have
  * set in `workspace` and clears it.  Bits: 1 = a non-finite router operand;
  * 2 = a kernel gave up waiting for its own data after about a second (a
- * library fault, not an input property); 4 = on the bf16 prefill path
- * (T > 16), a routed expert's output s_e r_e W_down[e] a left the fp16 range
- * (|v| > 65504) in which it is staged before the combine, so the output is
- * not valid.  0 = none.  Returns DECO_ERR_CUDA if the synchronisation fails. */
+ * library fault, not an input property, unless deco_set_wait_limit lowered
+ * the limit); 4 = on the bf16 prefill path (T > 16), an unscaled routed
+ * expert output W_down[e] a left the fp16 range (|v| > 65504) in which it is
+ * staged before the combine, so the output is not valid.  Since |a_j| <=
+ * sqrt(d_e) after the RMS normalisation, |v| <= sqrt(d_e) times the largest
+ * row 1-norm of W_down[e]: this depends on the weights only, never on x.
+ * 0 = none.  Returns DECO_ERR_CUDA if the synchronisation fails. */
 deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
 
 /* Size of the library's built-in device scratch used by
@@ -196,27 +206,51 @@ deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
  * allocates nothing, and runs the same kernels, with the same results, as
  * deco_moe_forward.
  *  - Shapes whose deco_moe_workspace_size exceeds DECO_STATIC_SCRATCH_BYTES
- *    are rejected with DECO_ERR_WORKSPACE before anything is launched (decode
- *    batches of the layers in this library fit: e.g. T = 16 needs ~20 MB at
- *    d_model 2048 / 64 experts and ~26 MB at d_model 4096 / 128 experts).
+ *    are rejected with DECO_ERR_WORKSPACE before anything is launched.  Decode
+ *    batches fit: T = 16 needs about 18 MiB at d_model 2048 / 64 experts and
+ *    about 52 MiB (82 % of the array) at d_model 4096 / 128 experts; 256
+ *    experts at d_model 4096 do not fit and are refused.
  *  - The first call on each device looks up the scratch array's device
  *    address (cudaGetSymbolAddress, a runtime call made with that device
- *    current); make that first call before any stream capture on the device.
+ *    current) and keeps it for the life of the process; make that first call
+ *    before any stream capture on the device, and do not use this entry point
+ *    on a device after cudaDeviceReset.
  *  - All calls on a device share the one array.  Calls whose executions
  *    overlap on the GPU (different streams, or several threads) race on it and
  *    give wrong results; serialise them, e.g. on one stream.  Each call
  *    clears what must start at zero; the rest is overwritten.
- * Other arguments, results and errors are those of deco_moe_forward. */
+ * Other arguments, results and errors are those of deco_moe_forward; the
+ * device error word of the last call is read with
+ * deco_moe_static_device_error. */
 deco_status_t deco_moe_forward_static(const deco_moe_shape_t* shape, const void* x,
                                       const deco_moe_weights_t* w, void* out, void* stream);
 
+/* deco_moe_device_error for deco_moe_forward_static, whose error word lives
+ * in the built-in scratch array of the current device: synchronises `stream`,
+ * returns the word in *code (bits as for deco_moe_device_error) and clears it.
+ * Allocates nothing. */
+deco_status_t deco_moe_static_device_error(int* code, void* stream);
+
+/* Fault-injection hook for tests of the kernels' timeout path: every later
+ * call's kernels give up a wait for data (a shared-memory barrier or another
+ * CTA's counter) after `cycles` SM clock cycles instead of about a second,
+ * set bit 2 of the device error word, stop issuing work and, before exiting,
+ * still wait (with the default limit) for every copy and tensor-core
+ * operation they issued.  A small limit therefore makes the calls give up
+ * without faulting; their outputs are then not valid.  0 restores the
+ * default.  Process-wide, not thread-safe; not for production use. */
+deco_status_t deco_set_wait_limit(long long cycles);
+
 /* Kernel timing hook for benchmarks.  While set (events != NULL), every later
  * deco_moe_forward call on this process records events[2*i] on its stream just
- * before its i-th kernel and events[2*i+1] just after it, for i < n_events/2;
- * the kernels are, in order: router, expert counts, expert scatter,
- * up-projection, down-projection.  `events` are cudaEvent_t handles owned by the
- * caller (passed as void*) and must outlive the calls.  Pass NULL to stop.
- * Not thread-safe; meant for a single benchmarking thread. */
+ * before the kernel of timing slot i and events[2*i+1] just after it, for
+ * i < n_events/2.  Slots: 0 router, 1 expert counts, 2 expert scatter,
+ * 3 up-projection, 4 down-projection (general and tensor-core paths),
+ * 5 projections, 6 shared down-projection, 7 combine (tensor-core path),
+ * 8 the whole layer (decode path, one kernel).  `events` are cudaEvent_t
+ * handles owned by the caller (passed as void*) and must outlive the calls.
+ * Pass NULL to stop.  Not thread-safe; meant for a single benchmarking
+ * thread. */
 deco_status_t deco_moe_set_profiling(void* const* events, int n_events);
 
 /* The name and description of the CUDA error behind the last DECO_ERR_CUDA

@@ -40,7 +40,7 @@ class DecoError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("E", ctypes.c_int),
                 ("d_e", ctypes.c_int), ("d_s", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("rms_eps", ctypes.c_float), ("residual", ctypes.c_int)]
+                ("rms_eps", ctypes.c_float), ("residual", ctypes.c_int), ("topk", ctypes.c_int)]
 
 
 class Weights(ctypes.Structure):
@@ -64,6 +64,8 @@ _sig = {
     "deco_moe_device_error": [_vp, ctypes.POINTER(ctypes.c_int), _vp],
     "deco_moe_set_profiling": [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int],
     "deco_moe_forward_static": [ctypes.POINTER(Shape), _vp, ctypes.POINTER(Weights), _vp, _vp],
+    "deco_moe_static_device_error": [ctypes.POINTER(ctypes.c_int), _vp],
+    "deco_set_wait_limit": [ctypes.c_longlong],
 }
 for _name, _args in _sig.items():
     _f = getattr(_lib, _name)
@@ -93,9 +95,9 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def make_shape(T, D, E, d_e, d_s, dtype, eps=1e-6, residual=False) -> Shape:
+def make_shape(T, D, E, d_e, d_s, dtype, eps=1e-6, residual=False, topk=0) -> Shape:
     return Shape(T, D, E, d_e, d_s, _DT[dtype] if isinstance(dtype, torch.dtype) else dtype,
-                 eps, int(bool(residual)))
+                 eps, int(bool(residual)), int(topk))
 
 
 def _weights(L: dict) -> Weights:
@@ -103,10 +105,11 @@ def _weights(L: dict) -> Weights:
                      ("W_r", "b_r", "W_up", "W_bar_up", "W_down", "s", "W_s_up", "W_s_down")])
 
 
-def layer_shape(x: torch.Tensor, L: dict, eps=1e-6, residual=False) -> Shape:
+def layer_shape(x: torch.Tensor, L: dict, eps=1e-6, residual=False, topk=0) -> Shape:
     E, d_e, D = L["W_up"].shape if "W_up" in L else (L["W_r"].shape[0], 64, x.shape[1])
     d_s = L["W_s_up"].shape[0] if "W_s_up" in L else 64
-    return make_shape(x.shape[0], x.shape[1], L["W_r"].shape[0], d_e, d_s, x.dtype, eps, residual)
+    return make_shape(x.shape[0], x.shape[1], L["W_r"].shape[0], d_e, d_s, x.dtype, eps, residual,
+                      topk)
 
 
 def workspace_size(shape: Shape) -> int:
@@ -120,9 +123,10 @@ def alloc_workspace(shape: Shape, device="cuda") -> torch.Tensor:
 
 
 def forward(x: torch.Tensor, L: dict, out=None, workspace=None, eps=1e-6, residual=False,
-            stream=None) -> torch.Tensor:
-    """out = DECO MoE layer(x) (+ x if residual).  L: dict of device tensors."""
-    shape = layer_shape(x, L, eps, residual)
+            stream=None, topk=0) -> torch.Tensor:
+    """out = DECO MoE layer(x) (+ x if residual).  L: dict of device tensors.
+    topk > 0 replaces ReLU routing by the TopK baseline with k = topk."""
+    shape = layer_shape(x, L, eps, residual, topk)
     if out is None:
         out = torch.empty_like(x)
     if workspace is None:
@@ -152,10 +156,10 @@ def forward_static(x: torch.Tensor, L: dict, out=None, eps=1e-6, residual=False,
     return out
 
 
-def routing(x: torch.Tensor, L: dict, workspace=None, stream=None) -> dict:
+def routing(x: torch.Tensor, L: dict, workspace=None, stream=None, topk=0) -> dict:
     """Router + token->expert tables; returns r, active, counts, offsets, perm, n_tok."""
     T, E = x.shape[0], L["W_r"].shape[0]
-    shape = layer_shape(x, L)
+    shape = layer_shape(x, L, topk=topk)
     if workspace is None:
         workspace = alloc_workspace(shape, x.device)
     dev = x.device
@@ -205,10 +209,11 @@ def dense_ffn(x, W1, W2, out=None, workspace=None, stream=None) -> torch.Tensor:
 
 
 # timing slots of deco_moe_set_profiling: slot i is bracketed by events 2i and
-# 2i+1.  The decode path (bf16, T <= 16) fills route, up, down and combine;
-# the general path route..down; the prefill path (bf16, T > 16) all eight.
+# 2i+1.  The general path fills route..down, the prefill path (bf16, T > 16)
+# route..combine, the decode path (bf16, T <= 16) only "layer" (one kernel).
 KERNELS = ("route", "count", "scatter", "up", "down")
 PREFILL_KERNELS = KERNELS + ("proj", "shared", "combine")
+ALL_SLOTS = PREFILL_KERNELS + ("layer",)
 
 
 def set_profiling(events):
@@ -235,3 +240,16 @@ def device_error(workspace, stream=None) -> int:
     _check(_lib.deco_moe_device_error(_ptr(workspace), ctypes.byref(code), _stream(stream)),
            "device_error")
     return code.value
+
+
+def static_device_error(stream=None) -> int:
+    """The device error word of the last forward_static call on this device (cleared)."""
+    code = ctypes.c_int(0)
+    _check(_lib.deco_moe_static_device_error(ctypes.byref(code), _stream(stream)),
+           "static_device_error")
+    return code.value
+
+
+def set_wait_limit(cycles: int):
+    """Test hook: kernels give up waits for data after `cycles` SM cycles (0: default)."""
+    _check(_lib.deco_set_wait_limit(int(cycles)), "set_wait_limit")

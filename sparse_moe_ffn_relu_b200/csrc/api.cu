@@ -23,12 +23,16 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace layout of one forward / routing call.
 struct Plan {
-  size_t err, r, act, u, hs, counts, offsets, n_tok, perm, pair_of, tiles, n_tiles, H, total;
-  // decode path (T <= 16)
-  size_t hs16, C16, P16, Ps16;
+  size_t err, err_bytes, r, act, u, hs, counts, offsets, n_tok, perm, pair_of, tiles, n_tiles, H, total;
+  // decode path (T <= 16): up-projection partials, shared hidden and NormSiLU
+  // tiles, per-CTA down-projection partials (the inter-CTA counters follow
+  // the error word)
+  size_t C16, HS, A16, Part;
   // bf16, T > 16: ambiguous router pairs; prefill path: routed expert output
   // rows (one fp16 row per pair) and the shared expert's fp32 output
-  size_t fb, blk, v_pairs, s_out;
+  size_t fb, blk, v_pairs, coef, s_out;
+  // TopK routing: fp32 logits and their error bounds
+  size_t zt, bt;
   int tile_rows;
   int sms;
 };
@@ -64,7 +68,12 @@ Plan make_plan(const deco_moe_shape_t& s) {
   };
   const size_t T = s.T, E = s.E, P = T * E;
   p.tile_rows = token_tile(s.d_model, s.dtype);
-  p.err = take(16);
+  p.sms = num_sms();
+  // error word (+ the prefill router's ambiguous-pair count), then the decode
+  // kernel's counters; all cleared by every call
+  p.err_bytes = 16;
+  if (s.T <= dec::kMaxT) p.err_bytes += 4 * (size_t)dec::sync_idx(s.E, s.d_model).total;
+  p.err = take(p.err_bytes);
   p.r = take(T * E * 4);
   p.act = take(T * E);
   p.u = take(T * s.d_e * 4);
@@ -77,20 +86,24 @@ Plan make_plan(const deco_moe_shape_t& s) {
   p.tiles = take((P / p.tile_rows + E) * 16);
   p.n_tiles = take(4);
   p.H = take(P * s.d_e * 4);       // NormSiLU activations (fp32; bf16 on the prefill path)
-  p.sms = num_sms();
   if (tiled_router(s)) {
     p.fb = take(P * 8);
     p.blk = take((size_t)((s.T + pf::kTabThreads - 1) / pf::kTabThreads) * E * 4);
   }
+  if (s.topk > 0) {
+    p.zt = take(P * 4);
+    p.bt = take(P * 4);
+  }
   if (prefill_eligible(s)) {
     p.v_pairs = take(P * s.d_model * 2);
+    p.coef = take(P * 4);
     p.s_out = take(T * s.d_model * 4);
   }
   if (s.T <= dec::kMaxT) {         // decode path buffers (see decode_kernels.cuh)
-    p.hs16 = take((size_t)dec::kTok * s.d_s * 4);         // [16][hi d_s | lo d_s] bf16
-    p.C16 = take(8 * E * dec::kTok * s.d_e * 4);           // [kp <= 8][E][16][d_e] fp32
-    p.P16 = take(E * dec::kTok * s.d_model * 4);           // [E][16][D] fp32
-    p.Ps16 = take((size_t)dec::down_nsq(s.d_s) * dec::kTok * s.d_model * 4);   // [nsq][16][D] fp32
+    p.C16 = take(8 * E * dec::kTok * s.d_e * 4);                       // [kp <= 8][E][16][d_e] fp32
+    p.HS = take((size_t)dec::down_nsq(s.d_s) * dec::kTileBytes);       // [nsq] 16 KB tiles
+    p.A16 = take(E * dec::kTileBytes);                                 // [E] 16 KB tiles
+    p.Part = take((size_t)std::max(p.sms, 1) * 2 * dec::kTok * dec::kDRows * 4);   // [G][2][16][128]
   }
   p.total = off;
   return p;
@@ -105,6 +118,7 @@ deco_status_t check_shape(const deco_moe_shape_t* s) {
   if (s->dtype != DECO_F32 && s->dtype != DECO_BF16) return DECO_ERR_INVALID_ARG;
   if (!(s->rms_eps >= 0.f) || !std::isfinite(s->rms_eps)) return DECO_ERR_INVALID_ARG;
   if (s->residual != 0 && s->residual != 1) return DECO_ERR_INVALID_ARG;
+  if (s->topk < 0 || s->topk > s->E) return DECO_ERR_INVALID_ARG;
   if (s->d_model % 64 || s->d_model > 16384) return DECO_ERR_UNSUPPORTED;
   if (s->E > 256) return DECO_ERR_UNSUPPORTED;
   if (s->d_e % 64 || s->d_e > 512) return DECO_ERR_UNSUPPORTED;
@@ -158,6 +172,25 @@ inline void prof_mark(int idx, cudaStream_t st) {
     cudaEventRecord(g_prof_events[idx], st);
 }
 
+// The decode kernel (decode_kernels.cuh) takes bf16 batches of up to 16 tokens
+// with d_model a multiple of 256 up to 4096 and d_e <= 256, on GPUs of at most
+// dec::kMaxSms SMs whose router CTAs leave room for the other phase-R rows.
+bool decode_grid_ok(int D, int E, int sms) {
+  if (D % 256 || D > 4096 || sms > dec::kMaxSms) return false;
+  if (dec::router_ctas(E) + 16 > sms) return false;
+  return dec::layer_smem(D).nstages >= 2;
+}
+
+bool decode_eligible(const deco_moe_shape_t& s, int sms) {
+  if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT) return false;
+  if (s.E > 256 || s.d_e > 256 || s.d_e % 64 || s.d_s % 64) return false;
+  return decode_grid_ok(s.d_model, s.E, sms);
+}
+
+// limit of the kernels' waits for data (deco_set_wait_limit; the drains of
+// copies already issued keep the default)
+long long g_wait_cycles = dec::kWaitCycles;
+
 // ---------------------------------------------------------------------------
 template <typename T, int TT>
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
@@ -203,7 +236,7 @@ template <typename T>
 cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
                         unsigned char* ws, const Plan& p, bool with_mean_shared, float* r,
                         uint8_t* act, int* counts, int* offsets, int* perm, int* n_tok,
-                        cudaStream_t st, int tile_rows) {
+                        cudaStream_t st, int tile_rows, bool decide_only = false) {
   RouteArgs ra{};
   ra.x = x;
   ra.T = s.T;
@@ -222,7 +255,43 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
   ra.err = reinterpret_cast<int*>(ws + p.err);
   prof_mark(0, st);
   cudaError_t err;
-  if (!with_mean_shared && tiled_router(s)) {
+  if (s.topk > 0) {
+    // TopK: logits and bounds from the general router, then the exact selection
+    ra.zt = reinterpret_cast<float*>(ws + p.zt);
+    ra.bt = reinterpret_cast<float*>(ws + p.bt);
+    if ((err = route_any<T>(ra, token_tile(s.d_model, s.dtype), st)) != cudaSuccess) return err;
+    TopkArgs ta{};
+    ta.x = x;
+    ta.W_r = w.W_r;
+    ta.b_r = w.b_r;
+    ta.T = s.T;
+    ta.D = s.d_model;
+    ta.E = s.E;
+    ta.k = s.topk;
+    ta.zt = ra.zt;
+    ta.bt = ra.bt;
+    ta.r = r;
+    ta.act = act;
+    ta.err = ra.err;
+    k_topk_select<T><<<(s.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st>>>(ta);
+  } else if (!with_mean_shared && s.dtype == DECO_BF16 && decode_eligible(s, p.sms)) {
+    // the decode forward's own router: kd_layer's router CTAs alone (the
+    // same per-row code and order, so the same decisions bit for bit)
+    dec::Args da{};
+    da.T = s.T;
+    da.D = s.d_model;
+    da.E = s.E;
+    da.wait_cycles = g_wait_cycles;
+    da.x = static_cast<const bf16*>(x);
+    da.W_r = static_cast<const bf16*>(w.W_r);
+    da.b_r = w.b_r;
+    da.r = r;
+    da.act = act;
+    da.err = reinterpret_cast<int*>(ws + p.err);
+    const uint32_t smem = dec::layer_smem(s.d_model).total;
+    if ((err = allow_smem(dec::kd_router, smem)) != cudaSuccess) return err;
+    dec::kd_router<<<dec::router_ctas(s.E), dec::kThreads, smem, st>>>(da);
+  } else if (!with_mean_shared && tiled_router(s)) {
     pf::RouterArgs rt{};
     rt.x = static_cast<const bf16*>(x);
     rt.W_r = static_cast<const bf16*>(w.W_r);
@@ -245,15 +314,17 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
   }
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   prof_mark(1, st);
+  if (decide_only) return cudaSuccess;
   if (!with_mean_shared && tiled_router(s)) {   // token-block tables
-    const int nb = (s.T + pf::kTabThreads - 1) / pf::kTabThreads;
+    const int nu = (s.T + pf::kTabUnit - 1) / pf::kTabUnit;   // units of 32 tokens, one warp each
+    const int nb = (nu + pf::kTabWarps - 1) / pf::kTabWarps;
     int* blk = reinterpret_cast<int*>(ws + p.blk);
     prof_mark(2, st);
     pf::k_tab_count<<<nb, pf::kTabThreads, 0, st>>>(act, s.T, s.E, n_tok, blk);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     prof_mark(3, st);
     prof_mark(4, st);
-    pf::k_tab_scatter<<<nb, pf::kTabThreads, 0, st>>>(act, s.T, s.E, blk, nb, counts, offsets, perm,
+    pf::k_tab_scatter<<<nb, pf::kTabThreads, 0, st>>>(act, s.T, s.E, blk, nu, counts, offsets, perm,
                                                       reinterpret_cast<int*>(ws + p.pair_of),
                                                       reinterpret_cast<int4*>(ws + p.tiles),
                                                       reinterpret_cast<int*>(ws + p.n_tiles), tile_rows);
@@ -308,42 +379,38 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// kd_down's resident operands: hidden rows, the NormSiLU tile, a zero row
-uint32_t dec_down_operand(const deco_moe_shape_t& s) {
-  return (uint32_t)dec::kTok * s.d_s * 4 + (uint32_t)dec::kTok * s.d_e * 4 + 1024;
-}
-
-bool decode_eligible(const deco_moe_shape_t& s, int sms) {
-  if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT) return false;
-  if (s.d_model % 256 || s.d_model > 4096) return false;
-  if (s.E > 256 || s.d_e > 256 || s.d_e % 64 || s.d_s % 64 || s.d_s > 2048) return false;
-  if (dec::router_ctas(s.E) + 16 > sms) return false;         // router CTAs leave room
-  const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
-  if (dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).nstages < 2) return false;
-  if (dec::smem_plan(xop, dec::kStageBytes).nstages < 2) return false;
-  if (dec::smem_plan(dec_down_operand(s), dec::kStageBytes).nstages < 2) return false;
-  return true;
-}
-
-// launch with an optional programmatic-dependent-launch edge to the previous kernel
-template <typename K, typename... Ps>
-cudaError_t launch_dec(K kernel, dim3 grid, dim3 block, uint32_t smem_total, bool pdl, cudaStream_t st,
-                       const Ps&... params) {
-  if (smem_total > 48 * 1024) {
-    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_total);
-    if (err != cudaSuccess) return err;
-  }
+// one CTA per SM, all resident at once (the CTAs wait on one another's
+// counters), so the launch is cooperative
+cudaError_t launch_layer(const CUtensorMap& tmU, const CUtensorMap& tmW, const CUtensorMap& tmS,
+                         const dec::Args& a, int sms, cudaStream_t st) {
+  const uint32_t smem = dec::layer_smem(a.D).total;
+  cudaError_t err = cudaFuncSetAttribute(dec::kd_layer, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem_total;
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(dec::kThreads);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, params...);
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dec::kd_layer, tmU, tmW, tmS, a);
+}
+
+// the decode kernel's buffers in a workspace laid out by make_plan
+void decode_buffers(dec::Args& a, unsigned char* ws, const Plan& p) {
+  a.wait_cycles = g_wait_cycles;
+  a.r = reinterpret_cast<float*>(ws + p.r);
+  a.act = reinterpret_cast<uint8_t*>(ws + p.act);
+  a.u = reinterpret_cast<float*>(ws + p.u);
+  a.HS = reinterpret_cast<bf16*>(ws + p.HS);
+  a.A = reinterpret_cast<bf16*>(ws + p.A16);
+  a.C = reinterpret_cast<float*>(ws + p.C16);
+  a.Part = reinterpret_cast<float*>(ws + p.Part);
+  a.err = reinterpret_cast<int*>(ws + p.err);
+  a.sync = reinterpret_cast<unsigned*>(ws + p.err + 16);
 }
 
 cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
@@ -365,46 +432,53 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
   a.s = w.s;
   a.W_s_up = static_cast<const bf16*>(w.W_s_up);
   a.W_s_down = static_cast<const bf16*>(w.W_s_down);
-  a.r = reinterpret_cast<float*>(ws + p.r);
-  a.act = reinterpret_cast<uint8_t*>(ws + p.act);
-  a.u = reinterpret_cast<float*>(ws + p.u);
-  a.hs = reinterpret_cast<bf16*>(ws + p.hs16);
-  a.C = reinterpret_cast<float*>(ws + p.C16);
-  a.P = reinterpret_cast<float*>(ws + p.P16);
-  a.Ps = reinterpret_cast<float*>(ws + p.Ps16);
-  a.err = reinterpret_cast<int*>(ws + p.err);
   a.out = static_cast<bf16*>(out);
-  // kd_down's weight tiles: 128 rows x 64 columns
+  a.pre_routed = s.topk > 0;
+  decode_buffers(a, ws, p);
+  // weight tiles of phases U and D: 128 rows x 64 columns
   CUtensorMap tmU, tmW, tmS;
   cudaError_t err;
   if ((err = make_map(&tmU, w.W_up, s.d_model, (uint64_t)s.E * s.d_e, dec::kDRows)) != cudaSuccess ||
       (err = make_map(&tmW, w.W_down, s.d_e, (uint64_t)s.E * s.d_model, dec::kDRows)) != cudaSuccess ||
       (err = make_map(&tmS, w.W_s_down, s.d_s, s.d_model, dec::kDRows)) != cudaSuccess)
     return err;
-  const uint32_t xop = dec::kTok * dec::x_pitch(s.d_model) + 4096;
-  const uint32_t route_smem = std::max(dec::smem_plan(xop, dec::row_stage_bytes(s.d_model)).total,
-                                       dec::smem_plan(xop, dec::kStageBytes).total);
-  const uint32_t down_smem = dec::smem_plan(dec_down_operand(s), dec::kStageBytes).total;
-  const dim3 grid(p.sms), block(dec::kThreads);
-  // with timing events between the kernels each one is timed on its own
-  const bool pdl = g_prof_events == nullptr;
-  prof_mark(0, st);
-  err = launch_dec(dec::kd_route, grid, block, route_smem, false, st, a);
-  if (err != cudaSuccess) return err;
-  prof_mark(1, st);
-  prof_mark(6, st);
-  err = launch_dec(dec::kd_up, grid, block, dec::smem_plan(dec::kTok * dec::x_pitch(s.d_model), dec::kStageBytes).total,
-                   pdl, st, tmU, a);
-  if (err != cudaSuccess) return err;
-  prof_mark(7, st);
-  prof_mark(8, st);
-  err = launch_dec(dec::kd_down, grid, block, down_smem, pdl, st, tmW, tmS, a);
-  if (err != cudaSuccess) return err;
-  prof_mark(9, st);
-  prof_mark(14, st);
-  err = launch_dec(dec::kd_combine, dim3((s.d_model + 255) / 256, s.T), dim3(256), 0, pdl, st, a);
-  prof_mark(15, st);
+  prof_mark(16, st);
+  err = launch_layer(tmU, tmW, tmS, a, p.sms, st);
+  prof_mark(17, st);
   return err;
+}
+
+// dense FFN y = W2 SiLU(W1 x) at decode batch sizes: the same kernel with no
+// routed experts (W1 streams as phase-R rows, W2 as phase-D units)
+size_t dense_decode_bytes(int D, int d_ff, int sms) {
+  return 16 + 4 * (size_t)dec::sync_idx(0, D).total + (size_t)dec::down_nsq(d_ff) * dec::kTileBytes +
+         (size_t)sms * 2 * dec::kTok * dec::kDRows * 4 + 3 * 256;
+}
+
+cudaError_t run_dense_decode(int T, int D, int d_ff, const void* x, const void* W1, const void* W2, void* out,
+                             unsigned char* ws, int sms, cudaStream_t st) {
+  dec::Args a{};
+  a.T = T;
+  a.D = D;
+  a.E = 0;
+  a.d_e = 0;
+  a.d_s = d_ff;
+  a.wait_cycles = g_wait_cycles;
+  a.x = static_cast<const bf16*>(x);
+  a.W_s_up = static_cast<const bf16*>(W1);
+  a.W_s_down = static_cast<const bf16*>(W2);
+  a.out = static_cast<bf16*>(out);
+  const size_t sync_bytes = 16 + 4 * (size_t)dec::sync_idx(0, D).total;
+  a.err = reinterpret_cast<int*>(ws);
+  a.sync = reinterpret_cast<unsigned*>(ws + 16);
+  const size_t hs_off = align256(sync_bytes);
+  a.HS = reinterpret_cast<bf16*>(ws + hs_off);
+  a.Part = reinterpret_cast<float*>(ws + align256(hs_off + (size_t)dec::down_nsq(d_ff) * dec::kTileBytes));
+  cudaError_t err = cudaMemsetAsync(ws, 0, sync_bytes, st);
+  if (err != cudaSuccess) return err;
+  CUtensorMap tmS;
+  if ((err = make_map(&tmS, W2, d_ff, D, dec::kDRows)) != cudaSuccess) return err;
+  return launch_layer(tmS, tmS, tmS, a, sms, st);   // no routed experts: the W_up / W_down maps are unused
 }
 
 // ---------------------------------------------------------------------------
@@ -433,6 +507,7 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   const int T = s.T, D = s.d_model, E = s.E, d_e = s.d_e, d_s = s.d_s;
   const uint64_t P = (uint64_t)T * E;
   pf::Args a{};
+  a.wait_cycles = g_wait_cycles;
   a.T = T;
   a.D = D;
   a.E = E;
@@ -451,6 +526,7 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   a.hs = reinterpret_cast<bf16*>(ws + p.hs);
   a.a_pairs = reinterpret_cast<bf16*>(ws + p.H);
   a.v_pairs = reinterpret_cast<__half*>(ws + p.v_pairs);
+  a.coef_pairs = reinterpret_cast<float*>(ws + p.coef);
   a.s_out = reinterpret_cast<float*>(ws + p.s_out);
   a.out = static_cast<bf16*>(out);
   a.err = reinterpret_cast<int*>(ws + p.err);
@@ -502,7 +578,8 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   prof_mark(13, st);
   // out = shared + routed rows in ascending expert order (+ x)
   prof_mark(14, st);
-  pf::k_combine<<<T, pf::kCThreads, 0, st>>>(a.s_out, a.v_pairs, a.pair_of, a.x, a.out, D, E, s.residual);
+  pf::k_combine<<<T, pf::kCThreads, 0, st>>>(a.s_out, a.v_pairs, a.coef_pairs, a.pair_of, a.x, a.out, D, E,
+                                             s.residual);
   prof_mark(15, st);
   return cudaGetLastError();
 }
@@ -511,6 +588,7 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
 cudaError_t run_dense_tc(int T, int D, int d_ff, const void* x, const void* W1, const void* W2, void* out,
                          unsigned char* ws, cudaStream_t st) {
   pf::Args a{};
+  a.wait_cycles = g_wait_cycles;
   a.T = T;
   a.D = D;
   a.E = 0;
@@ -543,7 +621,17 @@ cudaError_t run_dense_tc(int T, int D, int d_ff, const void* x, const void* W1, 
 template <typename T>
 cudaError_t run_forward(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w,
                         void* out, unsigned char* ws, const Plan& p, cudaStream_t st) {
-  if (s.T <= dec::kMaxT && decode_eligible(s, p.sms)) return run_decode(s, x, w, out, ws, p, st);
+  if (s.T <= dec::kMaxT && decode_eligible(s, p.sms)) {
+    if (s.topk > 0) {   // TopK decisions first; the layer kernel then has no router CTAs
+      cudaError_t err = run_routing<T>(s, x, w, ws, p, false, reinterpret_cast<float*>(ws + p.r),
+                                       reinterpret_cast<uint8_t*>(ws + p.act),
+                                       reinterpret_cast<int*>(ws + p.counts), reinterpret_cast<int*>(ws + p.offsets),
+                                       reinterpret_cast<int*>(ws + p.perm), reinterpret_cast<int*>(ws + p.n_tok), st,
+                                       p.tile_rows, /*decide_only=*/true);
+      if (err != cudaSuccess) return err;
+    }
+    return run_decode(s, x, w, out, ws, p, st);
+  }
   if (prefill_eligible(s)) return run_prefill(s, x, w, out, ws, p, st);
   float* r = reinterpret_cast<float*>(ws + p.r);
   uint8_t* act = reinterpret_cast<uint8_t*>(ws + p.act);
@@ -637,7 +725,7 @@ deco_status_t deco_moe_forward(const deco_moe_shape_t* shape, const void* x,
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   cudaStream_t cs = as_stream(stream);
   std::lock_guard<std::mutex> lock(g_smem_mutex);
-  cudaError_t err = cudaMemsetAsync(ws + p.err, 0, 16, cs);
+  cudaError_t err = cudaMemsetAsync(ws + p.err, 0, p.err_bytes, cs);
   if (err != cudaSuccess) return cuda_status(err, "forward: clearing the error word");
   err = shape->dtype == DECO_F32 ? run_forward<float>(*shape, x, *w, out, ws, p, cs)
                                  : run_forward<bf16>(*shape, x, *w, out, ws, p, cs);
@@ -699,6 +787,8 @@ deco_status_t deco_dense_ffn_workspace_size(int T, int d_model, int d_ff, int dt
   if (d_model % 64 || d_model > 16384 || d_ff % 64 || d_ff > (1 << 20) || T > (1 << 20))
     return DECO_ERR_UNSUPPORTED;
   *bytes = 256 + align256((size_t)T * d_ff * 4);
+  if (dtype == DECO_BF16 && T <= dec::kMaxT && decode_grid_ok(d_model, 0, num_sms()))
+    *bytes = std::max(*bytes, dense_decode_bytes(d_model, d_ff, num_sms()));
   return DECO_OK;
 }
 
@@ -740,7 +830,10 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
   da.out = out;
   da.residual = 0;
   cudaError_t err;
-  if (dtype == DECO_BF16)   // tensor cores at any batch size (a 128-row tile covers a small batch)
+  const int sms = num_sms();
+  if (dtype == DECO_BF16 && T <= dec::kMaxT && decode_grid_ok(d_model, 0, sms))   // weight streaming
+    return cuda_status(run_dense_decode(T, d_model, d_ff, x, W1, W2, out, ws, sms, cs), "dense_ffn");
+  if (dtype == DECO_BF16)   // tensor cores (a 128-row tile covers a small batch)
     return cuda_status(run_dense_tc(T, d_model, d_ff, x, W1, W2, out, ws, cs), "dense_ffn");
   const int tt = token_tile(d_model, dtype);
   if (dtype == DECO_F32) {
@@ -751,6 +844,12 @@ deco_status_t deco_dense_ffn_forward(int T, int d_model, int d_ff, int dtype, co
     if (err == cudaSuccess) err = launch_down<bf16>(da, cs);
   }
   return cuda_status(err, "dense_ffn");
+}
+
+deco_status_t deco_set_wait_limit(long long cycles) {
+  if (cycles < 0) return DECO_ERR_INVALID_ARG;
+  g_wait_cycles = cycles == 0 ? dec::kWaitCycles : cycles;
+  return DECO_OK;
 }
 
 deco_status_t deco_moe_set_profiling(void* const* events, int n_events) {
@@ -783,7 +882,9 @@ namespace {
 // The scratch every deco_moe_forward_static call on a device uses.  Host code
 // must not pass `g_static_scratch` itself to a kernel: on the host the name is
 // only a stand-in for the symbol, so its device address is looked up once per
-// device with cudaGetSymbolAddress and cached here.
+// device with cudaGetSymbolAddress and cached here.  The cache is not
+// invalidated by cudaDeviceReset (the module, and with it the array, may then
+// be reloaded elsewhere), so the entry point is not for use after a reset.
 static __device__ __align__(256) unsigned char g_static_scratch[DECO_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -825,4 +926,13 @@ extern "C" deco_status_t deco_moe_forward_static(const deco_moe_shape_t* shape, 
   // the forward pass clears the error word it keeps at the start of the
   // scratch and overwrites everything else it reads
   return deco_moe_forward(shape, x, w, out, scratch, DECO_STATIC_SCRATCH_BYTES, stream);
+}
+
+extern "C" deco_status_t deco_moe_static_device_error(int* code, void* stream) {
+  if (!code) return DECO_ERR_INVALID_ARG;
+  unsigned char* scratch = nullptr;
+  const cudaError_t err = static_scratch(&scratch);
+  if (err != cudaSuccess) return cuda_status(err, "static_device_error: scratch address");
+  // the error word sits at the start of every workspace plan
+  return deco_moe_device_error(scratch, code, stream);
 }

@@ -281,6 +281,133 @@ __device__ int exact_sign_warp(const Tx* x, const Tw* w, int D, float b,
   return carry < 0 ? -1 : ((carry > 0 || nz) ? 1 : 0);
 }
 
+// Exact sign (-1, 0, +1) of (b1 + sum_k x[k] w1[k]) - (b2 + sum_k x[k] w2[k]):
+// the exact comparison of two logits of one token (TopK ranking).  The same
+// integer accumulation as exact_sign_warp, with the second row's products and
+// bias entering negated: a window of kWin limbs in registers anchored at the
+// largest product, and the 640-bit fixed point in shared memory when a
+// product lies below the window.  Called by all 32 lanes of one warp.
+template <typename Tx, typename Tw>
+__device__ int exact_cmp_warp_limbs(const Tx* x, const Tw* w1, const Tw* w2, int D, float b1, float b2,
+                                    unsigned long long* limbs) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < kLimbs; i += 32) limbs[i] = 0ull;
+  __syncwarp();
+  for (int k = lane; k < D; k += 32) {
+    const FpParts px = fp_parts(to_f32(x[k]));
+    const FpParts p1 = fp_parts(to_f32(w1[k]));
+    const FpParts p2 = fp_parts(to_f32(w2[k]));
+    if (px.m && p1.m)
+      limbs_add_scaled(limbs, (unsigned long long)px.m * p1.m, px.e + p1.e - kLsbExp, px.neg != p1.neg);
+    if (px.m && p2.m)
+      limbs_add_scaled(limbs, (unsigned long long)px.m * p2.m, px.e + p2.e - kLsbExp, px.neg == p2.neg);
+  }
+  if (lane == 0) {
+    const FpParts q1 = fp_parts(b1), q2 = fp_parts(b2);
+    if (q1.m) limbs_add_scaled(limbs, q1.m, q1.e - kLsbExp, q1.neg);
+    if (q2.m) limbs_add_scaled(limbs, q2.m, q2.e - kLsbExp, !q2.neg);
+  }
+  __syncwarp();
+  int sign = 0;
+  if (lane == 0) {
+    long long carry = 0;
+    bool nz = false;
+    for (int i = 0; i < kLimbs; ++i) {
+      const long long v = (long long)limbs[i] + carry;
+      nz |= (v & 0xffffffffll) != 0;
+      carry = v >> 32;
+    }
+    sign = carry < 0 ? -1 : ((carry > 0 || nz) ? 1 : 0);
+  }
+  sign = __shfl_sync(kFull, sign, 0);
+  __syncwarp();
+  return sign;
+}
+
+template <typename Tx, typename Tw>
+__device__ int exact_cmp_warp(const Tx* x, const Tw* w1, const Tw* w2, int D, float b1, float b2,
+                              unsigned long long* limbs, bool* nonfinite) {
+  const int lane = threadIdx.x & 31;
+  bool bad = false;
+  int fmax = INT_MIN;
+  for (int k0 = lane * 8; k0 < D; k0 += 256) {
+    float xv[8], v1[8], v2[8];
+    load8(x + k0, xv);
+    load8(w1 + k0, v1);
+    load8(w2 + k0, v2);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const FpParts px = fp_parts(xv[q]), p1 = fp_parts(v1[q]), p2 = fp_parts(v2[q]);
+      bad |= !(px.finite && p1.finite && p2.finite);
+      if (px.m && p1.m) fmax = max(fmax, px.e + p1.e);
+      if (px.m && p2.m) fmax = max(fmax, px.e + p2.e);
+    }
+  }
+  const FpParts q1 = fp_parts(b1), q2 = fp_parts(b2);
+  bad |= !(q1.finite && q2.finite);
+  if (q1.m) fmax = max(fmax, q1.e);
+  if (q2.m) fmax = max(fmax, q2.e);
+  bad = __any_sync(kFull, bad);
+  fmax = __reduce_max_sync(kFull, fmax);
+  if (bad) {
+    *nonfinite = true;
+    return 0;
+  }
+  if (fmax == INT_MIN) return 0;
+  const int base = fmax + 64 - 32 * kWin;
+  long long L[kWin];
+#pragma unroll
+  for (int j = 0; j < kWin; ++j) L[j] = 0;
+  bool below = false;
+  for (int k0 = lane * 8; k0 < D; k0 += 256) {
+    float xv[8], v1[8], v2[8];
+    load8(x + k0, xv);
+    load8(w1 + k0, v1);
+    load8(w2 + k0, v2);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const FpParts px = fp_parts(xv[q]), p1 = fp_parts(v1[q]), p2 = fp_parts(v2[q]);
+      if (px.m && p1.m) {
+        const int o = px.e + p1.e - base;
+        if (o < 0) below = true;
+        else win_add(L, (unsigned long long)px.m * p1.m, o, px.neg != p1.neg);
+      }
+      if (px.m && p2.m) {
+        const int o = px.e + p2.e - base;
+        if (o < 0) below = true;
+        else win_add(L, (unsigned long long)px.m * p2.m, o, px.neg == p2.neg);
+      }
+    }
+  }
+  if (lane == 0) {
+    if (q1.m) {
+      const int o = q1.e - base;
+      if (o < 0) below = true;
+      else win_add(L, q1.m, o, q1.neg);
+    }
+    if (q2.m) {
+      const int o = q2.e - base;
+      if (o < 0) below = true;
+      else win_add(L, q2.m, o, !q2.neg);
+    }
+  }
+  if (__any_sync(kFull, below)) return exact_cmp_warp_limbs(x, w1, w2, D, b1, b2, limbs);
+#pragma unroll
+  for (int j = 0; j < kWin; ++j) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L[j] += __shfl_xor_sync(kFull, L[j], o);
+  }
+  long long carry = 0;
+  bool nz = false;
+#pragma unroll
+  for (int j = 0; j < kWin; ++j) {
+    const long long v = L[j] + carry;
+    nz |= (v & 0xffffffffll) != 0;
+    carry = v >> 32;
+  }
+  return carry < 0 ? -1 : ((carry > 0 || nz) ? 1 : 0);
+}
+
 // gamma_n = n u / (1 - n u) with u = 2^-24: the classical bound on the
 // relative error of an n-step fp32 recursive (FMA) summation.
 __device__ __forceinline__ float gamma_f32(int n) {

@@ -1,51 +1,56 @@
-// Decode-batch kernels (T <= 16 tokens, bf16) of the DECO MoE layer.
+// Decode-batch kernel (T <= 16 tokens, bf16) of the DECO MoE layer.
 //
 // At a few tokens the layer is bound by HBM: every weight byte is used by at
 // most 16 tokens, and only the routed experts that some token activates need
 // to be read (the paper's point about sparse activation saving memory access,
 // "DECO: Sparse Mixture-of-Experts with Dense-Comparable Performance on
-// End-Side Devices", §1 and §5).  Three kernels stream the weights once and
-// a fourth adds the partial results:
+// End-Side Devices", §1 and §5).  The whole layer is one persistent kernel,
+// kd_layer, with one CTA per SM (a cooperative launch, so every CTA is
+// resident), that streams each needed weight byte once through a shared-memory
+// ring and hands data between CTAs through counters in global memory instead
+// of kernel boundaries:
 //
-//   kd_route  router rows W_r (exact activation decisions, CUDA cores), and
-//             the mean up-projection W_bar_up and shared up-projection W_s_up
-//             (tensor cores) -> r, active, u = x W_bar_up^T, SiLU(x W_s_up^T)
-//   kd_up     W_up[e] of the union of active experts (tensor cores) -> g
-//   kd_down   units of 128 output rows of one active expert's W_down (or of a
-//             256-column part of W_s_down) arrive as TMA boxes; the CTA computes
-//             the expert's NormSiLU (subtract u, RMS over d_e, SiLU, times
-//             s_e r_e) when the expert changes and writes fp32 partials
-//   kd_combine adds the shared-expert parts and the active experts' partials
-//             in ascending expert order (+ the residual)
+//   phase R  CTAs [0, Cr): the router rows W_r (exact activation decisions on
+//            CUDA cores, see common.cuh) -> r, active.  The other CTAs: the
+//            rows of [W_bar_up ; W_s_up] -> u = x W_bar_up^T and the shared
+//            hidden SiLU(x W_s_up^T), kept as bf16 hi/lo tiles.
+//   phase U  after the router: the union of the batch's active experts; units
+//            (expert, 128 rows of W_up[e], K part) -> fp32 partial sums of
+//            g = x W_up[e]^T.  The CTA that completes an expert's last unit
+//            computes its NormSiLU for every token using it (subtract u, RMS
+//            over d_e, SiLU, times s_e r_e) as a bf16 hi/lo tile.
+//   phase D  units (128 output rows, then one K part of W_s_down or one active
+//            expert's W_down[e] in ascending order); a CTA adds its
+//            consecutive units of one row block in its tensor-core
+//            accumulators and writes one fp32 partial per row block.  The CTA
+//            that completes a row block adds its partials in CTA order (+ the
+//            residual) and writes the output rows: a fixed order, so the
+//            result is bitwise reproducible.
 //
-// Data movement: one CTA per SM, 8 consumer warps and 1 producer warp.  The
-// producer streams contiguous weight rows with bulk copies of >= 4 KB each
-// (cp.async.bulk, L2 evict-first) into a ring of shared-memory stages behind
-// mbarriers; on B200 a copy engine sustains HBM bandwidth with copies this
-// size, while small tensor-map boxes (2 KB) are limited by per-copy cost.
-// kd_route / kd_up give each CTA a contiguous range of weight rows at full
-// width and copy each row into a 16-byte padded shared-memory row, so that
-// ldmatrix reads of 8 rows hit 8 different bank groups; the 8 consumer warps
-// split the columns and add their partial sums in warp order.  kd_down loads
-// 128-row x 64-column tiles with TMA in the 128-byte swizzle, which ldmatrix
-// reads directly; each consumer warp owns 16 of the 128 rows.
-// Activations a later kernel consumes are written in a layout its ldmatrix
-// reads can use directly (an XOR swizzle of the 16-byte chunks inside each
-// row).
+// The same kernel with no routed experts is the equal-parameter dense FFN at
+// decode batch sizes.
 //
-// Arithmetic: the projections are thin dense contractions (up to 16 tokens
-// against 8-row chunks or 128-row units of weights) done with mma.sync
-// m16n8k16 (bf16 in, fp32 accumulate) with the weights as A: a tensor-core
-// instruction per 16x8x16 tile keeps the instruction count far below the
-// memory time, which is the bound at these batch sizes.
-// Intermediates fed back into a contraction (the shared expert's hidden
-// activations and the scaled NormSiLU outputs) are stored as a bf16 pair
+// Data movement: 8 consumer warps and 1 producer warp per CTA.  The producer
+// streams the CTA's weights in one continuous sequence of 33 KB stages behind
+// mbarriers: phase R rows as bulk copies into 16-byte padded rows, phase U
+// and D tiles as 128-row x 64-column TMA boxes in the 128-byte swizzle
+// (ldmatrix reads both without bank conflicts).  It needs only the union of
+// active experts, so the W_up and W_down streams run ahead of the consumers'
+// dependencies.  x stays resident in shared memory during phases R and U; in
+// phase D the consumers fetch each unit's 16 KB activation tile with cp.async
+// one unit ahead.
+//
+// Arithmetic: the projections are thin dense contractions done with mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate), weights as A, tokens as B: one
+// tensor-core instruction per 16x8x16 tile keeps the instruction count well
+// below the memory time.  Intermediates fed back into a contraction (the
+// shared hidden activations and the scaled NormSiLU outputs) are bf16 pairs
 // hi + lo with lo = bf16(v - hi), and both halves are multiplied, so they
 // carry ~16 significant bits instead of 8.
 //
-// Waits are bounded: after ~1 s a wait gives up, sets bit 2 of the device
-// error word and the CTA stops issuing work (no hang, no trap).  Consecutive
-// kernels use programmatic dependent launch.
+// Waits are bounded: after about a second a wait gives up, sets bit 2 of the
+// device error word and the CTA stops issuing work; before it exits it waits
+// (again bounded) for every copy it issued.  No trap, no assert.
 #pragma once
 
 #include <cuda.h>
@@ -56,14 +61,22 @@ namespace deco {
 namespace dec {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kMaxT = 16;                      // decode batches
 constexpr int kTok = 16;                       // token rows of every activation tile
-constexpr uint32_t kStageBytes = 32768;
+constexpr uint32_t kBoxStage = 32768;          // two 128 x 64 TMA boxes
+constexpr uint32_t kStageBytes = 33792;        // a ring stage: boxes, or <= 8 padded rows of <= 4 KB
 constexpr int kMaxStages = 8;
 constexpr size_t kSmemLimit = 232448;          // 227 KB opt-in per CTA on sm_100
 constexpr long long kWaitCycles = 2000000000ll;  // ~1 s at 1.9 GHz
 constexpr int kErrTimeout = 2;
+constexpr int kMaxSms = 160;                  // kd_layer grids (one CTA per SM) up to this size
+constexpr int kDRows = 128;                    // weight rows per unit (phases U and D)
+constexpr uint32_t kBoxBytes = kDRows * 128;   // 128 rows x 64 bf16 columns
+constexpr int kSq = 256;                       // K columns per shared-expert down unit
+constexpr int kTileElems = kTok * 2 * kSq;     // activation tile: 16 rows x (256 hi | 256 lo) bf16
+constexpr uint32_t kTileBytes = kTileElems * 2;
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -92,20 +105,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait for the phase with `parity` to complete.  Returns false (and
-// flags the CTA-wide abort word and the device error word) on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err) {
+// flags the CTA-wide abort word and the device error word) on timeout, or
+// when another thread of the CTA has aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                          long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       atomicOr(err, kErrTimeout);
       return false;
     }
   }
   return true;
+}
+// Bounded wait that ignores the abort word: the drain of copies already
+// issued, before a CTA that gave up exits.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity) && clock64() - t0 < kWaitCycles) {
+  }
 }
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t p;
@@ -147,10 +168,54 @@ __device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int co
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 __device__ __forceinline__ void consumer_sync() {   // the 8 consumer warps only
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+}
+// 16-byte global -> shared copy through L2 (generic proxy; cp.async.wait_group)
+__device__ __forceinline__ void cp_async16_cg(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// arrive on `bar` once this thread's cp.async copies so far have landed
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// inter-CTA counters (global memory, gpu scope)
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait (one thread) until *p >= target.  Returns false on timeout
+// (setting the abort and error words) or when the CTA has aborted.
+__device__ __forceinline__ bool spin_until(const unsigned* p, unsigned target, long long limit,
+                                           volatile int* abort_flag, int* err) {
+  if (ld_acquire(p) >= target) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(40);
+    if (ld_acquire(p) >= target) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit) {
+      *abort_flag = 1;
+      atomicOr(err, kErrTimeout);
+      return false;
+    }
+  }
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -180,21 +245,17 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk) {
   return base + (uint32_t)row * 128u + ((uint32_t)(chunk ^ (row & 7)) << 4);
 }
 
+// physical 16-byte chunk of logical chunk k in a row with index r: the low 3
+// bits are XOR-ed with the row index, so 8 consecutive rows of one logical
+// chunk sit in 8 different bank groups
+__host__ __device__ __forceinline__ int row_chunk(int r, int k) { return (k & ~7) | ((k ^ r) & 7); }
+
 // ---------------------------------------------------------------------------
-// Ring of weight stages shared by the three streaming kernels.
+// Shared-memory plan: [<= 1 KB alignment slack][barriers 1 KB][ring][operand].
+// kStaticReserve bytes are left for the kernels' static __shared__ arrays.
 
-struct Ring {
-  uint64_t* full;    // [kMaxStages]
-  uint64_t* empty;   // [kMaxStages]
-  unsigned char* stage;
-  uint32_t stage_bytes;
-  int nstages;
-};
-
-// dynamic shared memory: [<=1 KB alignment slack][barriers 1 KB][ring][operand];
-// kStaticReserve bytes are left for each kernel's static __shared__ arrays.
 constexpr uint32_t kHeaderBytes = 1024;
-constexpr uint32_t kStaticReserve = 1536;
+constexpr uint32_t kStaticReserve = 2048;
 
 struct SmemPlan {
   uint32_t ring_off, op_off, total, stage_bytes;
@@ -214,30 +275,40 @@ __host__ __device__ inline SmemPlan smem_plan(uint32_t operand_bytes, uint32_t s
   return p;
 }
 
-// barriers: full[8], empty[8], opbar, abort word; returns the 1024-B aligned base
-__device__ __forceinline__ unsigned char* ring_setup(unsigned char* smem_raw, const SmemPlan& sp, Ring& ring,
-                                                     uint64_t*& opbar, volatile int*& abort_flag) {
-  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-  ring.full = bars;
-  ring.empty = bars + kMaxStages;
-  opbar = bars + 2 * kMaxStages;
-  abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kMaxStages + 1);
-  ring.stage = smem + sp.ring_off;
-  ring.stage_bytes = sp.stage_bytes;
-  ring.nstages = sp.nstages;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kMaxStages; ++s) {
-      mbar_init(&ring.full[s], 1);
-      mbar_init(&ring.empty[s], kConsumerWarps);
-    }
-    mbar_init(opbar, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-  return smem;
+// Padded token rows of x: row t at t * x_pitch, so that ldmatrix reads of 8
+// rows at one 16-byte column hit 8 different bank groups.
+__host__ __device__ inline uint32_t x_pitch(int D) { return (uint32_t)D * 2u + 16u; }
+// phase R streams <= 8 (D <= 2048) or 4 (D <= 4096) padded weight rows per stage
+__host__ __device__ inline int rows_per_chunk(int D) { return D <= 2048 ? 8 : 4; }
+// the operand region: 16 padded x rows and the 4 KB cross-warp reduction
+// scratch (phases R, U), later two activation tiles (phase D)
+__host__ __device__ inline uint32_t operand_bytes(int D) {
+  const uint32_t xr = kTok * x_pitch(D) + 4096u;
+  return xr > 2u * kTileBytes ? xr : 2u * kTileBytes;
 }
+__host__ __device__ inline SmemPlan layer_smem(int D) { return smem_plan(operand_bytes(D), kStageBytes); }
+// phase-D activation tiles that fit the operand region (2..4)
+__host__ __device__ inline int tile_slots(int D) {
+  const int n = (int)(operand_bytes(D) / (uint32_t)kTileBytes);
+  return n < 4 ? n : 4;
+}
+
+// router CTAs of phase R: one router row each (E <= 64), else several
+__host__ __device__ inline int router_ctas(int E) { return E < 64 ? E : 64; }
+
+// K parts of phase U: the smallest power of two (<= 8) that gives every CTA
+// at least two units, while a part keeps >= 256 columns
+__host__ __device__ inline int up_kparts(int U, int d_e, int D, int G) {
+  const int units = U * ((d_e + kDRows - 1) / kDRows);
+  int kp = 1;
+  while (kp < 8 && D / (2 * kp) >= 256 && units * kp < 2 * G) kp *= 2;
+  return kp;
+}
+__host__ __device__ inline int down_nsq(int d_s) { return (d_s + kSq - 1) / kSq; }
+
+// the contiguous unit range [u0, u1) of CTA c among G (c * n < 2^31 for every
+// count of units or rows here: n <= 2^17, G <= kMaxSms)
+__host__ __device__ inline int range_lo(int c, int n, int G) { return c * n / G; }
 
 // ---------------------------------------------------------------------------
 
@@ -245,6 +316,8 @@ struct Args {
   int T, D, E, d_e, d_s;
   float eps;
   int residual;
+  long long wait_cycles;   // limit of the waits for data (kWaitCycles unless a test lowers it)
+  int pre_routed;          // r and act come from earlier kernels (TopK routing): no router CTAs
   const bf16* x;
   const bf16* W_r;
   const float* b_r;
@@ -257,46 +330,40 @@ struct Args {
   float* r;          // [T][E]
   uint8_t* act;      // [T][E]
   float* u;          // [T][d_e]
-  bf16* hs;          // [16 tok][hi d_s | lo d_s], chunk-swizzled rows: SiLU(x W_s_up^T)
-  float* C;          // [kp <= 8][E][16 tok][d_e] up-projection g = x W_up[e]^T (active experts),
-                     // partial sums over K parts
-  float* P;          // [E][16 slots][D] routed down-projection partials, slot i = the i-th
-                     // active token of expert e (ascending)
-  float* Ps;         // [ceil(d_s / 256)][16 tok][D] shared down-projection partials
+  bf16* HS;          // [nsq][16 tok][256 hi | 256 lo], chunk-swizzled rows: SiLU(x W_s_up^T)
+  bf16* A;           // [E][16 tok][256 hi | 256 lo]: s_e r_e NormSiLU(x W_up[e]^T), 0 for
+                     // tokens not using e
+  float* C;          // [kp <= 8][E][16 tok][d_e]: partial sums of x W_up[e]^T over K parts
+  float* Part;       // [G][2][16 tok][128]: a CTA's down-projection sum per row block
+  unsigned* sync;    // inter-CTA counters, zero at launch (layout: SyncIdx)
   int* err;
   bf16* out;
 };
 
-// physical 16-byte chunk of logical chunk k in a row with index r: the low 3
-// bits are XOR-ed with the row index, so 8 consecutive rows of one logical
-// chunk sit in 8 different bank groups
-__host__ __device__ __forceinline__ int row_chunk(int r, int k) { return (k & ~7) | ((k ^ r) & 7); }
-
-// per-expert token masks and the ascending list of experts some token uses
-__device__ __forceinline__ void build_union(const Args& a, uint16_t* emask, uint8_t* ulist, int* U) {
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-    uint16_t m = 0;
-    for (int t = 0; t < a.T; ++t)
-      if (__ldcg(a.act + (size_t)t * a.E + e)) m |= (uint16_t)(1u << t);
-    emask[e] = m;
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    int n = 0;
-    for (int base = 0; base < a.E; base += 32) {
-      const int e = base + lane;
-      const bool f = e < a.E && emask[e] != 0;
-      const unsigned bal = __ballot_sync(kFull, f);
-      if (f) ulist[n + __popc(bal & ((1u << lane) - 1u))] = (uint8_t)e;
-      n += __popc(bal);
-    }
-    if (lane == 0) *U = n;
-  }
-  __syncthreads();
+// counters: routed CTAs done, phase-R rows done, up units done per expert,
+// NormSiLU tile ready per expert, CTAs done per output row block
+struct SyncIdx {
+  int route_done, pre_done, g_cnt, a_ready, rb_cnt, total;
+};
+__host__ __device__ inline SyncIdx sync_idx(int E, int D) {
+  SyncIdx s;
+  s.route_done = 0;
+  s.pre_done = 1;
+  s.g_cnt = 2;
+  s.a_ready = 2 + E;
+  s.rb_cnt = 2 + 2 * E;
+  s.total = 2 + 2 * E + D / kDRows;
+  return s;
 }
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& q, float (&v)[8]) { unpack16(q, v); }
+// v as a bf16 pair (hi, lo = v - hi) at element j of a chunk-swizzled row of
+// 2L elements (hi part [0, L), lo part [L, 2L)); r is the row index
+__device__ __forceinline__ void store_row_hi_lo(bf16* row, int r, int L, int j, float v) {
+  const bf16 hi = __float2bfloat16_rn(v);
+  const bf16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+  row[row_chunk(r, j >> 3) * 8 + (j & 7)] = hi;
+  row[row_chunk(r, (L + j) >> 3) * 8 + (j & 7)] = lo;
+}
 
 // Reduce N = 2^m per-lane values across the warp: at each of the first m
 // levels a lane keeps one half of its values, sends the other half to its
@@ -328,27 +395,12 @@ __device__ __forceinline__ float warp_reduce_scatter(float (&v)[N], int lane) {
   return v[0];
 }
 
-// v as a bf16 pair (hi, lo = v - hi) at element j of a chunk-swizzled row of
-// 2L elements (hi part [0, L), lo part [L, 2L)); r is the row index
-__device__ __forceinline__ void store_row_hi_lo(bf16* row, int r, int L, int j, float v) {
-  const bf16 hi = __float2bfloat16_rn(v);
-  const bf16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-  row[row_chunk(r, j >> 3) * 8 + (j & 7)] = hi;
-  row[row_chunk(r, (L + j) >> 3) * 8 + (j & 7)] = lo;
-}
-
 // ---------------------------------------------------------------------------
-// Row-range streaming (kd_route, kd_up): a CTA's rows are taken in chunks of
-// `rc` rows (one stage), each row one bulk copy into a padded smem row of
-// pitch D*2 + 16 bytes.  For a chunk, warp w multiplies the 16 token rows of x
-// by the chunk's rows over columns [w*D/8, (w+1)*D/8): one m16n8 tile per
+// Phase R, padded weight rows (the rows of [W_bar_up ; W_s_up]): a CTA's rows
+// come in chunks of rc rows (one stage), each row one bulk copy into a padded
+// shared-memory row.  For a chunk, warp w multiplies the 16 token rows of x by
+// the chunk's rows over columns [w*D/8, (w+1)*D/8): one m16n8 tile per
 // 16-column step.  The 8 warps' 16 x 8 results are then added in warp order.
-
-__host__ __device__ inline uint32_t x_pitch(int D) { return (uint32_t)D * 2u + 16u; }
-__host__ __device__ inline int rows_per_chunk(int D) { return D <= 2048 ? 8 : 4; }
-__host__ __device__ inline uint32_t row_stage_bytes(int D) {
-  return ((uint32_t)rows_per_chunk(D) * x_pitch(D) + 1023u) & ~1023u;
-}
 
 __device__ __forceinline__ uint32_t x_addr(uint32_t xs, uint32_t pitch, int lane, int chunk) {
   return xs + (uint32_t)((lane & 7) + ((lane >> 3) & 1) * 8) * pitch + (uint32_t)(chunk + (lane >> 4)) * 16u;
@@ -367,15 +419,15 @@ __device__ __forceinline__ void stage_x(const Args& a, unsigned char* xs, uint64
   for (int t = 0; t < a.T; ++t) bulk_g2s(xs + (size_t)t * pitch, a.x + (size_t)t * a.D, (uint32_t)a.D * 2, bar);
 }
 // zero the rows T..15 of the 16-row x operand (consumer threads)
-__device__ __forceinline__ void zero_x_tail(const Args& a, unsigned char* xs, int tid, int nthreads) {
+__device__ __forceinline__ void zero_x_tail(const Args& a, unsigned char* xs) {
   const uint32_t pitch = x_pitch(a.D);
   const int words = (int)(pitch / 16);
-  for (int i = tid; i < (kTok - a.T) * words; i += nthreads)
+  for (int i = threadIdx.x; i < (kTok - a.T) * words; i += kConsumerThreads)
     reinterpret_cast<uint4*>(xs + (size_t)(a.T + i / words) * pitch)[i % words] = make_uint4(0u, 0u, 0u, 0u);
 }
 
-// y[16 tok][8 rows] for one chunk; returns in `red_out` (thread o < 128 of the
-// consumer warps gets output o = tok*8 + row)
+// y[16 tok][8 rows] for one chunk; thread o < 128 of the consumer warps gets
+// output o = tok * 8 + row
 __device__ __forceinline__ float chunk_gemv(uint32_t xs, uint32_t ws, uint32_t pitch, int D, int warp, int lane,
                                             float* red, bool math) {
   const int rc = rows_per_chunk(D);
@@ -405,567 +457,738 @@ __device__ __forceinline__ float chunk_gemv(uint32_t xs, uint32_t ws, uint32_t p
 }
 
 // ---------------------------------------------------------------------------
-// kd_route
-//
-// CTAs [0, Cr) with Cr = min(E, 64): router rows on CUDA cores with an exact
-// sign decision (see common.cuh), the 8 warps of a CTA splitting each row's
-// columns.  The remaining CTAs split the rows of [W_bar_up ; W_s_up] evenly
-// and write u = x W_bar_up^T and SiLU(x W_s_up^T) (as hi/lo pairs) for them.
+// Router rows (phase R of CTAs [0, Cr), and the routing-only kernel): rows
+// e = c + Cr i of W_r, packed in one stage; for each row the 8 consumer warps
+// split the D columns (16-byte chunks), and their partial sums are added in
+// warp order.  The activation decision is exact: the fp32 sum comes with a
+// rigorous error bound and, inside it, the sign is settled by exact integer
+// accumulation (common.cuh).
 
-// router CTAs of kd_route: one router row each (E <= 64), else several
-__host__ __device__ inline int router_ctas(int E) { return E < 64 ? E : 64; }
+__device__ __forceinline__ int router_rows(const Args& a, int c, int Cr) { return (a.E - c + Cr - 1) / Cr; }
 
-__global__ void __launch_bounds__(kThreads, 1) kd_route(const __grid_constant__ Args a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  __shared__ unsigned long long limbs[1][kLimbs];
-  const int Cr = router_ctas(a.E);
-  const bool router_cta = (int)blockIdx.x < Cr;
-  const uint32_t pitch = x_pitch(a.D);
-  // operand: x rows, then the 4 KB cross-warp reduction scratch
-  const SmemPlan sp = smem_plan(kTok * pitch + 4096, router_cta ? kStageBytes : row_stage_bytes(a.D));
-  Ring ring;
-  uint64_t* xbar;
-  volatile int* abort_flag;
-  unsigned char* smem = ring_setup(smem_raw, sp, ring, xbar, abort_flag);
-  unsigned char* xsm = smem + sp.op_off;
-  float* red = reinterpret_cast<float*>(xsm + kTok * pitch);
+// producer side: x and the router rows of CTA c into stage 0 (one thread)
+__device__ __forceinline__ void issue_router(const Args& a, int c, int Cr, unsigned char* xsm, uint64_t* xbar,
+                                             unsigned char* stage, uint64_t* full, uint64_t pol) {
+  const int nrow = router_rows(a, c, Cr);
+  const uint32_t rowbytes = (uint32_t)a.D * 2;
+  stage_x(a, xsm, xbar);
+  mbar_expect_tx(full, nrow * rowbytes);
+  for (int j = 0; j < nrow; ++j)
+    bulk_g2s(stage + (size_t)j * rowbytes, a.W_r + (size_t)(c + Cr * j) * a.D, rowbytes, full, pol);
+}
+
+// consumer side: r and active of the CTA's rows for every token (8 warps);
+// `ok` says the stage and x are in shared memory
+__device__ __forceinline__ void route_rows(const Args& a, int c, int Cr, const unsigned char* xsm,
+                                           const unsigned char* stage, float* red, unsigned long long* limbs,
+                                           bool ok) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_trigger();
-
-  if (router_cta) {
-    // router rows e = blockIdx.x + Cr i; for each row the 8 consumer warps
-    // split the D columns (16-byte chunks), and their partial sums are added
-    // in warp order
-    const int nrow = (a.E - (int)blockIdx.x + Cr - 1) / Cr;
-    const uint32_t rowbytes = (uint32_t)a.D * 2;
-    const int per = (int)(kStageBytes / rowbytes);   // router rows per stage
-    const int nst = (nrow + per - 1) / per;
-    if (warp == kConsumerWarps) {
-      if (lane == 0) {
-        const uint64_t pol = evict_first_policy();
-        stage_x(a, xsm, xbar);
-        for (int k = 0; k < nst; ++k) {
-          const int n = min(per, nrow - k * per);
-          mbar_expect_tx(&ring.full[k], n * rowbytes);
-          for (int j = 0; j < n; ++j)
-            bulk_g2s(ring.stage + (size_t)k * kStageBytes + (size_t)j * rowbytes,
-                     a.W_r + (size_t)(blockIdx.x + Cr * (k * per + j)) * a.D, rowbytes, &ring.full[k], pol);
-        }
-      }
-      return;
-    }
-    // a value goes through <= 8 ceil(D / 2048) products in its lane, 5
-    // butterfly levels, 7 cross-warp additions and the bias
-    const int n_terms = 8 * ((a.D + 2047) / 2048) + 16;
-    const float gm = gamma_f32(n_terms);
-    const float bscale = 2.f * gm * (1.f + 2.f * gm);
-    const float tiny = float(n_terms) * 2.8025969e-45f;
-    bool bad = false;
-    // every consumer warp waits for x and for every stage, so every issued
-    // copy is awaited before the CTA exits
-    bool ok = mbar_wait(xbar, 0, abort_flag, a.err);
-    for (int k = 0; k < nst; ++k) ok = ok && mbar_wait(&ring.full[k], 0, abort_flag, a.err);
-    for (int i = 0; i < nrow; ++i) {
-      const int e = blockIdx.x + Cr * i;
-      const bf16* wrow =
-          reinterpret_cast<const bf16*>(ring.stage + (size_t)(i / per) * kStageBytes + (size_t)(i % per) * rowbytes);
-      float v[32];
+  const uint32_t pitch = x_pitch(a.D);
+  const int nrow = router_rows(a, c, Cr);
+  // a value goes through <= 8 ceil(D / 2048) products in its lane, 5
+  // butterfly levels, 7 cross-warp additions and the bias
+  const int n_terms = 8 * ((a.D + 2047) / 2048) + 16;
+  const float gm = gamma_f32(n_terms);
+  const float bscale = 2.f * gm * (1.f + 2.f * gm);
+  const float tiny = float(n_terms) * 2.8025969e-45f;
+  bool bad = false;
+  for (int i = 0; i < nrow; ++i) {
+    const int e = c + Cr * i;
+    const bf16* wrow = reinterpret_cast<const bf16*>(stage + (size_t)i * a.D * 2);
+    float v[32];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) v[q] = 0.f;
-      // z partials in v[t], sum |x w| partials in v[16 + t]
-      if (ok) {
+    for (int q = 0; q < 32; ++q) v[q] = 0.f;
+    // z partials in v[t], sum |x w| partials in v[16 + t]
+    if (ok) {
 #pragma unroll 1
-        for (int ch = warp * 32 + lane; ch < a.D / 8; ch += kConsumerWarps * 32) {
-          float wv[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(wrow + (size_t)ch * 8), wv);
+      for (int ch = warp * 32 + lane; ch < a.D / 8; ch += kConsumerWarps * 32) {
+        float wv[8];
+        unpack16(*reinterpret_cast<const uint4*>(wrow + (size_t)ch * 8), wv);
 #pragma unroll
-          for (int t = 0; t < kTok; ++t) {
-            if (t < a.T) {
-              float xv[8];
-              bf16x8_to_f32(*reinterpret_cast<const uint4*>(xsm + (size_t)t * pitch + (size_t)ch * 16), xv);
+        for (int t = 0; t < kTok; ++t) {
+          if (t < a.T) {
+            float xv[8];
+            unpack16(*reinterpret_cast<const uint4*>(xsm + (size_t)t * pitch + (size_t)ch * 16), xv);
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                v[t] = fmaf(xv[q], wv[q], v[t]);
-                v[16 + t] = fmaf(fabsf(xv[q]), fabsf(wv[q]), v[16 + t]);
-              }
+            for (int q = 0; q < 8; ++q) {
+              v[t] = fmaf(xv[q], wv[q], v[t]);
+              v[16 + t] = fmaf(fabsf(xv[q]), fabsf(wv[q]), v[16 + t]);
             }
           }
         }
       }
-      red[warp * 32 + lane] = warp_reduce_scatter<32>(v, lane);   // lane l: this warp's value l
-      consumer_sync();
-      if (warp == 0 && ok) {
-        float tot = 0.f;
+    }
+    red[warp * 32 + lane] = warp_reduce_scatter<32>(v, lane);   // lane l: this warp's value l
+    consumer_sync();
+    if (warp == 0 && ok) {
+      float tot = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) tot += red[w * 32 + lane];
-        const float S = __shfl_sync(kFull, tot, (lane + 16) & 31);
-        const float b = a.b_r[e];
-        const int t = lane;
-        const bool mine = t < a.T;
-        const float z = tot + b;
-        const float B = bscale * (S + fabsf(b)) + tiny;
-        const bool sure = fabsf(z) > B;
-        bool on = sure && z > 0.f;
-        // guard band: exact re-evaluation of the sign, the whole warp per score
-        unsigned need = __ballot_sync(kFull, mine && !sure);
-        while (need) {
-          const int tt = __ffs(need) - 1;
-          need &= need - 1;
-          const int sg = exact_sign_warp(reinterpret_cast<const bf16*>(xsm + (size_t)tt * pitch), wrow, a.D, b,
-                                         limbs[0], &bad);
-          if (lane == tt) on = sg > 0;
-        }
-        if (mine) {
-          a.r[(size_t)t * a.E + e] = on ? fmaxf(z, 0.f) : 0.f;
-          a.act[(size_t)t * a.E + e] = on ? 1 : 0;
-        }
+      for (int w = 0; w < kConsumerWarps; ++w) tot += red[w * 32 + lane];
+      const float S = __shfl_sync(kFull, tot, (lane + 16) & 31);
+      const float b = a.b_r[e];
+      const int t = lane;
+      const bool mine = t < a.T;
+      const float z = tot + b;
+      const float B = bscale * (S + fabsf(b)) + tiny;
+      const bool sure = fabsf(z) > B;
+      bool on = sure && z > 0.f;
+      // guard band: exact re-evaluation of the sign, the whole warp per score
+      unsigned need = __ballot_sync(kFull, mine && !sure);
+      while (need) {
+        const int tt = __ffs(need) - 1;
+        need &= need - 1;
+        const int sg = exact_sign_warp(reinterpret_cast<const bf16*>(xsm + (size_t)tt * pitch), wrow, a.D, b,
+                                       limbs, &bad);
+        if (lane == tt) on = sg > 0;
       }
-      consumer_sync();   // red is reused by the next row
-    }
-    if (bad && lane == 0) atomicOr(a.err, 1);
-    return;
-  }
-
-  // rows of [W_bar_up ; W_s_up], split evenly over the remaining CTAs
-  const int nrows = a.d_e + a.d_s;
-  const int G = gridDim.x - Cr, c = blockIdx.x - Cr;
-  const int ra = (int)((long long)c * nrows / G), rb = (int)((long long)(c + 1) * nrows / G);
-  const int rc = rows_per_chunk(a.D);
-  const int nchunks = (rb - ra + rc - 1) / rc;
-  auto row_src = [&](int g) -> const bf16* {
-    return g < a.d_e ? a.W_bar + (size_t)g * a.D : a.W_s_up + (size_t)(g - a.d_e) * a.D;
-  };
-  if (warp == kConsumerWarps) {
-    if (lane == 0 && nchunks > 0) {
-      const uint64_t pol = evict_first_policy();
-      stage_x(a, xsm, xbar);
-      for (int k = 0; k < nchunks; ++k) {
-        const int s = k % ring.nstages;
-        if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
-        const int g0 = ra + k * rc, n = min(rc, rb - g0);
-        mbar_expect_tx(&ring.full[s], (uint32_t)n * a.D * 2);
-        for (int i = 0; i < n; ++i)
-          bulk_g2s(ring.stage + (size_t)s * ring.stage_bytes + (size_t)i * pitch, row_src(g0 + i),
-                   (uint32_t)a.D * 2, &ring.full[s], pol);
+      if (mine) {
+        a.r[(size_t)t * a.E + e] = on ? fmaxf(z, 0.f) : 0.f;
+        a.act[(size_t)t * a.E + e] = on ? 1 : 0;
       }
     }
-    return;
+    consumer_sync();   // red is reused by the next row
   }
-  if (nchunks == 0) return;
-  zero_x_tail(a, xsm, threadIdx.x, kConsumerWarps * 32);
-  consumer_sync();
-  bool ok = mbar_wait(xbar, 0, abort_flag, a.err);
-  for (int k = 0; k < nchunks; ++k) {
-    const int s = k % ring.nstages;
-    ok = ok && mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err);
-    const float v = chunk_gemv(smem_u32(xsm), smem_u32(ring.stage + (size_t)s * ring.stage_bytes), pitch, a.D,
-                               warp, lane, red, ok);
-    if (ok && lane == 0) mbar_arrive(&ring.empty[s]);
-    const int o = threadIdx.x;
-    const int t = o >> 3, i = o & 7;
-    const int g = ra + k * rc + i;
-    if (ok && o < 128 && i < rc && g < rb) {
-      if (g < a.d_e) {
-        if (t < a.T) a.u[(size_t)t * a.d_e + g] = v;
-      } else {
-        const int j = g - a.d_e;   // shared hidden unit
-        store_row_hi_lo(a.hs + (size_t)t * 2 * a.d_s, t, a.d_s, j, t < a.T ? silu_f(v) : 0.f);
-      }
-    }
-  }
+  if (bad && (threadIdx.x & 31) == 0) atomicOr(a.err, 1);
 }
 
-// ---------------------------------------------------------------------------
-// kd_up: g = x W_up[e]^T for the experts some token uses, as fp32 partial
-// sums over K parts.  Units are (expert e of the union, block of 128 rows of
-// W_up[e], K part p of D / kp columns), with kp <= 8 the smallest power of
-// two that gives every CTA at least two units; CTA c takes a contiguous range
-// of them.  Weights arrive as 128 x 64 TMA boxes (two per 32 KB stage, the
-// 128-byte swizzle ldmatrix reads directly), x stays resident in padded
-// shared-memory rows, and consumer warp w multiplies rows 16w..16w+15 of the
-// unit by the 16 token rows.  Results go to C[p][e][t][j]; kd_down adds the
-// K parts in order.  (NormSiLU runs in kd_down.)
+// Barriers and bookkeeping kept in the 1 KB header: ring full/empty, x, the
+// union of active experts, the producer's last word (stages issued).
+constexpr int kTileSlots = 4;                  // phase-D activation tiles in flight (at most)
+constexpr int kLoaderLanes = 31;               // producer-warp lanes 1..31 load them
 
-constexpr int kDRows = 128;                  // weight rows per unit (kd_up, kd_down)
-constexpr uint32_t kBoxBytes = kDRows * 128; // 128 rows x 64 bf16 columns
-
-__host__ __device__ inline int up_kparts(int U, int d_e, int D, int G) {
-  const int units = U * ((d_e + kDRows - 1) / kDRows);
-  int kp = 1;
-  while (kp < 8 && D / (2 * kp) >= 256 && units * kp < 2 * G) kp *= 2;
-  return kp;
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-    kd_up(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ Args a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  __shared__ uint16_t emask[256];
-  __shared__ uint8_t ulist[256];
-  __shared__ int s_U;
-  const uint32_t pitch = x_pitch(a.D);
-  const SmemPlan sp = smem_plan(kTok * pitch, kStageBytes);
-  Ring ring;
+struct Ctl {
+  uint64_t* full;
+  uint64_t* empty;
   uint64_t* xbar;
+  uint64_t* ubar;
+  uint64_t* pbar;
+  uint64_t* xfree;   // consumers are done with x (its region then holds the tile ring)
+  uint64_t* tfull;   // [kTileSlots] activation tile landed
+  uint64_t* tempty;  // [kTileSlots] consumers done with the tile
   volatile int* abort_flag;
-  unsigned char* smem = ring_setup(smem_raw, sp, ring, xbar, abort_flag);
-  unsigned char* xsm = smem + sp.op_off;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // x does not depend on the router: stage it before waiting for it
-  if (threadIdx.x == 0) stage_x(a, xsm, xbar);
-  if (warp < kConsumerWarps) zero_x_tail(a, xsm, threadIdx.x, kConsumerWarps * 32);
-  pdl_wait();          // router outputs
-  pdl_trigger();
-  build_union(a, emask, ulist, &s_U);
-  const int nrb = (a.d_e + kDRows - 1) / kDRows;
-  const int kp = up_kparts(s_U, a.d_e, a.D, gridDim.x);
-  const int Kp = a.D / kp;
-  const int NU = s_U * nrb * kp;
-  const int u0 = (int)((long long)blockIdx.x * NU / gridDim.x);
-  const int u1 = (int)((long long)(blockIdx.x + 1) * NU / gridDim.x);
-  if (warp == kConsumerWarps) {
-    if (lane == 0) {
-      const uint64_t pol = evict_first_policy();
-      int k = 0;
-      for (int u = u0; u < u1; ++u) {
-        const int p = u % kp, rb = (u / kp) % nrb, e = ulist[u / (kp * nrb)];
-        const int row = e * a.d_e + rb * kDRows;
-        for (int c0 = 0; c0 < Kp; c0 += 128, ++k) {
-          const int s = k % ring.nstages;
-          if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
-          const int nb = min(2, (Kp - c0) / 64);
-          mbar_expect_tx(&ring.full[s], (uint32_t)nb * kBoxBytes);
-          for (int b = 0; b < nb; ++b)
-            tma_2d(ring.stage + (size_t)s * ring.stage_bytes + b * kBoxBytes, &tmU, p * Kp + c0 + 64 * b, row,
-                   &ring.full[s], pol);
-        }
-        if (*abort_flag) break;
-      }
-    }
-    return;
-  }
-  // the x copies were issued unconditionally: always await them
-  bool ok = mbar_wait(xbar, 0, abort_flag, a.err);
-  const uint32_t x_u32 = smem_u32(xsm);
-  const int ntiles = (a.T + 7) / 8;
-  int k = 0;
-  for (int u = u0; u < u1; ++u) {
-    const int p = u % kp, rb = (u / kp) % nrb, e = ulist[u / (kp * nrb)];
-    float acc[2][4] = {};
-    for (int c0 = 0; c0 < Kp; c0 += 128, ++k) {
-      const int s = k % ring.nstages;
-      ok = ok && mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err);
-      const int nb = min(2, (Kp - c0) / 64);
-      if (ok) {
-        const uint32_t st = smem_u32(ring.stage + (size_t)s * ring.stage_bytes);
-        for (int b = 0; b < nb; ++b) {
-          const uint32_t box = st + b * kBoxBytes;
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1, a2,
-                    a3);
-            const int kc = (p * Kp + c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-              if (nt < ntiles) {
-                uint32_t b0, b1;
-                ldsm_x2(x_u32 + (uint32_t)(8 * nt + (lane & 7)) * pitch + (uint32_t)kc * 16u, b0, b1);
-                mma16816(acc[nt], a0, a1, a2, a3, b0, b1);
-              }
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ring.empty[s]);
-    }
-    if (!ok) continue;
-    // acc[nt][i]: row 16 warp + lane/4 + 8 (i >> 1), token 8 nt + 2 (lane & 3) + (i & 1)
-    const int j0 = rb * kDRows + 16 * warp + (lane >> 2);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = 8 * nt + 2 * (lane & 3) + (i & 1);
-        const int j = j0 + 8 * (i >> 1);
-        if (t < a.T && j < a.d_e) a.C[(((size_t)p * a.E + e) * kTok + t) * a.d_e + j] = acc[nt][i];
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// kd_down: the routed and the shared down-projections as fp32 partial sums.
-//
-// Units are (expert e of the union, block of 128 output rows), with all of d_e
-// as K, and (K part q of 256 columns of W_s_down, block of 128 output rows)
-// for the shared expert.  CTA c takes a contiguous range of the units (shared
-// ones first, then experts ascending), so consecutive units mostly share an
-// expert.  A unit's weights arrive as TMA boxes of 128 rows x 64 columns
-// (16 KB, 128-byte swizzle, the layout ldmatrix reads without bank
-// conflicts), two boxes per 32 KB stage; consumer warp w multiplies the unit's
-// rows 16w..16w+15 (m16n8k16, weights as A, tokens as B).  B rows are the
-// shared expert's hidden activations (hi/lo, resident in shared memory) or the
-// expert's NormSiLU activations, which the CTA computes when the expert
-// changes: c = g - u, h = c / sqrt(mean c^2 + eps), a = s_e r_e SiLU(h), stored
-// as hi/lo in compact slots (slot i = the i-th active token of e).  Results go
-// to P[e][slot][row] and Ps[q][token][row]; kd_combine adds them.
-
-constexpr int kSq = 256;                     // K columns per shared-expert unit
-
-__host__ __device__ inline int down_nsq(int d_s) { return (d_s + kSq - 1) / kSq; }
-
-struct DUnit {
-  bool shared;
-  int e, q, rb, K, kb0;   // kb0: first K column of the unit within its matrix row
+  volatile int* k_issued;
+  int* bcast;        // [4] consumer broadcast words
+  unsigned char* stage;
+  uint32_t stage_bytes;
+  int nstages;
 };
 
-__device__ __forceinline__ DUnit down_unit(const Args& a, const uint8_t* ulist, int nrb, int u) {
+__device__ __forceinline__ unsigned char* ctl_setup(unsigned char* smem_raw, const SmemPlan& sp, Ctl& c) {
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+  c.full = bars;
+  c.empty = bars + kMaxStages;
+  c.xbar = bars + 2 * kMaxStages;
+  c.ubar = c.xbar + 1;
+  c.pbar = c.xbar + 2;
+  c.xfree = c.xbar + 3;
+  c.tfull = c.xbar + 4;
+  c.tempty = c.tfull + kTileSlots;
+  int* words = reinterpret_cast<int*>(c.tempty + kTileSlots);
+  c.abort_flag = words;
+  c.k_issued = words + 1;
+  c.bcast = words + 2;
+  c.stage = smem + sp.ring_off;
+  c.stage_bytes = sp.stage_bytes;
+  c.nstages = sp.nstages;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMaxStages; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], kConsumerWarps);
+    }
+    mbar_init(c.xbar, 1);
+    mbar_init(c.ubar, 1);
+    mbar_init(c.pbar, 1);
+    mbar_init(c.xfree, kConsumerWarps);
+    for (int s = 0; s < kTileSlots; ++s) {
+      mbar_init(&c.tfull[s], kLoaderLanes);
+      mbar_init(&c.tempty[s], kConsumerWarps);
+    }
+    *c.abort_flag = 0;
+    *c.k_issued = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  return smem;
+}
+
+// ---------------------------------------------------------------------------
+// Routing alone (deco_moe_routing on decode batches): the router CTAs of
+// kd_layer's phase R, with the same code, so the same decisions bit for bit.
+
+__global__ void __launch_bounds__(kThreads, 1) kd_router(const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ unsigned long long limbs[kLimbs];
+  const int Cr = router_ctas(a.E);
+  const SmemPlan sp = layer_smem(a.D);
+  Ctl ctl;
+  unsigned char* smem = ctl_setup(smem_raw, sp, ctl);
+  unsigned char* xsm = smem + sp.op_off;
+  float* red = reinterpret_cast<float*>(xsm + kTok * x_pitch(a.D));
+  const int warp = threadIdx.x >> 5;
+  if (warp == kConsumerWarps) {
+    if ((threadIdx.x & 31) == 0) issue_router(a, blockIdx.x, Cr, xsm, ctl.xbar, ctl.stage, &ctl.full[0],
+                                              evict_first_policy());
+    return;
+  }
+  // both waits always run (bounded), so every issued copy lands before exit
+  bool ok = mbar_wait(ctl.xbar, 0, ctl.abort_flag, a.err, a.wait_cycles);
+  ok = mbar_wait(&ctl.full[0], 0, ctl.abort_flag, a.err, a.wait_cycles) && ok;
+  ok = __all_sync(kFull, ok);   // warp-uniform: it guards warp-collective instructions
+  if (!ok && (threadIdx.x & 31) == 0) {
+    mbar_drain(ctl.xbar, 0);
+    mbar_drain(&ctl.full[0], 0);
+  }
+  route_rows(a, blockIdx.x, Cr, xsm, ctl.stage, red, limbs, ok);
+}
+
+// ---------------------------------------------------------------------------
+// The layer.
+
+// Unit of phase D: row block rb of the output, j < nsq a K part of W_s_down,
+// else the (j - nsq)-th active expert.
+struct DUnit {
+  int rb, j, e, K, col0;
+};
+__device__ __forceinline__ DUnit down_unit(const Args& a, const uint8_t* ulist, int nsq, int J, int u) {
   DUnit d;
-  const int ns = down_nsq(a.d_s) * nrb;
-  d.shared = u < ns;
-  if (d.shared) {
-    d.q = u / nrb;
-    d.rb = u - d.q * nrb;
-    d.kb0 = d.q * kSq;
-    d.K = min(kSq, a.d_s - d.kb0);
+  d.rb = u / J;
+  d.j = u - d.rb * J;
+  if (d.j < nsq) {
     d.e = -1;
+    d.col0 = d.j * kSq;
+    d.K = min(kSq, a.d_s - d.col0);
   } else {
-    const int v = u - ns, ui = v / nrb;
-    d.rb = v - ui * nrb;
-    d.e = ulist[ui];
-    d.q = 0;
-    d.kb0 = 0;
+    d.e = ulist[d.j - nsq];
+    d.col0 = 0;
     d.K = a.d_e;
   }
   return d;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    kd_down(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
-            const __grid_constant__ Args a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  __shared__ uint16_t emask[256];
-  __shared__ uint8_t ulist[256];
-  __shared__ int s_U;
-  // operand: hs rows (16 x 4 d_s bytes), the NormSiLU tile (16 x 4 d_e bytes),
-  // a zero row for slots past the expert's tokens (4 d_e <= 1 KB)
-  const uint32_t hbytes = (uint32_t)kTok * a.d_s * 4;
-  const uint32_t tbytes = (uint32_t)kTok * a.d_e * 4;
-  const SmemPlan sp = smem_plan(hbytes + tbytes + 1024, kStageBytes);
-  Ring ring;
-  uint64_t* hbar;
-  volatile int* abort_flag;
-  unsigned char* smem = ring_setup(smem_raw, sp, ring, hbar, abort_flag);
-  unsigned char* hsm = smem + sp.op_off;
-  unsigned char* tile = hsm + hbytes;
-  unsigned char* zrow = tile + tbytes;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_trigger();
-  for (int i = threadIdx.x; i < 1024 / 16; i += blockDim.x) reinterpret_cast<uint4*>(zrow)[i] = make_uint4(0, 0, 0, 0);
-  // The router's outputs are complete: this grid starts only after every CTA
-  // of kd_up passed its own wait on the router.
-  build_union(a, emask, ulist, &s_U);
-  const int nrb = a.D / kDRows;
-  const int NU = (down_nsq(a.d_s) + s_U) * nrb;
-  const int kp_up = up_kparts(s_U, a.d_e, a.D, gridDim.x);   // kd_up runs on the same grid
-  const int u0 = (int)((long long)blockIdx.x * NU / gridDim.x);
-  const int u1 = (int)((long long)(blockIdx.x + 1) * NU / gridDim.x);
-
-  if (warp == kConsumerWarps) {
-    if (lane == 0) {
-      const uint64_t pol = evict_first_policy();
-      mbar_expect_tx(hbar, hbytes);
-      bulk_g2s(hsm, a.hs, hbytes, hbar);
-      // weights do not depend on kd_up: they stream while it finishes
-      int k = 0;
-      for (int u = u0; u < u1; ++u) {
-        const DUnit d = down_unit(a, ulist, nrb, u);
-        const int row = d.shared ? d.rb * kDRows : d.e * a.D + d.rb * kDRows;
-        for (int c0 = 0; c0 < d.K; c0 += 128, ++k) {
-          const int s = k % ring.nstages;
-          if (!mbar_wait(&ring.empty[s], ((k / ring.nstages) & 1) ^ 1, abort_flag, a.err)) break;
-          const int nb = min(2, (d.K - c0) / 64);
-          mbar_expect_tx(&ring.full[s], (uint32_t)nb * kBoxBytes);
-          for (int b = 0; b < nb; ++b)
-            tma_2d(ring.stage + (size_t)s * ring.stage_bytes + b * kBoxBytes, d.shared ? &tmS : &tmW,
-                   d.kb0 + c0 + 64 * b, row, &ring.full[s], pol);
-        }
-        if (*abort_flag) break;
-      }
+// CTAs whose unit range meets row block rb, in ascending order (one warp:
+// lane l tests CTAs l, l + 32, ...); returns the count and fills
+// src[i] = 2 c + (slot of rb in c's partials)
+__device__ __forceinline__ int rb_sources(int rb, int J, int NU, int G, int* src) {
+  const int lane = threadIdx.x & 31;
+  int n = 0;
+  for (int c0 = 0; c0 < G; c0 += 32) {
+    const int c = c0 + lane;
+    bool hit = false;
+    int slot = 0;
+    if (c < G) {
+      const int v0 = range_lo(c, NU, G), v1 = range_lo(c + 1, NU, G);
+      hit = v0 < v1 && v0 < (rb + 1) * J && v1 > rb * J;
+      slot = rb - v0 / J;
     }
-    return;
+    const unsigned m = __ballot_sync(kFull, hit);
+    if (hit) src[n + __popc(m & ((1u << lane) - 1u))] = 2 * c + slot;
+    n += __popc(m);
   }
+  return n;
+}
 
-  pdl_wait();   // g (kd_up), u, r (kd_route)
-  bool ok = mbar_wait(hbar, 0, abort_flag, a.err);
-  const uint32_t hs_u32 = smem_u32(hsm), tile_u32 = smem_u32(tile), z_u32 = smem_u32(zrow);
-  int cur_e = -1, n_cur = 0, k = 0;
-  for (int u = u0; u < u1; ++u) {
-    const DUnit d = down_unit(a, ulist, nrb, u);
-    if (!d.shared && d.e != cur_e) {
-      // NormSiLU rows of expert e, one warp per active token
-      consumer_sync();   // every warp is done with the previous tile
-      const int e = d.e;
-      const uint32_t m_e = emask[e];
-      n_cur = __popc(m_e);
-      if (ok && !*abort_flag) {
-        for (int slot = warp; slot < n_cur; slot += kConsumerWarps) {
-          uint32_t m = m_e;
-          for (int i = 0; i < slot; ++i) m &= m - 1;
-          const int t = __ffs(m) - 1;
-          // every load of the token's row is issued before the first is used
-          const float rte = __ldcg(a.r + (size_t)t * a.E + e);
-          const float se = __ldg(a.s + e);
-          float gp[8][8], uq[8];   // [K part][value], d_e <= 256: 8 values per lane
+// NormSiLU tile of expert e (consumer threads): c = sum of the K parts of g
+// minus u, h = c / sqrt(mean c^2 + eps), a = s_e r_e SiLU(h) as hi/lo rows;
+// rows of tokens not using e are zero.
+__device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  bf16* tile = a.A + (size_t)e * kTileElems;
+  for (int i = threadIdx.x; i < kTok * 64; i += kConsumerThreads) {   // 64 chunks of 16 B per row
+    const int t = i >> 6;
+    if (!((m_e >> t) & 1u)) reinterpret_cast<uint4*>(tile)[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  const int n_e = __popc(m_e);
+  for (int slot = warp; slot < n_e; slot += kConsumerWarps) {
+    uint32_t m = m_e;
+    for (int i = 0; i < slot; ++i) m &= m - 1;
+    const int t = __ffs(m) - 1;
+    // every load of the token's row is issued before the first is used
+    const float rte = __ldcg(a.r + (size_t)t * a.E + e);
+    const float se = __ldg(a.s + e);
+    float gp[8][8], uq[8];   // [K part][value], d_e <= 256: 8 values per lane
 #pragma unroll
-          for (int pp = 0; pp < 8; ++pp)
+    for (int pp = 0; pp < 8; ++pp)
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int j = lane + 32 * q;
-              gp[pp][q] = (pp < kp_up && j < a.d_e)
-                              ? __ldcg(a.C + (((size_t)pp * a.E + e) * kTok + t) * a.d_e + j) : 0.f;
-            }
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j = lane + 32 * q;
-            uq[q] = j < a.d_e ? __ldcg(a.u + (size_t)t * a.d_e + j) : 0.f;
-          }
-          float cv[8];
-          float ss = 0.f;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float g = 0.f;   // kd_up's K parts, in order (absent parts add an exact 0)
-#pragma unroll
-            for (int pp = 0; pp < 8; ++pp) g += gp[pp][q];
-            cv[q] = g - uq[q];
-            ss = fmaf(cv[q], cv[q], ss);
-          }
-          ss = warp_sum(ss);
-          const float rinv = 1.f / sqrtf(ss / float(a.d_e) + a.eps);
-          const float coef = se * rte;
-          bf16* row = reinterpret_cast<bf16*>(tile + (size_t)slot * 4 * a.d_e);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j = lane + 32 * q;
-            if (j < a.d_e) store_row_hi_lo(row, slot, a.d_e, j, coef * silu_f(cv[q] * rinv));
-          }
-        }
+      for (int q = 0; q < 8; ++q) {
+        const int j = lane + 32 * q;
+        gp[pp][q] = (pp < kp && j < a.d_e) ? __ldcg(a.C + (((size_t)pp * a.E + e) * kTok + t) * a.d_e + j) : 0.f;
       }
-      consumer_sync();
-      cur_e = e;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = lane + 32 * q;
+      uq[q] = j < a.d_e ? __ldcg(a.u + (size_t)t * a.d_e + j) : 0.f;
     }
-    // B rows of this unit: tokens (shared) or slots (routed); rows past n read zeros
-    const int n = d.shared ? a.T : n_cur;
-    const int ntiles = (n + 7) / 8;
-    const int L = d.shared ? a.d_s : a.d_e;            // hi half length of a B row
-    uint32_t brow[2];
-    int bsw[2];
+    float cv[8];
+    float ss = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int r = 8 * nt + (lane & 7);
-      // hidden rows of tokens >= T are zeros (kd_route writes all 16 rows)
-      const bool on = d.shared || r < n;
-      brow[nt] = on ? (d.shared ? hs_u32 : tile_u32) + (uint32_t)r * 4u * (uint32_t)L : z_u32;
-      bsw[nt] = on ? r : 0;
+    for (int q = 0; q < 8; ++q) {
+      float g = 0.f;   // the K parts in order (absent parts add an exact 0)
+#pragma unroll
+      for (int pp = 0; pp < 8; ++pp) g += gp[pp][q];
+      cv[q] = g - uq[q];
+      ss = fmaf(cv[q], cv[q], ss);
     }
-    const int kcb = d.kb0 / 8;                          // first 16-byte chunk of the unit in a B row
-    float acc[2][4] = {};
-    for (int c0 = 0; c0 < d.K; c0 += 128, ++k) {
-      const int s = k % ring.nstages;
-      ok = ok && mbar_wait(&ring.full[s], (k / ring.nstages) & 1, abort_flag, a.err);
-      const int nb = min(2, (d.K - c0) / 64);
-      if (ok) {
-        const uint32_t st = smem_u32(ring.stage + (size_t)s * ring.stage_bytes);
-        for (int b = 0; b < nb; ++b) {
-          const uint32_t box = st + b * kBoxBytes;
+    ss = warp_sum(ss);
+    const float rinv = 1.f / sqrtf(ss / float(a.d_e) + a.eps);
+    const float coef = se * rte;
+    bf16* row = tile + (size_t)t * 2 * kSq;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1, a2,
-                    a3);
-            const int kc = kcb + (c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-              if (nt < ntiles) {
-                uint32_t bh0, bh1, bl0, bl1;
-                ldsm_x2(brow[nt] + (uint32_t)row_chunk(bsw[nt], kc) * 16u, bh0, bh1);
-                ldsm_x2(brow[nt] + (uint32_t)row_chunk(bsw[nt], kc + L / 8) * 16u, bl0, bl1);
-                mma16816(acc[nt], a0, a1, a2, a3, bh0, bh1);
-                mma16816(acc[nt], a0, a1, a2, a3, bl0, bl1);
-              }
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ring.empty[s]);
-    }
-    if (!ok) continue;
-    // acc[nt][i]: row 16 warp + lane/4 + 8 (i >> 1), column 8 nt + 2 (lane & 3) + (i & 1)
-    const int r0 = d.rb * kDRows + 16 * warp + (lane >> 2);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int col = 8 * nt + 2 * (lane & 3) + (i & 1);
-        const int row = r0 + 8 * (i >> 1);
-        if (col < n) {
-          float* dst = d.shared ? a.Ps + ((size_t)d.q * kTok + col) * a.D
-                                : a.P + ((size_t)d.e * kTok + col) * a.D;
-          dst[row] = acc[nt][i];
-        }
-      }
+    for (int q = 0; q < 8; ++q) {
+      const int j = lane + 32 * q;
+      if (j < a.d_e) store_row_hi_lo(row, t, kSq, j, coef * silu_f(cv[q] * rinv));
     }
   }
 }
 
-// ---------------------------------------------------------------------------
-// kd_combine: out[t][row] = sum over the shared-expert K parts q of Ps[q][t][row]
-// + sum over t's active experts e, ascending, of P[e][slot][row] (+ x[t][row]);
-// a fixed order, so the result is bitwise reproducible.
-
-__global__ void __launch_bounds__(256) kd_combine(const __grid_constant__ Args a) {
-  __shared__ int list_e[256], list_s[256], n_list;
-  const int t = blockIdx.y, lane = threadIdx.x & 31;
-  // The router's outputs are complete: this grid starts only after every CTA
-  // of kd_down started, and kd_down starts only after kd_up passed its wait on
-  // the router.  The token's expert list is built while kd_down finishes.
-  if (threadIdx.x < 32) {
-    int n = 0;
-    for (int e0 = 0; e0 < a.E; e0 += 32) {
-      const int e = e0 + lane;
-      uint32_t toks = 0;   // tokens using e (all flags loaded before any is used)
-      if (e < a.E) {
-        uint8_t fl[kTok];
+// out rows of row block rb: the sources' partials in CTA order (+ x)
+__device__ void combine_rb(const Args& a, int rb, const int* src, int n) {
+  const int n4 = a.T * (kDRows / 4);
+  for (int o = threadIdx.x; o < n4; o += kConsumerThreads) {
+    const int t = o / (kDRows / 4), q = o - t * (kDRows / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int i = 0;
+    for (; i + 4 <= n; i += 4) {
+      float4 v[4];
 #pragma unroll
-        for (int tp = 0; tp < kTok; ++tp) fl[tp] = tp < a.T ? __ldcg(a.act + (size_t)tp * a.E + e) : 0;
+      for (int k = 0; k < 4; ++k)
+        v[k] = __ldcg(reinterpret_cast<const float4*>(a.Part + ((size_t)src[i + k] * kTok + t) * kDRows) + q);
 #pragma unroll
-        for (int tp = 0; tp < kTok; ++tp) toks |= (fl[tp] ? 1u : 0u) << tp;
+      for (int k = 0; k < 4; ++k) {
+        acc.x += v[k].x;
+        acc.y += v[k].y;
+        acc.z += v[k].z;
+        acc.w += v[k].w;
       }
-      const bool f = (toks >> t) & 1u;
-      const int slot = __popc(toks & ((1u << t) - 1u));
-      const unsigned m = __ballot_sync(kFull, f);
-      if (f) {
-        const int i = n + __popc(m & ((1u << lane) - 1u));
-        list_e[i] = e;
-        list_s[i] = slot;
-      }
-      n += __popc(m);
     }
-    if (lane == 0) n_list = n;
+    for (; i < n; ++i) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(a.Part + ((size_t)src[i] * kTok + t) * kDRows) + q);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    const size_t o_idx = (size_t)t * a.D + (size_t)rb * kDRows + 4 * q;
+    if (a.residual) {
+      const uint2 xr = *reinterpret_cast<const uint2*>(a.x + o_idx);
+      acc.x += __uint_as_float(xr.x << 16);
+      acc.y += __uint_as_float(xr.x & 0xffff0000u);
+      acc.z += __uint_as_float(xr.y << 16);
+      acc.w += __uint_as_float(xr.y & 0xffff0000u);
+    }
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 w;
+    w.x = *reinterpret_cast<const uint32_t*>(&lo);
+    w.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(a.out + o_idx) = w;
   }
-  __syncthreads();
-  pdl_wait();   // the partials (kd_down)
-  const int row = blockIdx.x * 256 + threadIdx.x;
-  if (row >= a.D) return;
-  float v = 0.f;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    kd_layer(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmW,
+             const __grid_constant__ CUtensorMap tmS, const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ unsigned long long limbs[kLimbs];
+  __shared__ uint16_t emask[256];
+  __shared__ uint8_t ulist[256];
+  __shared__ int s_U;
+  __shared__ int s_src[kMaxSms];
+  const int G = gridDim.x, c = blockIdx.x;
+  const int Cr = (a.E > 0 && !a.pre_routed) ? router_ctas(a.E) : 0;
+  const bool router_cta = c < Cr;
+  const uint32_t pitch = x_pitch(a.D);
+  const SmemPlan sp = layer_smem(a.D);
+  if (threadIdx.x == 0) s_U = 0;   // read as 0 or the union's size, even by a consumer that gave up
+  Ctl ctl;
+  unsigned char* smem = ctl_setup(smem_raw, sp, ctl);
+  unsigned char* xsm = smem + sp.op_off;
+  float* red = reinterpret_cast<float*>(xsm + kTok * pitch);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SyncIdx si = sync_idx(a.E, a.D);
+  unsigned* sync = a.sync;
+  // phase R rows of a non-router CTA
+  const int nrows = a.d_e + a.d_s;
+  const int Gp = G - Cr, cp = c - Cr;
+  const int ra = router_cta ? 0 : range_lo(cp, nrows, Gp), rbr = router_cta ? 0 : range_lo(cp + 1, nrows, Gp);
+  const int rc = rows_per_chunk(a.D);
+  const int nchunks = (rbr - ra + rc - 1) / rc;
+  const int nrb_up = (a.d_e + kDRows - 1) / kDRows;
+  const int nrb = a.D / kDRows;
   const int nsq = down_nsq(a.d_s);
-  for (int q = 0; q < nsq; ++q) v += __ldcg(a.Ps + ((size_t)q * kTok + t) * a.D + row);
-  const int n = n_list;
-  for (int i = 0; i < n; ++i) v += __ldcg(a.P + ((size_t)list_e[i] * kTok + list_s[i]) * a.D + row);
-  if (a.residual) v += __bfloat162float(a.x[(size_t)t * a.D + row]);
-  a.out[(size_t)t * a.D + row] = __float2bfloat16_rn(v);
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer warp ----------------
+    const uint64_t pol = evict_first_policy();
+    int k = 0;
+    bool ok = true;
+    auto next_stage = [&](int& s) -> bool {   // lane 0: wait for a free stage
+      s = k % ctl.nstages;
+      return mbar_wait(&ctl.empty[s], ((k / ctl.nstages) & 1) ^ 1, ctl.abort_flag, a.err, a.wait_cycles);
+    };
+    if (lane == 0) {
+      if (router_cta) {
+        int s;
+        if ((ok = next_stage(s))) {   // the first round of stages is free
+          issue_router(a, c, Cr, xsm, ctl.xbar, ctl.stage + (size_t)s * ctl.stage_bytes, &ctl.full[s], pol);
+          ++k;
+        }
+      } else {
+        stage_x(a, xsm, ctl.xbar);
+        for (int ch = 0; ch < nchunks && ok; ++ch) {
+          int s;
+          if (!(ok = next_stage(s))) break;
+          const int g0 = ra + ch * rc, n = min(rc, rbr - g0);
+          mbar_expect_tx(&ctl.full[s], (uint32_t)n * a.D * 2);
+          for (int i = 0; i < n; ++i) {
+            const int g = g0 + i;
+            const bf16* src = g < a.d_e ? a.W_bar + (size_t)g * a.D : a.W_s_up + (size_t)(g - a.d_e) * a.D;
+            bulk_g2s(ctl.stage + (size_t)s * ctl.stage_bytes + (size_t)i * pitch, src, (uint32_t)a.D * 2,
+                     &ctl.full[s], pol);
+          }
+          ++k;
+        }
+      }
+      // the union of active experts needs every router row
+      if (ok) ok = spin_until(sync + si.route_done, (unsigned)Cr, a.wait_cycles, ctl.abort_flag, a.err);
+    }
+    ok = __shfl_sync(kFull, ok, 0);
+    if (ok) {
+      ld_acquire(sync + si.route_done);   // each lane acquires the router CTAs' writes itself
+      for (int e = lane; e < a.E; e += 32) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int t = 0; t < kTok; ++t)
+          if (t < a.T && __ldcg(a.act + (size_t)t * a.E + e)) m |= 1u << t;
+        emask[e] = (uint16_t)m;
+      }
+      __syncwarp();
+      int n = 0;
+      for (int base = 0; base < a.E; base += 32) {
+        const int e = base + lane;
+        const bool f = e < a.E && emask[e] != 0;
+        const unsigned bal = __ballot_sync(kFull, f);
+        if (f) ulist[n + __popc(bal & ((1u << lane) - 1u))] = (uint8_t)e;
+        n += __popc(bal);
+      }
+      if (lane == 0) s_U = n;
+    } else if (lane == 0) {
+      s_U = 0;
+    }
+    __syncwarp();
+    const int U = s_U;
+    if (lane != 0) {
+      // ---- lanes 1..31: the activation tile of each phase-D unit, in order,
+      // into the tile ring (the x region, once the consumers are done with x)
+      const int J = nsq + U, NUd = nrb * J;
+      const int v0 = range_lo(c, NUd, G), v1 = range_lo(c + 1, NUd, G);
+      const int nslots = tile_slots(a.D);
+      bool lok = ok && mbar_wait(ctl.xfree, 0, ctl.abort_flag, a.err, a.wait_cycles);
+      for (int v = v0; v < v1 && lok; ++v) {
+        const int i = v - v0, slot = i % nslots;
+        if (!(lok = mbar_wait(&ctl.tempty[slot], ((i / nslots) & 1) ^ 1, ctl.abort_flag, a.err, a.wait_cycles)))
+          break;
+        const DUnit d = down_unit(a, ulist, nsq, J, v);
+        const unsigned* f = d.e < 0 ? sync + si.pre_done : sync + si.a_ready + d.e;
+        if (!(lok = spin_until(f, d.e < 0 ? (unsigned)Gp : 1u, a.wait_cycles, ctl.abort_flag, a.err))) break;
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(
+            d.e < 0 ? a.HS + (size_t)d.j * kTileElems : a.A + (size_t)d.e * kTileElems);
+        unsigned char* dst = xsm + (size_t)slot * kTileBytes;
+        for (int q = lane - 1; q < (int)(kTileBytes / 16); q += kLoaderLanes)
+          cp_async16_cg(dst + (size_t)q * 16, src + (size_t)q * 16);
+        cp_async_mbar_arrive(&ctl.tfull[slot]);
+      }
+      cp_async_wait_all();   // every copy lands before the lane exits
+      return;
+    }
+    {
+      mbar_arrive(ctl.ubar);   // consumers read the union (or see the abort)
+      // phase U: W_up boxes
+      const int kp = up_kparts(U, a.d_e, a.D, G);
+      const int Kp = a.D / kp;
+      const int NUu = U * nrb_up * kp;
+      const int u0 = range_lo(c, NUu, G), u1 = range_lo(c + 1, NUu, G);
+      for (int u = u0; u < u1 && ok; ++u) {
+        const int p = u % kp, rbu = (u / kp) % nrb_up, e = ulist[u / (kp * nrb_up)];
+        const int row = e * a.d_e + rbu * kDRows;
+        for (int c0 = 0; c0 < Kp; c0 += 128) {
+          int s;
+          if (!(ok = next_stage(s))) break;
+          const int nb = min(2, (Kp - c0) / 64);
+          mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
+          for (int b = 0; b < nb; ++b)
+            tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, &tmU, p * Kp + c0 + 64 * b, row,
+                   &ctl.full[s], pol);
+          ++k;
+        }
+      }
+      // phase D: W_s_down / W_down boxes
+      const int J = nsq + U, NUd = nrb * J;
+      const int v0 = range_lo(c, NUd, G), v1 = range_lo(c + 1, NUd, G);
+      for (int v = v0; v < v1 && ok; ++v) {
+        const DUnit d = down_unit(a, ulist, nsq, J, v);
+        const bool sh = d.e < 0;
+        const int row = sh ? d.rb * kDRows : d.e * a.D + d.rb * kDRows;
+        for (int c0 = 0; c0 < d.K; c0 += 128) {
+          int s;
+          if (!(ok = next_stage(s))) break;
+          const int nb = min(2, (d.K - c0) / 64);
+          mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
+          for (int b = 0; b < nb; ++b)
+            tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, sh ? &tmS : &tmW,
+                   d.col0 + c0 + 64 * b, row, &ctl.full[s], pol);
+          ++k;
+        }
+      }
+      *ctl.k_issued = k;
+      mbar_arrive(ctl.pbar);
+    }
+    return;
+  }
+
+  // ---------------- consumer warps ----------------
+  const uint32_t x_u32 = smem_u32(xsm);
+  int k = 0;          // ring stages consumed
+  int k_ok = 0;       // stages whose data this thread saw arrive
+  bool ok = true;
+  // `ok` is kept warp-uniform (it guards ldmatrix / mma.sync / ballots); every
+  // consumer thread runs the same loops and barriers whatever its value
+  auto wait_full = [&]() -> bool {
+    const int s = k % ctl.nstages;
+    bool w = ok && mbar_wait(&ctl.full[s], (k / ctl.nstages) & 1, ctl.abort_flag, a.err, a.wait_cycles);
+    if (w) k_ok = k + 1;
+    return __all_sync(kFull, w);
+  };
+  auto release = [&](int s) {   // the warp is done with stage s
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl.empty[s]);
+  };
+  zero_x_tail(a, xsm);
+  consumer_sync();
+  const bool x_ok = mbar_wait(ctl.xbar, 0, ctl.abort_flag, a.err, a.wait_cycles);
+  ok = __all_sync(kFull, x_ok);
+
+  // ---- phase R ----
+  if (router_cta) {
+    const int s = k % ctl.nstages;
+    ok = wait_full();
+    route_rows(a, c, Cr, xsm, ctl.stage + (size_t)s * ctl.stage_bytes, red, limbs, ok);
+    release(s);
+    ++k;
+  } else {
+    for (int ch = 0; ch < nchunks; ++ch) {
+      const int s = k % ctl.nstages;
+      ok = wait_full();
+      const float v = chunk_gemv(x_u32, smem_u32(ctl.stage + (size_t)s * ctl.stage_bytes), pitch, a.D, warp,
+                                 lane, red, ok);
+      release(s);
+      ++k;
+      const int o = threadIdx.x;
+      const int t = o >> 3, i = o & 7;
+      const int g = ra + ch * rc + i;
+      if (ok && o < 128 && i < rc && g < rbr) {
+        if (g < a.d_e) {
+          if (t < a.T) a.u[(size_t)t * a.d_e + g] = v;
+        } else {
+          const int j = g - a.d_e;   // shared hidden unit
+          store_row_hi_lo(a.HS + (size_t)(j / kSq) * kTileElems + (size_t)t * 2 * kSq, t, kSq, j % kSq,
+                          t < a.T ? silu_f(v) : 0.f);
+        }
+      }
+    }
+  }
+  consumer_sync();
+  if (threadIdx.x == 0)   // releases every consumer thread's phase-R writes (they precede the barrier)
+    atom_add_acq_rel(sync + (router_cta ? si.route_done : si.pre_done), 1u);
+
+  // ---- the union (from the producer), one value for every consumer thread ----
+  if (threadIdx.x == 0) {
+    const bool w = mbar_wait(ctl.ubar, 0, ctl.abort_flag, a.err, a.wait_cycles);
+    ctl.bcast[3] = w ? s_U : 0;
+    ctl.bcast[0] = w;
+  }
+  consumer_sync();
+  ok = ok && ctl.bcast[0];
+  const int U = ctl.bcast[3];
+  const int kp = up_kparts(U, a.d_e, a.D, G);
+  const int Kp = a.D / kp;
+  const int NUu = U * nrb_up * kp;
+  const int ntiles = (a.T + 7) / 8;
+
+  // ---- phase U ----
+  {
+    const int u0 = range_lo(c, NUu, G), u1 = range_lo(c + 1, NUu, G);
+    for (int u = u0; u < u1; ++u) {
+      const int p = u % kp, rbu = (u / kp) % nrb_up, e = ulist[u / (kp * nrb_up)];
+      float acc[2][4] = {};
+      for (int c0 = 0; c0 < Kp; c0 += 128) {
+        const int s = k % ctl.nstages;
+        const bool w = wait_full();
+        ok = ok && w;
+        const int nb = min(2, (Kp - c0) / 64);
+        if (ok) {
+          const uint32_t st = smem_u32(ctl.stage + (size_t)s * ctl.stage_bytes);
+          for (int b = 0; b < nb; ++b) {
+            const uint32_t box = st + b * kBoxBytes;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1, a2,
+                      a3);
+              const int kc = (p * Kp + c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+                if (nt < ntiles) {
+                  uint32_t b0, b1;
+                  ldsm_x2(x_u32 + (uint32_t)(8 * nt + (lane & 7)) * pitch + (uint32_t)kc * 16u, b0, b1);
+                  mma16816(acc[nt], a0, a1, a2, a3, b0, b1);
+                }
+              }
+            }
+          }
+        }
+        release(s);
+        ++k;
+      }
+      // acc[nt][i]: row 16 warp + lane/4 + 8 (i >> 1), token 8 nt + 2 (lane & 3) + (i & 1)
+      if (ok) {
+        const int j0 = rbu * kDRows + 16 * warp + (lane >> 2);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 8 * nt + 2 * (lane & 3) + (i & 1);
+            const int j = j0 + 8 * (i >> 1);
+            if (t < a.T && j < a.d_e) a.C[(((size_t)p * a.E + e) * kTok + t) * a.d_e + j] = acc[nt][i];
+          }
+        }
+      }
+      // the CTA that completes expert e's units computes its NormSiLU tile
+      consumer_sync();
+      if (threadIdx.x == 0) {
+        int last = 0;
+        if (ok) {
+          const unsigned old = atom_add_acq_rel(sync + si.g_cnt + e, 1u);
+          last = old + 1 == (unsigned)(nrb_up * kp);
+          // u comes from phase R
+          if (last) last = spin_until(sync + si.pre_done, (unsigned)Gp, a.wait_cycles, ctl.abort_flag, a.err);
+        }
+        ctl.bcast[0] = last;
+      }
+      consumer_sync();
+      if (ctl.bcast[0]) {
+        norm_silu_tile(a, e, emask[e], kp);
+        consumer_sync();
+        if (threadIdx.x == 0) st_release(sync + si.a_ready + e, 1u);
+      }
+      ok = __all_sync(kFull, ok && !*ctl.abort_flag);
+    }
+  }
+
+  // ---- phase D ----
+  // x is no longer needed: its region becomes the ring of activation tiles
+  // that the producer warp's lanes 1..31 fill
+  __syncwarp();
+  if (lane == 0) mbar_arrive(ctl.xfree);
+  {
+    const int J = nsq + U, NUd = nrb * J;
+    const int v0 = range_lo(c, NUd, G), v1 = range_lo(c + 1, NUd, G);
+    const int nslots = tile_slots(a.D);
+    int cur_rb = -1, slot = -1;
+    float acc[2][4] = {};
+    auto flush = [&]() {      // this CTA's partial of row block cur_rb
+      if (ok) {
+        const int r0 = 16 * warp + (lane >> 2);
+        float* dst = a.Part + (size_t)(2 * c + slot) * kTok * kDRows;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 8 * nt + 2 * (lane & 3) + (i & 1);
+            if (t < a.T) dst[(size_t)t * kDRows + r0 + 8 * (i >> 1)] = acc[nt][i];
+          }
+      }
+      consumer_sync();
+      if (warp == 0) {
+        int last = 0;
+        if (ok) {
+          const int n = rb_sources(cur_rb, J, NUd, G, s_src);
+          if (lane == 0) {
+            const unsigned old = atom_add_acq_rel(sync + si.rb_cnt + cur_rb, 1u);   // releases the partial
+            last = old + 1 == (unsigned)n ? n : 0;
+          }
+        }
+        if (lane == 0) ctl.bcast[0] = last;
+      }
+      consumer_sync();
+      const int n = ctl.bcast[0];
+      if (n) combine_rb(a, cur_rb, s_src, n);
+      consumer_sync();   // s_src is rewritten by the next flush
+    };
+    for (int v = v0; v < v1; ++v) {
+      const DUnit d = down_unit(a, ulist, nsq, J, v);
+      const int i = v - v0, ts = i % nslots;
+      if (d.rb != cur_rb) {
+        if (cur_rb >= 0) flush();
+        cur_rb = d.rb;
+        slot = cur_rb - v0 / J;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[nt][q] = 0.f;
+      }
+      ok = __all_sync(kFull, ok && mbar_wait(&ctl.tfull[ts], (i / nslots) & 1, ctl.abort_flag, a.err,
+                                             a.wait_cycles));
+      const uint32_t bt = smem_u32(xsm + (size_t)ts * kTileBytes);
+      uint32_t brow[2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) brow[nt] = bt + (uint32_t)(8 * nt + (lane & 7)) * (uint32_t)(4 * kSq);
+      const int br = lane & 7;   // B row index for the swizzle (8 nt + br has the same low 3 bits)
+      for (int c0 = 0; c0 < d.K; c0 += 128) {
+        const int s = k % ctl.nstages;
+        const bool w = wait_full();
+        ok = ok && w;
+        const int nb = min(2, (d.K - c0) / 64);
+        if (ok) {
+          const uint32_t st = smem_u32(ctl.stage + (size_t)s * ctl.stage_bytes);
+          for (int b = 0; b < nb; ++b) {
+            const uint32_t box = st + b * kBoxBytes;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1, a2,
+                      a3);
+              const int kc = (c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+                if (nt < ntiles) {
+                  uint32_t bh0, bh1, bl0, bl1;
+                  ldsm_x2(brow[nt] + (uint32_t)row_chunk(br, kc) * 16u, bh0, bh1);
+                  ldsm_x2(brow[nt] + (uint32_t)row_chunk(br, kc + kSq / 8) * 16u, bl0, bl1);
+                  mma16816(acc[nt], a0, a1, a2, a3, bh0, bh1);
+                  mma16816(acc[nt], a0, a1, a2, a3, bl0, bl1);
+                }
+              }
+            }
+          }
+        }
+        release(s);
+        ++k;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.tempty[ts]);   // this warp is done with the tile
+    }
+    if (cur_rb >= 0) flush();
+  }
+
+  // ---- exit: a CTA that gave up waits for every copy it issued ----
+  cp_async_wait<0>();
+  consumer_sync();
+  if (threadIdx.x == 0 && *ctl.abort_flag) {
+    if (!x_ok) mbar_drain(ctl.xbar, 0);
+    mbar_drain(ctl.pbar, 0);
+    const int ki = *ctl.k_issued;
+    for (int kk = k_ok; kk < ki; ++kk) mbar_drain(&ctl.full[kk % ctl.nstages], (kk / ctl.nstages) & 1);
+  }
 }
 
 }  // namespace dec

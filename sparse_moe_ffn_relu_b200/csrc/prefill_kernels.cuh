@@ -15,13 +15,14 @@
 //   kProj    [x] x [W_bar_up; W_s_up]^T        -> u (fp32), hs = SiLU(.) (bf16)
 //   kUp      gathered x rows of expert e's pairs x W_up[e]^T, epilogue
 //            NormSiLU: subtract u, RMS over the d_e columns a thread holds,
-//            SiLU, times s_e * r_e            -> a (bf16, one row per pair)
+//            SiLU                             -> a (bf16, one row per pair),
+//                                                s_e * r_e (fp32, per pair)
 //   kDown    a rows of expert e x W_down[e]^T  -> v (fp16, one row per pair)
 //   kShared  hs x W_s_down^T                   -> S (fp32)
 //
 // and two CUDA-core kernels around them: k_router (exact ReLU routing) and
-// k_combine, out = S + the token's routed rows v in ascending expert order
-// (a fixed order: deterministic) + the residual, one CTA per token with
+// k_combine, out = S + the token's routed rows s_e r_e v in ascending expert
+// order (a fixed order: deterministic) + the residual, one CTA per token with
 // coalesced row reads.
 //
 // Tiles are 128 rows x 256 columns x 64-element K blocks (128 B: one 128-byte
@@ -89,6 +90,7 @@ struct Args {
   int T, D, E, d_e, d_s;
   float eps;
   int residual;
+  long long wait_cycles;      // limit of the waits for data (dec::kWaitCycles unless a test lowers it)
   int K;            // contraction length (a multiple of 64)
   int n_tiles_n;    // column tiles per row tile
   int m_tiles;      // row tiles of kProj / kShared
@@ -103,9 +105,11 @@ struct Args {
   const int* pair_of;         // [T][E] pair index of (t, e) or -1
   float* u;                   // [T][d_e]
   bf16* hs;                   // [T][d_s]
-  bf16* a_pairs;              // [pairs][d_e]
-  __half* v_pairs;            // [pairs][D] fp16: 3 more significant bits than bf16
-                              // for the only intermediate that is not an MMA operand
+  bf16* a_pairs;              // [pairs][d_e] NormSiLU outputs, SiLU(h): |a| <= sqrt(d_e)
+  float* coef_pairs;          // [pairs] s_e r_e of each pair, applied in the combine
+  __half* v_pairs;            // [pairs][D] W_down[e] a in fp16 (3 more significant bits than
+                              // bf16); unscaled by s_e r_e, so |v| <= sqrt(d_e) max_j ||W_down[e][j]||_1
+                              // is a property of the weights, not of the input
   float* s_out;               // [T][D] shared-expert output (MoE layer; null: kShared writes out)
   bf16* out;                  // [T][D]
   int* err;
@@ -449,7 +453,8 @@ __device__ __forceinline__ void epilogue(const Args& a, const Tile& t, uint32_t 
     }
     tmem_wait_st();
     const float inv = rsqrtf(ss / (float)a.d_e + a.eps);
-    // pass 2: a = SiLU(c / rms) * s_e * r_e, bf16, 64 columns per box
+    if (ok) a.coef_pairs[pair] = coef;
+    // pass 2: a = SiLU(c / rms), bf16, 64 columns per box (s_e r_e is applied in the combine)
     bf16* dst = a.a_pairs + (size_t)pair * a.d_e;
     for (int c0 = 0; c0 < a.d_e; c0 += 64) {
       uint8_t* box = full_warp ? box_begin(o) : nullptr;
@@ -458,7 +463,7 @@ __device__ __forceinline__ void epilogue(const Args& a, const Tile& t, uint32_t 
         float v[32];
         tmem_ld32(trow + c0 + 32 * h, v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = silu_fast(v[j] * inv) * coef;
+        for (int j = 0; j < 32; ++j) v[j] = silu_fast(v[j] * inv);
         uint4 w[4];
         pack_bf16x32(v, w);
         if (full_warp) {
@@ -566,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = tile_at<MODE>(a, idx);
         const CUtensorMap* mb = (MODE == kProj && t.bmap) ? &tmB2 : &tmB;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, a.err)) break;
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, a.err, a.wait_cycles)) break;
           mbar_expect_tx(&full[stage], bytes);
           if (MODE != kUp) tma_2d(sm + stage * kABytes, &tmA, kb * kBK, t.arow, &full[stage]);
           tma_2d(sm + kStages * kABytes + stage * kBBytes, mb, kb * kBK, t.brow, &full[stage]);
@@ -602,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tok[q] = row < t.rows ? a.perm[t.arow + row] : -1;
       }
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, a.err)) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, a.err, a.wait_cycles)) {
           stop = true;
           break;
         }
@@ -631,11 +636,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool stop = false;
       for (int idx = blockIdx.x; idx < total && !stop; idx += gridDim.x, ++lt) {
         const int b = lt & 1;
-        if (!mbar_wait(&acce[b], ((lt >> 1) & 1) ^ 1, abort_flag, a.err)) break;
+        if (!mbar_wait(&acce[b], ((lt >> 1) & 1) ^ 1, abort_flag, a.err, a.wait_cycles)) break;
         tc_fence_after();
         const uint32_t dt = tmem + b * kBN;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, a.err)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, a.err, a.wait_cycles)) {
             stop = true;
             break;
           }
@@ -669,7 +674,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int lt = 0;
     for (int idx = blockIdx.x; idx < total; idx += gridDim.x, ++lt) {
       const int b = lt & 1;
-      if (!mbar_wait(&accf[b], (lt >> 1) & 1, abort_flag, a.err)) break;
+      // warp-uniform: tcgen05.ld below is warp-collective
+      if (!__all_sync(kFull, mbar_wait(&accf[b], (lt >> 1) & 1, abort_flag, a.err, a.wait_cycles))) break;
       tc_fence_after();
       const Tile t = tile_at<MODE>(a, idx);
       epilogue<MODE>(a, t, tmem + ((uint32_t)(warp * 32) << 16) + b * kBN, warp, o, &tmO, &tmO2);
@@ -896,16 +902,19 @@ __global__ void __launch_bounds__(256) k_router_exact(const RouterArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// out[t] = S[t] + sum over the token's active experts, ascending, of v[pair]
-// (+ x[t]): one CTA per token, 8 columns per thread, 16-byte coalesced loads.
+// out[t] = S[t] + sum over the token's active experts, ascending, of
+// s_e r_e v[pair] (+ x[t]): one CTA per token, 8 columns per thread, 16-byte
+// coalesced loads.
 
 constexpr int kCThreads = 256;
 
 __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__ S, const __half* __restrict__ v,
+                                                       const float* __restrict__ coef,
                                                        const int* __restrict__ pair_of,
                                                        const bf16* __restrict__ x, bf16* __restrict__ out,
                                                        int D, int E, int residual) {
   __shared__ int list[256];
+  __shared__ float list_c[256];
   __shared__ int n_list;
   const int t = blockIdx.x, lane = threadIdx.x & 31;
   if (threadIdx.x < 32) {   // the token's pairs in ascending expert order
@@ -921,6 +930,8 @@ __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__
   }
   __syncthreads();
   const int n = n_list;
+  if (threadIdx.x < n) list_c[threadIdx.x] = coef[list[threadIdx.x]];
+  __syncthreads();
   for (int c = threadIdx.x * 8; c < D; c += kCThreads * 8) {
     const float4* sp = reinterpret_cast<const float4*>(S + (size_t)t * D + c);
     const float4 s0 = sp[0], s1 = sp[1];
@@ -935,11 +946,12 @@ __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__
       for (int j = 0; j < 8; ++j) {
         if (i + j >= n) break;
         const uint32_t ws4[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+        const float cf = list_c[i + j];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws4[h]));
-          acc[2 * h] += f.x;
-          acc[2 * h + 1] += f.y;
+          acc[2 * h] = fmaf(cf, f.x, acc[2 * h]);
+          acc[2 * h + 1] = fmaf(cf, f.y, acc[2 * h + 1]);
         }
       }
     }
@@ -961,15 +973,16 @@ __global__ void __launch_bounds__(kCThreads) k_combine(const float* __restrict__
 // ---------------------------------------------------------------------------
 // Token -> expert tables for large batches: a stable counting sort of the
 // active (token, expert) pairs by expert, tokens ascending within an expert.
-// The tokens are cut into blocks of 256; k_tab_count counts each block's
-// pairs per expert (and every token's pair count), k_tab_scatter gives every
-// block its first position per expert and places its pairs, warps in order
-// and lanes in order inside a warp.  Block 0 also writes counts, offsets and
-// the list of row tiles (<= tile_rows pairs of one expert each).
+// The tokens are cut into units of 32, one warp each.  k_tab_count counts a
+// unit's pairs per expert with one ballot per expert (and every token's pair
+// count); k_tab_scatter gives each unit, per expert, the pairs of the experts
+// before it plus the pairs of the same expert in earlier units, and places
+// the unit's pairs lane by lane.  Unit 0 also writes counts, offsets and the
+// list of row tiles (<= tile_rows pairs of one expert each).
 
-constexpr int kTabThreads = 128;
+constexpr int kTabThreads = 128;                 // 4 units per block
 constexpr int kTabWarps = kTabThreads / 32;
-constexpr int kTabStage = 8192;   // block counts staged in shared memory (32 KB) up to this size
+constexpr int kTabUnit = 32;                     // tokens per unit
 
 // active flags of token t for experts e0..e0+31 as bits (independent loads)
 __device__ __forceinline__ uint32_t row_bits(const uint8_t* row, bool ok, int E, int e0) {
@@ -981,138 +994,115 @@ __device__ __forceinline__ uint32_t row_bits(const uint8_t* row, bool ok, int E,
 }
 
 __global__ void __launch_bounds__(kTabThreads) k_tab_count(const uint8_t* __restrict__ act, int T, int E,
-                                                           int* __restrict__ n_tok, int* __restrict__ blk_counts) {
-  __shared__ int wc[kTabWarps][256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kTabThreads + threadIdx.x;
+                                                           int* __restrict__ n_tok, int* __restrict__ unit_counts) {
+  const int lane = threadIdx.x & 31;
+  const int u = blockIdx.x * kTabWarps + (threadIdx.x >> 5);
+  if (u * kTabUnit >= T) return;   // whole warps
+  const int t = u * kTabUnit + lane;
   const bool ok = t < T;
   const uint8_t* row = act + (size_t)(ok ? t : 0) * E;
   int n = 0;
   for (int e0 = 0; e0 < E; e0 += 32) {
     const uint32_t bits = row_bits(row, ok, E, e0);
     n += __popc(bits);
+    int mine = 0;   // lane j keeps the count of expert e0 + j
     for (int j = 0; j < 32 && e0 + j < E; ++j) {
-      const unsigned m = __ballot_sync(kFull, (bits >> j) & 1u);
-      if (lane == 0) wc[warp][e0 + j] = __popc(m);
+      const int c = __popc(__ballot_sync(kFull, (bits >> j) & 1u));
+      if (lane == j) mine = c;
     }
+    if (e0 + lane < E) unit_counts[(size_t)u * E + e0 + lane] = mine;
   }
   if (ok) n_tok[t] = n;
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kTabThreads) {
-    int c = 0;
-#pragma unroll
-    for (int w = 0; w < kTabWarps; ++w) c += wc[w][e];
-    blk_counts[(size_t)blockIdx.x * E + e] = c;
-  }
-}
-
-// exclusive prefix sum of v[0..n) (n <= 256) by one warp, in place; returns the total
-__device__ __forceinline__ int warp_exclusive_scan(int* v, int n) {
-  const int lane = threadIdx.x & 31;
-  int loc[8], sum = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane * 8 + i;
-    loc[i] = e < n ? v[e] : 0;
-    sum += loc[i];
-  }
-  int incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(kFull, incl, o);
-    if (lane >= o) incl += y;
-  }
-  int run = incl - sum;
-  const int total = __shfl_sync(kFull, incl, 31);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane * 8 + i;
-    if (e < n) v[e] = run;
-    run += loc[i];
-  }
-  return total;
 }
 
 __global__ void __launch_bounds__(kTabThreads) k_tab_scatter(const uint8_t* __restrict__ act, int T, int E,
-                                                             const int* __restrict__ blk_counts, int nb,
+                                                             const int* __restrict__ unit_counts, int nu,
                                                              int* counts, int* offsets, int* perm, int* pair_of,
                                                              int4* tiles, int* n_tiles, int tile_rows) {
-  __shared__ int cnt[256], off[256], base[256], ntl[256];
-  __shared__ int wc[kTabWarps][256];
-  __shared__ int bc[kTabStage];   // the block counts, when they fit
+  __shared__ int base[kTabWarps][256];   // first position of the unit's pairs, per expert
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // every block: counts per expert and the number of pairs in earlier blocks
-  // (the [nb][E] block counts are staged with coalesced loads when they fit)
-  const bool staged = nb * E <= kTabStage;
-  if (staged) {
-    for (int i = threadIdx.x; i < nb * E; i += kTabThreads) bc[i] = blk_counts[i];
-    __syncthreads();
+  const int u = blockIdx.x * kTabWarps + warp;
+  if (u * kTabUnit >= T) return;   // whole warps; no block-wide barrier below
+  // per expert (lane j: experts j, j + 32, ...): the total count and the
+  // pairs in earlier units
+  int tot[8], before[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    tot[i] = 0;
+    before[i] = 0;
   }
-  for (int e = threadIdx.x; e < E; e += kTabThreads) {
-    int c = 0, before = 0;
-    for (int b = 0; b < nb; ++b) {
-      const int v = staged ? bc[b * E + e] : blk_counts[(size_t)b * E + e];
-      c += v;
-      if (b < (int)blockIdx.x) before += v;
-    }
-    cnt[e] = c;
-    off[e] = c;
-    base[e] = before;
-    ntl[e] = (c + tile_rows - 1) / tile_rows;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int P = warp_exclusive_scan(off, E);
-    if (blockIdx.x == 0 && lane == 0) offsets[E] = P;
-  } else if (warp == 1 && blockIdx.x == 0) {
-    const int nt = warp_exclusive_scan(ntl, E);
-    if (lane == 0) *n_tiles = nt;
-  }
-  __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int e = threadIdx.x; e < E; e += kTabThreads) {
-      counts[e] = cnt[e];
-      offsets[e] = off[e];
-    }
-    // row tiles: expert e's tiles start at ntl[e] (now its exclusive prefix)
-    for (int e = warp; e < E; e += kTabWarps) {
-      const int n = (cnt[e] + tile_rows - 1) / tile_rows;
-      for (int j = lane; j < n; j += 32)
-        tiles[ntl[e] + j] = make_int4(e, off[e] + j * tile_rows, min(tile_rows, cnt[e] - j * tile_rows), 0);
+  for (int v = 0; v < nu; ++v) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) {
+        const int c = unit_counts[(size_t)v * E + e];
+        tot[i] += c;
+        if (v < u) before[i] += c;
+      }
     }
   }
-  // this block's tokens: per-warp counts per expert, then positions
-  const int t = blockIdx.x * kTabThreads + threadIdx.x;
+  // exclusive scan of tot over experts (ascending e = i * 32 + lane)
+  int run = 0, ntl_run = 0;
+  int off[8], toff[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = (lane + 32 * i < E) ? tot[i] : 0;
+    const int nt = (c + tile_rows - 1) / tile_rows;
+    int incl = c, incl_t = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o), yt = __shfl_up_sync(kFull, incl_t, o);
+      if (lane >= o) {
+        incl += y;
+        incl_t += yt;
+      }
+    }
+    off[i] = run + incl - c;
+    toff[i] = ntl_run + incl_t - nt;
+    run += __shfl_sync(kFull, incl, 31);
+    ntl_run += __shfl_sync(kFull, incl_t, 31);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) base[warp][e] = off[i] + before[i];
+  }
+  if (u == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e >= E) continue;
+      counts[e] = tot[i];
+      offsets[e] = off[i];
+      const int n = (tot[i] + tile_rows - 1) / tile_rows;
+      for (int j = 0; j < n; ++j)
+        tiles[toff[i] + j] = make_int4(e, off[i] + j * tile_rows, min(tile_rows, tot[i] - j * tile_rows), 0);
+    }
+    if (lane == 0) {
+      offsets[E] = run;
+      *n_tiles = ntl_run;
+    }
+  }
+  __syncwarp();
+  // this unit's tokens: lane = token
+  const int t = u * kTabUnit + lane;
   const bool ok = t < T;
   const uint8_t* row = act + (size_t)(ok ? t : 0) * E;
-  uint32_t rb[8];   // this token's flags, 32 experts per word (E <= 256)
-#pragma unroll
-  for (int c = 0; c < 8; ++c) rb[c] = c * 32 < E ? row_bits(row, ok, E, c * 32) : 0u;
-  for (int e = 0; e < E; ++e) {
-    const unsigned m = __ballot_sync(kFull, (rb[e >> 5] >> (e & 31)) & 1u);
-    if (lane == 0) wc[warp][e] = __popc(m);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kTabThreads) {
-    int run = off[e] + base[e];
-#pragma unroll
-    for (int w = 0; w < kTabWarps; ++w) {
-      const int v = wc[w][e];
-      wc[w][e] = run;
-      run += v;
-    }
-  }
-  __syncthreads();
   const unsigned lt = (1u << lane) - 1u;
-  for (int e = 0; e < E; ++e) {
-    const bool f = (rb[e >> 5] >> (e & 31)) & 1u;
-    const unsigned m = __ballot_sync(kFull, f);
-    if (f) {
-      const int pos = wc[warp][e] + __popc(m & lt);
-      perm[pos] = t;
-      pair_of[(size_t)t * E + e] = pos;
-    } else if (ok) {
-      pair_of[(size_t)t * E + e] = -1;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const uint32_t bits = row_bits(row, ok, E, e0);
+    for (int j = 0; j < 32 && e0 + j < E; ++j) {
+      const int e = e0 + j;
+      const bool f = (bits >> j) & 1u;
+      const unsigned m = __ballot_sync(kFull, f);
+      if (f) {
+        const int pos = base[warp][e] + __popc(m & lt);
+        perm[pos] = t;
+        pair_of[(size_t)t * E + e] = pos;
+      } else if (ok) {
+        pair_of[(size_t)t * E + e] = -1;
+      }
     }
   }
 }

@@ -91,6 +91,8 @@ struct RouteArgs {
   float* u;          // [T][d_e]
   float* hs;         // [T][d_s]
   int* err;
+  float* zt;         // TopK routing: [T][E] fp32 logits (router rows then decide nothing)
+  float* bt;         // TopK routing: [T][E] bound on |fp32 logit - exact logit|
 };
 
 template <typename T, int TT>
@@ -128,6 +130,14 @@ __global__ void __launch_bounds__(kThreads) k_route(RouteArgs a) {
     for (int tt = 0; tt < nt; ++tt) {
       float z = acc[tt] + b;
       const float B = scale * (aacc[tt] + fabsf(b)) + tiny;
+      if (a.zt) {                // TopK: k_topk_select ranks the logits
+        if (lane == 0) {
+          const size_t o = (size_t)(t0 + tt) * a.E + e;
+          a.zt[o] = z;
+          a.bt[o] = B;
+        }
+        continue;
+      }
       bool on;
       if (fabsf(z) > B) {
         on = z > 0.f;
@@ -487,6 +497,137 @@ __global__ void k_mean_up(const T* __restrict__ W_up, T* __restrict__ W_bar, int
       W_bar[i] = __double2bfloat16(m);
     }
   }
+}
+
+
+// ---------------------------------------------------------------------------
+// TopK routing (the conventional baseline DECO is compared with at the same
+// activation ratio, "DECO: Sparse Mixture-of-Experts with Dense-Comparable
+// Performance on End-Side Devices", §5): each token keeps its k largest
+// logits, ties to the lower expert index, with weights ReLU(z).  The ranking
+// is exact: one warp per token ranks the fp32 logits, and the selection
+// stands if the k-th lower bound (logit - B) lies above every unselected
+// upper bound (logit + B); otherwise only the experts whose intervals overlap
+// that boundary are ranked among themselves by exact comparisons
+// (exact_cmp_warp), while the ones above or below it are certain.
+
+struct TopkArgs {
+  const void* x;
+  const void* W_r;
+  const float* b_r;
+  int T, D, E, k;
+  const float* zt;   // [T][E] fp32 logits
+  const float* bt;   // [T][E] their error bounds
+  float* r;          // [T][E]
+  uint8_t* act;      // [T][E]
+  int* err;
+};
+
+constexpr int kTopkWarps = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kTopkWarps * 32) k_topk_select(const TopkArgs a) {
+  __shared__ float sz[kTopkWarps][256];
+  __shared__ int mlist[kTopkWarps][256];
+  __shared__ int mrank[kTopkWarps][256];
+  __shared__ unsigned long long limbs[kTopkWarps][kLimbs];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTopkWarps + warp;
+  if (t >= a.T) return;   // whole warps only: no block-wide barrier below
+  const float inf = __int_as_float(0x7f800000);
+  float z[8], B[8];
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    z[i] = -inf;
+    B[i] = 0.f;
+    if (e < a.E) {
+      z[i] = a.zt[(size_t)t * a.E + e];
+      B[i] = a.bt[(size_t)t * a.E + e];
+      if (!(fabsf(z[i]) < inf) || !(B[i] < inf)) {   // non-finite operand: rank it last
+        bad = true;
+        z[i] = -inf;
+        B[i] = 0.f;
+      }
+      sz[warp][e] = z[i];
+    }
+  }
+  __syncwarp();
+  // rank by the fp32 logit, ties to the lower index
+  bool in[8];
+  float lo = inf, hi = -inf;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    in[i] = false;
+    if (e >= a.E) continue;
+    int rank = 0;
+    for (int f = 0; f < a.E; ++f) {
+      const float v = sz[warp][f];
+      rank += (v > z[i] || (v == z[i] && f < e)) ? 1 : 0;
+    }
+    in[i] = rank < a.k;
+    if (in[i]) lo = fminf(lo, z[i] - B[i]);
+    else hi = fmaxf(hi, z[i] + B[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(kFull, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, o));
+  }
+  bad = __any_sync(kFull, bad);
+  if (!(lo > hi) && !bad) {
+    // the boundary is not certain: experts above hi are in, below lo are
+    // out, the rest (M) are ranked exactly among themselves
+    int n_in = 0, n_m = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      const bool live = e < a.E;
+      const bool sure_in = live && z[i] - B[i] > hi;
+      const bool sure_out = live && z[i] + B[i] < lo;
+      const bool m = live && !sure_in && !sure_out;
+      n_in += __popc(__ballot_sync(kFull, sure_in));
+      const unsigned bm = __ballot_sync(kFull, m);
+      if (m) mlist[warp][n_m + __popc(bm & ((1u << lane) - 1u))] = e;
+      n_m += __popc(bm);
+      in[i] = sure_in;
+    }
+    __syncwarp();
+    for (int i = lane; i < n_m; i += 32) mrank[warp][i] = 0;
+    __syncwarp();
+    const T* x = static_cast<const T*>(a.x) + (size_t)t * a.D;
+    const T* W = static_cast<const T*>(a.W_r);
+    for (int i = 0; i < n_m; ++i)
+      for (int j = i + 1; j < n_m; ++j) {   // mlist ascending: on an exact tie i ranks above j
+        const int ei = mlist[warp][i], ej = mlist[warp][j];
+        const int sg = exact_cmp_warp(x, W + (size_t)ei * a.D, W + (size_t)ej * a.D, a.D, a.b_r[ei], a.b_r[ej],
+                                      limbs[warp], &bad);
+        if (lane == 0) {
+          if (sg >= 0) mrank[warp][j] += 1;
+          else mrank[warp][i] += 1;
+        }
+        __syncwarp();
+      }
+    const int need = a.k - n_in;
+    for (int i = 0; i < n_m; ++i) {
+      const int e = mlist[warp][i];
+      const bool take = mrank[warp][i] < need;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (take && e == lane + 32 * q) in[q] = true;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    if (e >= a.E) continue;
+    const size_t o = (size_t)t * a.E + e;
+    a.act[o] = in[i] ? 1 : 0;
+    a.r[o] = in[i] ? fmaxf(z[i], 0.f) : 0.f;
+  }
+  if (bad && lane == 0) atomicOr(a.err, 1);
 }
 
 }  // namespace deco

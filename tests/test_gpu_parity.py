@@ -297,3 +297,207 @@ def test_routing_exact_wide_exponent_range(lib, T, dtype):
     G = to_gpu(L, lib)
     act = _routing_check(lib, shape, L, G)
     assert act[:, 0].all() and not act[:, 1].any() and not act[:, 2].any()
+
+
+def _plant_near_zero_logits(L, pairs):
+    """Set b_r[e] = -fl32(x_t . W_r[e]) for each (t, e): the exact logit of t
+    at e is then the fp32 rounding residual of its dot product (|z| below half
+    an fp32 ulp of the sum, either sign, or exactly 0 when the sum is an fp32
+    value), the hardest case for a sign decision made from an fp32 sum."""
+    import math
+    x64, W64 = O.to_f64(L["x"]), O.to_f64(L["W_r"])
+    for t, e in pairs:
+        dot = math.fsum((x64[t] * W64[e]).tolist())     # products exact in fp64
+        L["b_r"][e] = -float(np.float32(dot))
+    return L
+
+
+@pytest.mark.parametrize("name", ["edge_decode_t1", "edge_decode_t16", "large_t16",
+                                  "edge_prefill_t4096"])
+def test_routing_exact_on_planted_near_zero_logits(lib, name):
+    """The router each forward path runs (the decode kernels' router for bf16
+    batches of up to 16 tokens, the tiled router above) decides logits whose
+    exact value is a rounding residual or exactly zero like the oracle does."""
+    shape, L = case(name)
+    T, E = shape.T, shape.E
+    rng = np.random.default_rng(7)
+    es = rng.choice(E, min(E, 24), replace=False)
+    pairs = [(int(rng.integers(T)), int(e)) for e in es]
+    L = _plant_near_zero_logits(L, pairs)
+    G = to_gpu(L, lib)
+    if T <= 16:
+        act = _routing_check(lib, shape, L, G)
+    else:
+        toks = np.unique(np.array([t for t, _ in pairs] + [0, T - 1]))
+        act = _routing_check(lib, shape, L, G, tokens=toks)
+    # the forward pass of the same batch uses the same decisions
+    out = lib.forward(G["x"], G, eps=shape.eps)
+    torch.cuda.synchronize()
+    toks = sorted({t for t, _ in pairs} | {0, T - 1})
+    ref = oracle_forward(O.to_f64(L["x"]), to_oracle(L, shape.dtype), shape.eps, toks)
+    check_close(out.double().cpu().numpy()[toks], ref, shape.dtype, f"planted {name}")
+
+
+@pytest.mark.parametrize("T", [1, 5, 16])
+def test_dense_ffn_decode_path(lib, T):
+    # bf16, T <= 16: the weight-streaming kernel with no routed experts
+    from synth import make_dense
+    Dn = make_dense(T, 2048, 17408, "bf16", 6)
+    out = lib.dense_ffn(Dn["x"].cuda(), Dn["W1"].cuda(), Dn["W2"].cuda())
+    torch.cuda.synchronize()
+    ref = O.dense_ffn(O.to_f64(Dn["x"]), O.to_f64(Dn["W1"]), O.to_f64(Dn["W2"]))
+    check_close(out.double().cpu().numpy(), ref, "bf16", f"dense decode T={T}")
+    out2 = lib.dense_ffn(Dn["x"].cuda(), Dn["W1"].cuda(), Dn["W2"].cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+@pytest.mark.parametrize("shape", [LayerShape(16, 512, 16, 256, 256, "bf16"),      # decode kernel
+                                   LayerShape(300, 320, 5, 192, 320, "bf16")])     # tensor-core kernels
+def test_timeout_path_reports_and_recovers(lib, shape):
+    """With the wait limit lowered to a few hundred cycles the kernels give up
+    their waits for data: they set bit 2 of the device error word, wait for
+    the copies and tensor-core operations they already issued, and return.
+    The next call with the default limit is correct."""
+    L = make_layer(shape, 61)
+    G = to_gpu(L, lib)
+    ws = lib.alloc_workspace(lib.layer_shape(G["x"], G))
+    ref = O.layer_forward(O.to_f64(L["x"]), to_oracle(L, "bf16"), shape.eps)
+    lib.set_wait_limit(300)
+    try:
+        for _ in range(3):
+            lib.forward(G["x"], G, workspace=ws, eps=shape.eps)
+            assert lib.device_error(ws) & 2
+    finally:
+        lib.set_wait_limit(0)
+    out = lib.forward(G["x"], G, workspace=ws, eps=shape.eps)
+    assert lib.device_error(ws) == 0
+    check_close(out.double().cpu().numpy(), ref, "bf16", f"after timeouts {shape}")
+
+
+# --------------------------------------------------------------------------
+# TopK routing (the baseline of the paper's §5 comparison)
+
+def _topk_k(E):
+    return max(1, int(round(0.2 * E)))
+
+
+def _topk_check(lib, shape, L, G, k, tokens=None):
+    res = lib.routing(G["x"], G, topk=k)
+    torch.cuda.synchronize()
+    act_gpu = _np(res["active"]).astype(bool)
+    x64 = O.to_f64(L["x"])
+    toks = np.arange(shape.T) if tokens is None else np.asarray(tokens)
+    z, act, r = O.topk_route(x64[toks], O.to_f64(L["W_r"]), O.to_f64(L["b_r"]), k)
+    np.testing.assert_array_equal(act_gpu[toks], act)
+    assert (act_gpu.sum(axis=1) == k).all()
+    counts, offsets, perm, n_tok = O.routing_tables(act_gpu)
+    np.testing.assert_array_equal(_np(res["counts"]), counts)
+    np.testing.assert_array_equal(_np(res["offsets"]), offsets)
+    np.testing.assert_array_equal(_np(res["perm"])[: offsets[-1]], perm)
+    scale = np.abs(z).max()
+    assert np.abs(_np(res["r"])[toks] - r).max() <= 1e-5 * scale
+    return act_gpu
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "edge_decode_t1", "edge_decode_t16", "large_t16",
+                                  "edge_prefill_t4096"])
+def test_topk_routing_bit_exact(lib, name):
+    shape, L = case(name)
+    G = to_gpu(L, lib)
+    k = _topk_k(shape.E)
+    toks = None
+    if shape.T > 64:
+        toks = np.sort(np.random.default_rng(2).choice(shape.T, 64, replace=False))
+    _topk_check(lib, shape, L, G, k, toks)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_topk_routing_exact_ties(lib, dtype):
+    """Rows 1 and 3 of W_r copy row 0 (same bias): exact ties, which go to
+    the lower index.  Row 5 is row 4 with one weight moved by one unit in the
+    last place of the storage format, so the two logits differ by x_t[7]
+    times that unit: inside the fp32 sums' error bounds, where the exact
+    comparison decides."""
+    import math
+    shape = LayerShape(40, 256, 8, 64, 64, dtype)
+    L = make_layer(shape, 71)
+    W = L["W_r"].float()
+    W[1] = W[0]
+    W[3] = W[0]
+    W[5] = W[4]
+    w47 = float(W[4, 7])
+    W[5, 7] = w47 + 2.0 ** (math.floor(math.log2(abs(w47))) - (7 if dtype == "bf16" else 23))
+    b = L["b_r"]
+    b[1] = b[0]
+    b[3] = b[0]
+    b[5] = b[4]
+    # make rows 0, 4 sit at the boundary of a k = 2 selection for many tokens
+    b[0] += 2.0
+    b[4] += 2.0
+    L["W_r"] = W.to(L["W_r"].dtype)
+    G = to_gpu(L, lib)
+    for k in (1, 2, 3, 4):
+        _topk_check(lib, shape, L, G, k)
+
+
+@pytest.mark.parametrize("shape", [LayerShape(16, 2048, 64, 256, 1024, "bf16"),   # decode kernel
+                                   LayerShape(300, 320, 5, 192, 320, "bf16"),     # tensor-core kernels
+                                   LayerShape(37, 256, 8, 128, 192, "f32")])      # general kernels
+def test_topk_forward_parity(lib, shape):
+    L = make_layer(shape, 73)
+    G = to_gpu(L, lib)
+    k = _topk_k(shape.E)
+    out = lib.forward(G["x"], G, eps=shape.eps, topk=k)
+    torch.cuda.synchronize()
+    L64 = to_oracle(L, shape.dtype)
+    x64 = O.to_f64(L["x"])
+    _, act, r = O.topk_route(x64, L64["W_r"], L64["b_r"], k)
+    # the layer with the TopK decisions: the oracle's per-expert terms
+    ref = np.zeros((shape.T, shape.D))
+    for t in range(shape.T):
+        u = L64["W_bar_up"] @ x64[t]
+        y = O.shared_expert(x64[t], L64["W_s_up"], L64["W_s_down"])
+        for e in range(shape.E):
+            if act[t, e]:
+                y = y + (L64["s"][e] * r[t, e]) * O.expert_output(x64[t], L64["W_up"][e], L64["W_down"][e], u,
+                                                                 shape.eps)
+        ref[t] = y
+    check_close(out.double().cpu().numpy(), ref, shape.dtype, f"topk forward {shape}")
+
+
+def test_residual_stack_prefill_t16384(lib):
+    """The 8-layer residual stack of the larger layer (d_model 4096, 128
+    experts) at T = 16384 tokens: the tensor-core path, whose routed outputs
+    are staged in fp16.  Activations grow several-fold per layer without a
+    normalisation between layers, which once pushed the staged values out of
+    the fp16 range; they are now staged before the s_e r_e scaling.  Each
+    layer is checked on the GPU's own input to it (teacher forcing) on
+    sampled tokens: random ones, the last one, and per layer the token with
+    the fewest active experts and the token with the logit closest to zero."""
+    base = case("large_t16384")[0]
+    T = base.T
+    x = make_layer(base, 3, layer=0)["x"].cuda()
+    ws = None
+    rng = np.random.default_rng(5)
+    for l in range(8):
+        W = make_layer(base, 3, layer=l, with_x=False)
+        G = to_gpu(W, lib)
+        if ws is None:
+            ws = lib.alloc_workspace(lib.layer_shape(x, G, residual=True))
+        out = lib.forward(x, G, workspace=ws, eps=base.eps, residual=True)
+        assert lib.device_error(ws) == 0
+        rt = lib.routing(x, G)
+        n_act = rt["n_tok"].cpu().numpy()
+        r = rt["r"]
+        zmin = torch.where(r > 0, r, torch.full_like(r, float("inf"))).min(dim=1).values
+        toks = set(rng.choice(T, 8, replace=False).tolist()) | {T - 1, int(np.argmin(n_act)),
+                                                                  int(torch.argmin(zmin).item())}
+        toks = sorted(toks)
+        x64 = x[toks].double().cpu().numpy()
+        L64 = to_oracle(W, "bf16")
+        ref = x64 + oracle_forward(x64, L64, base.eps, range(len(toks)), parallel=False)
+        check_close(out.double().cpu().numpy()[toks], ref, "bf16", f"stack T=16384 layer {l}")
+        x = out
+        del G, rt
+    assert torch.isfinite(x.float()).all()
