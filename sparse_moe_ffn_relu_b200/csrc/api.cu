@@ -27,7 +27,7 @@ struct Plan {
   // decode path (T <= 16): up-projection partials, shared hidden and NormSiLU
   // tiles, per-CTA down-projection partials (the inter-CTA counters follow
   // the error word)
-  size_t C16, HS, A16, Part;
+  size_t C16, HS, A16, Part, tmask;
   // bf16, T > 16: ambiguous router pairs; prefill path: routed expert output
   // rows (one fp16 row per pair) and the shared expert's fp32 output
   size_t fb, blk, v_pairs, coef, s_out;
@@ -104,6 +104,7 @@ Plan make_plan(const deco_moe_shape_t& s) {
     p.HS = take((size_t)dec::down_nsq(s.d_s) * dec::kTileBytes);       // [nsq] 16 KB tiles
     p.A16 = take(E * dec::kTileBytes);                                 // [E] 16 KB tiles
     p.Part = take((size_t)std::max(p.sms, 1) * 2 * dec::kTok * dec::kDRows * 4);   // [G][2][16][128]
+    p.tmask = take(E * 4);                                             // [E] token masks
   }
   p.total = off;
   return p;
@@ -287,6 +288,7 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
     da.b_r = w.b_r;
     da.r = r;
     da.act = act;
+    da.tmask = reinterpret_cast<unsigned*>(ws + p.tmask);
     da.err = reinterpret_cast<int*>(ws + p.err);
     const uint32_t smem = dec::layer_smem(s.d_model).total;
     if ((err = allow_smem(dec::kd_router, smem)) != cudaSuccess) return err;
@@ -404,6 +406,7 @@ void decode_buffers(dec::Args& a, unsigned char* ws, const Plan& p) {
   a.wait_cycles = g_wait_cycles;
   a.r = reinterpret_cast<float*>(ws + p.r);
   a.act = reinterpret_cast<uint8_t*>(ws + p.act);
+  a.tmask = reinterpret_cast<unsigned*>(ws + p.tmask);
   a.u = reinterpret_cast<float*>(ws + p.u);
   a.HS = reinterpret_cast<bf16*>(ws + p.HS);
   a.A = reinterpret_cast<bf16*>(ws + p.A16);
@@ -474,8 +477,7 @@ cudaError_t run_dense_decode(int T, int D, int d_ff, const void* x, const void* 
   const size_t hs_off = align256(sync_bytes);
   a.HS = reinterpret_cast<bf16*>(ws + hs_off);
   a.Part = reinterpret_cast<float*>(ws + align256(hs_off + (size_t)dec::down_nsq(d_ff) * dec::kTileBytes));
-  cudaError_t err = cudaMemsetAsync(ws, 0, sync_bytes, st);
-  if (err != cudaSuccess) return err;
+  cudaError_t err;
   CUtensorMap tmS;
   if ((err = make_map(&tmS, W2, d_ff, D, dec::kDRows)) != cudaSuccess) return err;
   return launch_layer(tmS, tmS, tmS, a, sms, st);   // no routed experts: the W_up / W_down maps are unused
@@ -725,7 +727,11 @@ deco_status_t deco_moe_forward(const deco_moe_shape_t* shape, const void* x,
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   cudaStream_t cs = as_stream(stream);
   std::lock_guard<std::mutex> lock(g_smem_mutex);
-  cudaError_t err = cudaMemsetAsync(ws + p.err, 0, p.err_bytes, cs);
+  cudaError_t err = cudaSuccess;
+  // the decode kernel clears its counters and (with ReLU routing, when it is
+  // the call's only kernel) the error word itself
+  const bool self_clearing = shape->T <= dec::kMaxT && decode_eligible(*shape, p.sms);
+  if (!self_clearing || shape->topk > 0) err = cudaMemsetAsync(ws + p.err, 0, 16, cs);
   if (err != cudaSuccess) return cuda_status(err, "forward: clearing the error word");
   err = shape->dtype == DECO_F32 ? run_forward<float>(*shape, x, *w, out, ws, p, cs)
                                  : run_forward<bf16>(*shape, x, *w, out, ws, p, cs);

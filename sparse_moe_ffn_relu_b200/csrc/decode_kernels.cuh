@@ -30,15 +30,17 @@
 // The same kernel with no routed experts is the equal-parameter dense FFN at
 // decode batch sizes.
 //
-// Data movement: 8 consumer warps and 1 producer warp per CTA.  The producer
-// streams the CTA's weights in one continuous sequence of 33 KB stages behind
-// mbarriers: phase R rows as bulk copies into 16-byte padded rows, phase U
-// and D tiles as 128-row x 64-column TMA boxes in the 128-byte swizzle
-// (ldmatrix reads both without bank conflicts).  It needs only the union of
-// active experts, so the W_up and W_down streams run ahead of the consumers'
-// dependencies.  x stays resident in shared memory during phases R and U; in
-// phase D the consumers fetch each unit's 16 KB activation tile with cp.async
-// one unit ahead.
+// Data movement: 8 consumer warps, 1 producer warp and 1 loader warp per CTA.
+// The producer streams the CTA's weights in one continuous sequence of 33 KB
+// stages behind mbarriers: phase R rows as bulk copies into 16-byte padded
+// rows, phase U and D tiles as 128-row x 64-column TMA boxes in the 128-byte
+// swizzle (ldmatrix reads both without bank conflicts).  It needs only the
+// union of active experts, so the W_up and W_down streams run ahead of the
+// consumers' dependencies.  x stays resident in shared memory during phases R
+// and U; in phase D the loader warp waits for each unit's 16 KB activation
+// tile to be ready and brings it in with cp.async into a ring of up to four
+// tiles.  (The loader has a warp of its own: spinning lanes in the producer's
+// warp would take issue slots from the lane that streams the weights.)
 //
 // Arithmetic: the projections are thin dense contractions done with mma.sync
 // m16n8k16 (bf16 in, fp32 accumulate), weights as A, tokens as B: one
@@ -53,6 +55,7 @@
 // (again bounded) for every copy it issued.  No trap, no assert.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda.h>
 
 #include "common.cuh"
@@ -62,11 +65,12 @@ namespace dec {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kThreads = kConsumerThreads + 32;
+constexpr int kProducerWarp = kConsumerWarps;       // weight ring (lane 0)
+constexpr int kLoaderWarp = kConsumerWarps + 1;     // phase-D activation tiles
+constexpr int kThreads = kConsumerThreads + 64;
 constexpr int kMaxT = 16;                      // decode batches
 constexpr int kTok = 16;                       // token rows of every activation tile
-constexpr uint32_t kBoxStage = 32768;          // two 128 x 64 TMA boxes
-constexpr uint32_t kStageBytes = 33792;        // a ring stage: boxes, or <= 8 padded rows of <= 4 KB
+constexpr uint32_t kStageBytes = 33792;        // a ring stage: two TMA boxes, or <= 8 padded weight rows
 constexpr int kMaxStages = 8;
 constexpr size_t kSmemLimit = 232448;          // 227 KB opt-in per CTA on sm_100
 constexpr long long kWaitCycles = 2000000000ll;  // ~1 s at 1.9 GHz
@@ -255,7 +259,7 @@ __host__ __device__ __forceinline__ int row_chunk(int r, int k) { return (k & ~7
 // kStaticReserve bytes are left for the kernels' static __shared__ arrays.
 
 constexpr uint32_t kHeaderBytes = 1024;
-constexpr uint32_t kStaticReserve = 2048;
+constexpr uint32_t kStaticReserve = 3072;
 
 struct SmemPlan {
   uint32_t ring_off, op_off, total, stage_bytes;
@@ -329,13 +333,14 @@ struct Args {
   const bf16* W_s_down;
   float* r;          // [T][E]
   uint8_t* act;      // [T][E]
+  unsigned* tmask;   // [E] bit t set iff token t activates expert e (written by the router CTAs)
   float* u;          // [T][d_e]
   bf16* HS;          // [nsq][16 tok][256 hi | 256 lo], chunk-swizzled rows: SiLU(x W_s_up^T)
   bf16* A;           // [E][16 tok][256 hi | 256 lo]: s_e r_e NormSiLU(x W_up[e]^T), 0 for
                      // tokens not using e
   float* C;          // [kp <= 8][E][16 tok][d_e]: partial sums of x W_up[e]^T over K parts
   float* Part;       // [G][2][16 tok][128]: a CTA's down-projection sum per row block
-  unsigned* sync;    // inter-CTA counters, zero at launch (layout: SyncIdx)
+  unsigned* sync;    // inter-CTA counters (layout: SyncIdx); kd_layer clears them itself
   int* err;
   bf16* out;
 };
@@ -396,11 +401,13 @@ __device__ __forceinline__ float warp_reduce_scatter(float (&v)[N], int lane) {
 }
 
 // ---------------------------------------------------------------------------
-// Phase R, padded weight rows (the rows of [W_bar_up ; W_s_up]): a CTA's rows
-// come in chunks of rc rows (one stage), each row one bulk copy into a padded
-// shared-memory row.  For a chunk, warp w multiplies the 16 token rows of x by
-// the chunk's rows over columns [w*D/8, (w+1)*D/8): one m16n8 tile per
-// 16-column step.  The 8 warps' 16 x 8 results are then added in warp order.
+// Phase R, rows of [W_bar_up ; W_s_up]: a CTA's rows come in chunks of rc
+// consecutive rows (one stage), each row one bulk copy into a 16-byte padded
+// shared-memory row, the copies of a chunk issued by rc lanes at once (a bulk
+// copy takes a while to issue).  For a chunk, warp w multiplies the 16 token
+// rows of x (padded the same way) by the chunk's rows over columns
+// [w*D/8, (w+1)*D/8): one m16n8 tile per 16-column step.  The 8 warps' 16 x 8
+// results are then added in warp order.
 
 __device__ __forceinline__ uint32_t x_addr(uint32_t xs, uint32_t pitch, int lane, int chunk) {
   return xs + (uint32_t)((lane & 7) + ((lane >> 3) & 1) * 8) * pitch + (uint32_t)(chunk + (lane >> 4)) * 16u;
@@ -412,11 +419,14 @@ __device__ __forceinline__ uint32_t w_addr(uint32_t ws, uint32_t pitch, int lane
   return ws + (uint32_t)r * pitch + (uint32_t)(chunk + ((lane >> 3) & 1)) * 16u;
 }
 
-// issue the T row copies of x into padded rows (one thread)
-__device__ __forceinline__ void stage_x(const Args& a, unsigned char* xs, uint64_t* bar) {
-  const uint32_t pitch = x_pitch(a.D);
-  mbar_expect_tx(bar, (uint32_t)a.T * a.D * 2);
-  for (int t = 0; t < a.T; ++t) bulk_g2s(xs + (size_t)t * pitch, a.x + (size_t)t * a.D, (uint32_t)a.D * 2, bar);
+// the T row copies of x into padded rows, issued by lanes 0..T-1 of the
+// calling warp in parallel (a bulk copy takes a while to issue); every lane
+// of the warp calls this
+__device__ __forceinline__ void stage_x(const Args& a, unsigned char* xs, uint64_t* bar, int lane) {
+  if (lane == 0) mbar_expect_tx(bar, (uint32_t)a.T * a.D * 2);
+  __syncwarp();
+  if (lane < a.T)
+    bulk_g2s(xs + (size_t)lane * x_pitch(a.D), a.x + (size_t)lane * a.D, (uint32_t)a.D * 2, bar);
 }
 // zero the rows T..15 of the 16-row x operand (consumer threads)
 __device__ __forceinline__ void zero_x_tail(const Args& a, unsigned char* xs) {
@@ -428,8 +438,8 @@ __device__ __forceinline__ void zero_x_tail(const Args& a, unsigned char* xs) {
 
 // y[16 tok][8 rows] for one chunk; thread o < 128 of the consumer warps gets
 // output o = tok * 8 + row
-__device__ __forceinline__ float chunk_gemv(uint32_t xs, uint32_t ws, uint32_t pitch, int D, int warp, int lane,
-                                            float* red, bool math) {
+__device__ __forceinline__ float chunk_gemv(uint32_t xs, uint32_t ws, uint32_t pitch, uint32_t wpitch, int D,
+                                            int warp, int lane, float* red, bool math) {
   const int rc = rows_per_chunk(D);
   float d[4] = {0.f, 0.f, 0.f, 0.f};
   if (math) {
@@ -437,7 +447,7 @@ __device__ __forceinline__ float chunk_gemv(uint32_t xs, uint32_t ws, uint32_t p
     for (int ch = c0; ch < c1; ch += 2) {
       uint32_t a0, a1, a2, a3, b0, b1;
       ldsm_x4(x_addr(xs, pitch, lane, ch), a0, a1, a2, a3);
-      ldsm_x2(w_addr(ws, pitch, lane, ch, rc), b0, b1);
+      ldsm_x2(w_addr(ws, wpitch, lane, ch, rc), b0, b1);
       mma16816(d, a0, a1, a2, a3, b0, b1);
     }
   }
@@ -466,14 +476,16 @@ __device__ __forceinline__ float chunk_gemv(uint32_t xs, uint32_t ws, uint32_t p
 
 __device__ __forceinline__ int router_rows(const Args& a, int c, int Cr) { return (a.E - c + Cr - 1) / Cr; }
 
-// producer side: x and the router rows of CTA c into stage 0 (one thread)
+// producer side: x and the router rows of CTA c into stage 0, issued by the
+// lanes of the calling warp in parallel (every lane calls this)
 __device__ __forceinline__ void issue_router(const Args& a, int c, int Cr, unsigned char* xsm, uint64_t* xbar,
-                                             unsigned char* stage, uint64_t* full, uint64_t pol) {
-  const int nrow = router_rows(a, c, Cr);
+                                             unsigned char* stage, uint64_t* full, uint64_t pol, int lane) {
+  const int nrow = router_rows(a, c, Cr);   // <= 4
   const uint32_t rowbytes = (uint32_t)a.D * 2;
-  stage_x(a, xsm, xbar);
-  mbar_expect_tx(full, nrow * rowbytes);
-  for (int j = 0; j < nrow; ++j)
+  if (lane == 0) mbar_expect_tx(full, nrow * rowbytes);
+  stage_x(a, xsm, xbar, lane);              // (synchronises the warp first)
+  const int j = lane - kTok;
+  if (j >= 0 && j < nrow)
     bulk_g2s(stage + (size_t)j * rowbytes, a.W_r + (size_t)(c + Cr * j) * a.D, rowbytes, full, pol);
 }
 
@@ -545,22 +557,25 @@ __device__ __forceinline__ void route_rows(const Args& a, int c, int Cr, const u
         a.r[(size_t)t * a.E + e] = on ? fmaxf(z, 0.f) : 0.f;
         a.act[(size_t)t * a.E + e] = on ? 1 : 0;
       }
+      const unsigned m = __ballot_sync(kFull, mine && on);
+      if (lane == 0) a.tmask[e] = m;
     }
     consumer_sync();   // red is reused by the next row
   }
   if (bad && (threadIdx.x & 31) == 0) atomicOr(a.err, 1);
 }
 
-// Barriers and bookkeeping kept in the 1 KB header: ring full/empty, x, the
-// union of active experts, the producer's last word (stages issued).
+// Barriers and bookkeeping kept in the 1 KB header: weight ring full/empty,
+// x landed, union built, the producer's last word (stages issued), x
+// released by the consumers, activation-tile ring full/empty.
 constexpr int kTileSlots = 4;                  // phase-D activation tiles in flight (at most)
-constexpr int kLoaderLanes = 31;               // producer-warp lanes 1..31 load them
+constexpr int kLoaderLanes = 32;               // the loader warp's lanes load them
 
 struct Ctl {
   uint64_t* full;
   uint64_t* empty;
   uint64_t* xbar;
-  uint64_t* ubar;
+  uint64_t* ubar;    // the producer warp has built the union of active experts
   uint64_t* pbar;
   uint64_t* xfree;   // consumers are done with x (its region then holds the tile ring)
   uint64_t* tfull;   // [kTileSlots] activation tile landed
@@ -626,11 +641,12 @@ __global__ void __launch_bounds__(kThreads, 1) kd_router(const __grid_constant__
   unsigned char* xsm = smem + sp.op_off;
   float* red = reinterpret_cast<float*>(xsm + kTok * x_pitch(a.D));
   const int warp = threadIdx.x >> 5;
-  if (warp == kConsumerWarps) {
-    if ((threadIdx.x & 31) == 0) issue_router(a, blockIdx.x, Cr, xsm, ctl.xbar, ctl.stage, &ctl.full[0],
-                                              evict_first_policy());
+  if (warp == kProducerWarp) {
+    issue_router(a, blockIdx.x, Cr, xsm, ctl.xbar, ctl.stage, &ctl.full[0], evict_first_policy(),
+                 threadIdx.x & 31);
     return;
   }
+  if (warp == kLoaderWarp) return;
   // both waits always run (bounded), so every issued copy lands before exit
   bool ok = mbar_wait(ctl.xbar, 0, ctl.abort_flag, a.err, a.wait_cycles);
   ok = mbar_wait(&ctl.full[0], 0, ctl.abort_flag, a.err, a.wait_cycles) && ok;
@@ -645,31 +661,68 @@ __global__ void __launch_bounds__(kThreads, 1) kd_router(const __grid_constant__
 // ---------------------------------------------------------------------------
 // The layer.
 
-// Unit of phase D: row block rb of the output, j < nsq a K part of W_s_down,
-// else the (j - nsq)-th active expert.
+// The schedule of phases U and D (every CTA takes a contiguous share of each
+// phase's units, in order).
+struct Sched {
+  int U;              // active experts (the union)
+  int kp, Kp, nrb_up, nrb, nsq;
+  int NU;             // phase-U units
+  int J, ND;          // phase-D units per row block, and in all
+};
+
+__device__ __forceinline__ Sched make_sched(const Args& a, int U, int G) {
+  Sched S;
+  S.U = U;
+  S.nrb_up = (a.d_e + kDRows - 1) / kDRows;
+  S.nrb = a.D / kDRows;
+  S.nsq = down_nsq(a.d_s);
+  S.kp = up_kparts(U, a.d_e, a.D, G);
+  S.Kp = a.D / S.kp;
+  S.NU = U * S.nrb_up * S.kp;
+  S.J = S.nsq + U;
+  S.ND = S.nrb * S.J;
+  return S;
+}
+
+// unit u of phase U: index of its expert in the union, the block of 128 rows
+// of W_up[e] and the K part
+struct UUnit {
+  int ei, rbu, p;
+};
+__device__ __forceinline__ UUnit up_unit(const Sched& S, int u) {
+  UUnit q;
+  q.p = u % S.kp;
+  q.rbu = (u / S.kp) % S.nrb_up;
+  q.ei = u / (S.kp * S.nrb_up);
+  return q;
+}
+
+// Unit v of phase D: row block rb of the output, then j < nsq a K part of
+// W_s_down, the rest the active experts' W_down in ascending order.
 struct DUnit {
   int rb, j, e, K, col0;
 };
-__device__ __forceinline__ DUnit down_unit(const Args& a, const uint8_t* ulist, int nsq, int J, int u) {
+__device__ __forceinline__ DUnit down_unit(const Args& a, const uint8_t* ulist, const Sched& S, int v) {
   DUnit d;
-  d.rb = u / J;
-  d.j = u - d.rb * J;
-  if (d.j < nsq) {
+  d.rb = v / S.J;
+  d.j = v - d.rb * S.J;
+  if (d.j < S.nsq) {
     d.e = -1;
     d.col0 = d.j * kSq;
     d.K = min(kSq, a.d_s - d.col0);
   } else {
-    d.e = ulist[d.j - nsq];
+    d.e = ulist[d.j - S.nsq];
     d.col0 = 0;
     d.K = a.d_e;
   }
   return d;
 }
 
-// CTAs whose unit range meets row block rb, in ascending order (one warp:
-// lane l tests CTAs l, l + 32, ...); returns the count and fills
-// src[i] = 2 c + (slot of rb in c's partials)
-__device__ __forceinline__ int rb_sources(int rb, int J, int NU, int G, int* src) {
+// The partials of row block rb in the fixed order of the combine: the CTAs
+// whose unit range meets rb, ascending (one warp: lane l tests CTAs l,
+// l + 32, ...).  Returns the count and fills src[i] = 2 c + (which of the
+// CTA's two row blocks).
+__device__ __forceinline__ int rb_sources(int rb, const Sched& S, int G, int* src) {
   const int lane = threadIdx.x & 31;
   int n = 0;
   for (int c0 = 0; c0 < G; c0 += 32) {
@@ -677,9 +730,9 @@ __device__ __forceinline__ int rb_sources(int rb, int J, int NU, int G, int* src
     bool hit = false;
     int slot = 0;
     if (c < G) {
-      const int v0 = range_lo(c, NU, G), v1 = range_lo(c + 1, NU, G);
-      hit = v0 < v1 && v0 < (rb + 1) * J && v1 > rb * J;
-      slot = rb - v0 / J;
+      const int v0 = range_lo(c, S.ND, G), v1 = range_lo(c + 1, S.ND, G);
+      hit = v0 < v1 && v0 < (rb + 1) * S.J && v1 > rb * S.J;
+      slot = rb - v0 / S.J;
     }
     const unsigned m = __ballot_sync(kFull, hit);
     if (hit) src[n + __popc(m & ((1u << lane) - 1u))] = 2 * c + slot;
@@ -699,6 +752,7 @@ __device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
     if (!((m_e >> t) & 1u)) reinterpret_cast<uint4*>(tile)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   const int n_e = __popc(m_e);
+  const bool live = 8 * lane < a.d_e;   // lane l holds features 8 l .. 8 l + 7
   for (int slot = warp; slot < n_e; slot += kConsumerWarps) {
     uint32_t m = m_e;
     for (int i = 0; i < slot; ++i) m &= m - 1;
@@ -706,81 +760,111 @@ __device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
     // every load of the token's row is issued before the first is used
     const float rte = __ldcg(a.r + (size_t)t * a.E + e);
     const float se = __ldg(a.s + e);
-    float gp[8][8], uq[8];   // [K part][value], d_e <= 256: 8 values per lane
+    float4 gp[8][2], uq[2];
 #pragma unroll
-    for (int pp = 0; pp < 8; ++pp)
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int j = lane + 32 * q;
-        gp[pp][q] = (pp < kp && j < a.d_e) ? __ldcg(a.C + (((size_t)pp * a.E + e) * kTok + t) * a.d_e + j) : 0.f;
-      }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int j = lane + 32 * q;
-      uq[q] = j < a.d_e ? __ldcg(a.u + (size_t)t * a.d_e + j) : 0.f;
+    for (int pp = 0; pp < 8; ++pp) {
+      const float4* src = reinterpret_cast<const float4*>(a.C + (((size_t)pp * a.E + e) * kTok + t) * a.d_e) + 2 * lane;
+      gp[pp][0] = (pp < kp && live) ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+      gp[pp][1] = (pp < kp && live) ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    const float4* usrc = reinterpret_cast<const float4*>(a.u + (size_t)t * a.d_e) + 2 * lane;
+    uq[0] = live ? __ldcg(usrc) : make_float4(0.f, 0.f, 0.f, 0.f);
+    uq[1] = live ? __ldcg(usrc + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
     float cv[8];
     float ss = 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      float g = 0.f;   // the K parts in order (absent parts add an exact 0)
+    for (int h = 0; h < 2; ++h) {
+      float g[4] = {0.f, 0.f, 0.f, 0.f};   // the K parts in order (absent parts add an exact 0)
 #pragma unroll
-      for (int pp = 0; pp < 8; ++pp) g += gp[pp][q];
-      cv[q] = g - uq[q];
-      ss = fmaf(cv[q], cv[q], ss);
+      for (int pp = 0; pp < 8; ++pp) {
+        g[0] += gp[pp][h].x;
+        g[1] += gp[pp][h].y;
+        g[2] += gp[pp][h].z;
+        g[3] += gp[pp][h].w;
+      }
+      cv[4 * h + 0] = g[0] - uq[h].x;
+      cv[4 * h + 1] = g[1] - uq[h].y;
+      cv[4 * h + 2] = g[2] - uq[h].z;
+      cv[4 * h + 3] = g[3] - uq[h].w;
     }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) ss = fmaf(cv[q], cv[q], ss);
     ss = warp_sum(ss);
     const float rinv = 1.f / sqrtf(ss / float(a.d_e) + a.eps);
     const float coef = se * rte;
-    bf16* row = tile + (size_t)t * 2 * kSq;
+    if (live) {
+      uint32_t hi[4], lo[4];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int j = lane + 32 * q;
-      if (j < a.d_e) store_row_hi_lo(row, t, kSq, j, coef * silu_f(cv[q] * rinv));
+      for (int q = 0; q < 4; ++q) {
+        const float v0 = coef * silu_f(cv[2 * q] * rinv), v1 = coef * silu_f(cv[2 * q + 1] * rinv);
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+        const float2 hf = __bfloat1622float2(h2);
+        const __nv_bfloat162 l2 = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+        hi[q] = *reinterpret_cast<const uint32_t*>(&h2);
+        lo[q] = *reinterpret_cast<const uint32_t*>(&l2);
+      }
+      bf16* row = tile + (size_t)t * 2 * kSq;
+      reinterpret_cast<uint4*>(row)[row_chunk(t, lane)] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      reinterpret_cast<uint4*>(row)[row_chunk(t, kSq / 8 + lane)] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
   }
 }
 
-// out rows of row block rb: the sources' partials in CTA order (+ x)
+// out rows of row block rb: the sources' partials in CTA order (+ x).  A
+// thread owns output float4s o and o + 256 (T * 32 of them); up to 8
+// sources' loads for both are in flight before they are added in order.
+__device__ __forceinline__ void add4(float4& a, const float4& b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+
 __device__ void combine_rb(const Args& a, int rb, const int* src, int n) {
-  const int n4 = a.T * (kDRows / 4);
-  for (int o = threadIdx.x; o < n4; o += kConsumerThreads) {
-    const int t = o / (kDRows / 4), q = o - t * (kDRows / 4);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int i = 0;
-    for (; i + 4 <= n; i += 4) {
-      float4 v[4];
+  constexpr int kQ = kDRows / 4;   // float4s per token row of a block
+  const int n4 = a.T * kQ;
+  for (int o0 = threadIdx.x; o0 < n4; o0 += 2 * kConsumerThreads) {
+    const int o1 = o0 + kConsumerThreads;
+    const bool two = o1 < n4;
+    const int t0 = o0 / kQ, q0 = o0 - t0 * kQ;
+    const int t1 = two ? o1 / kQ : t0, q1 = two ? o1 - t1 * kQ : q0;
+    float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+    for (int i = 0; i < n; i += 8) {
+      float4 v0[8], v1[8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        v[k] = __ldcg(reinterpret_cast<const float4*>(a.Part + ((size_t)src[i + k] * kTok + t) * kDRows) + q);
+      for (int k = 0; k < 8; ++k) {
+        if (i + k < n) {
+          const float* P = a.Part + (size_t)src[i + k] * kTok * kDRows;
+          v0[k] = __ldcg(reinterpret_cast<const float4*>(P + (size_t)t0 * kDRows) + q0);
+          v1[k] = __ldcg(reinterpret_cast<const float4*>(P + (size_t)t1 * kDRows) + q1);
+        }
+      }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        acc.x += v[k].x;
-        acc.y += v[k].y;
-        acc.z += v[k].z;
-        acc.w += v[k].w;
+      for (int k = 0; k < 8; ++k) {
+        if (i + k < n) {
+          add4(acc0, v0[k]);
+          add4(acc1, v1[k]);
+        }
       }
     }
-    for (; i < n; ++i) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(a.Part + ((size_t)src[i] * kTok + t) * kDRows) + q);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (h == 1 && !two) break;
+      float4 acc = h ? acc1 : acc0;
+      const size_t o_idx = (size_t)(h ? t1 : t0) * a.D + (size_t)rb * kDRows + 4 * (h ? q1 : q0);
+      if (a.residual) {
+        const uint2 xr = *reinterpret_cast<const uint2*>(a.x + o_idx);
+        acc.x += __uint_as_float(xr.x << 16);
+        acc.y += __uint_as_float(xr.x & 0xffff0000u);
+        acc.z += __uint_as_float(xr.y << 16);
+        acc.w += __uint_as_float(xr.y & 0xffff0000u);
+      }
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 w;
+      w.x = *reinterpret_cast<const uint32_t*>(&lo);
+      w.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(a.out + o_idx) = w;
     }
-    const size_t o_idx = (size_t)t * a.D + (size_t)rb * kDRows + 4 * q;
-    if (a.residual) {
-      const uint2 xr = *reinterpret_cast<const uint2*>(a.x + o_idx);
-      acc.x += __uint_as_float(xr.x << 16);
-      acc.y += __uint_as_float(xr.x & 0xffff0000u);
-      acc.z += __uint_as_float(xr.y << 16);
-      acc.w += __uint_as_float(xr.y & 0xffff0000u);
-    }
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 w;
-    w.x = *reinterpret_cast<const uint32_t*>(&lo);
-    w.y = *reinterpret_cast<const uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(a.out + o_idx) = w;
   }
 }
 
@@ -789,16 +873,18 @@ __global__ void __launch_bounds__(kThreads, 1)
              const __grid_constant__ CUtensorMap tmS, const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ unsigned long long limbs[kLimbs];
-  __shared__ uint16_t emask[256];
+  __shared__ uint16_t emask[256];   // the producer warp's union: token masks, active experts
   __shared__ uint8_t ulist[256];
   __shared__ int s_U;
+  __shared__ uint16_t cmask[256];   // the consumer warps' own copy
+  __shared__ uint8_t clist[256];
   __shared__ int s_src[kMaxSms];
   const int G = gridDim.x, c = blockIdx.x;
   const int Cr = (a.E > 0 && !a.pre_routed) ? router_ctas(a.E) : 0;
   const bool router_cta = c < Cr;
   const uint32_t pitch = x_pitch(a.D);
   const SmemPlan sp = layer_smem(a.D);
-  if (threadIdx.x == 0) s_U = 0;   // read as 0 or the union's size, even by a consumer that gave up
+  if (threadIdx.x == 0) s_U = 0;
   Ctl ctl;
   unsigned char* smem = ctl_setup(smem_raw, sp, ctl);
   unsigned char* xsm = smem + sp.op_off;
@@ -812,42 +898,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ra = router_cta ? 0 : range_lo(cp, nrows, Gp), rbr = router_cta ? 0 : range_lo(cp + 1, nrows, Gp);
   const int rc = rows_per_chunk(a.D);
   const int nchunks = (rbr - ra + rc - 1) / rc;
-  const int nrb_up = (a.d_e + kDRows - 1) / kDRows;
-  const int nrb = a.D / kDRows;
-  const int nsq = down_nsq(a.d_s);
 
-  if (warp == kConsumerWarps) {
+  // x (and a router CTA's rows, into stage 0 of the first round, which is
+  // free) are issued by the producer warp's lanes in parallel, and are in
+  // flight while the counters are cleared
+  const uint64_t pol = evict_first_policy();
+  if (warp == kProducerWarp) {
+    if (router_cta) issue_router(a, c, Cr, xsm, ctl.xbar, ctl.stage, &ctl.full[0], pol, lane);
+    else stage_x(a, xsm, ctl.xbar, lane);
+  }
+  // Every call starts with its counters at zero: CTA 0 clears them (and the
+  // error word, unless earlier kernels of the call may have set it), and the
+  // grid-wide barrier of the cooperative launch orders that before any use.
+  if (c == 0) {
+    for (int i = threadIdx.x; i < si.total; i += blockDim.x) sync[i] = 0u;
+    if (!a.pre_routed && threadIdx.x == 0) *a.err = 0;
+  }
+  cooperative_groups::this_grid().sync();
+
+  if (warp == kProducerWarp) {
     // ---------------- producer warp ----------------
-    const uint64_t pol = evict_first_policy();
-    int k = 0;
+    int k = router_cta ? 1 : 0;
     bool ok = true;
     auto next_stage = [&](int& s) -> bool {   // lane 0: wait for a free stage
       s = k % ctl.nstages;
       return mbar_wait(&ctl.empty[s], ((k / ctl.nstages) & 1) ^ 1, ctl.abort_flag, a.err, a.wait_cycles);
     };
-    if (lane == 0) {
-      if (router_cta) {
-        int s;
-        if ((ok = next_stage(s))) {   // the first round of stages is free
-          issue_router(a, c, Cr, xsm, ctl.xbar, ctl.stage + (size_t)s * ctl.stage_bytes, &ctl.full[s], pol);
-          ++k;
+    // phase R rows of a non-router CTA: chunks of consecutive rows of
+    // [W_bar_up ; W_s_up], one bulk copy per row, issued by rc lanes at once
+    if (!router_cta) {
+      const uint32_t rowbytes = (uint32_t)a.D * 2;
+      for (int ch = 0; ch < nchunks && ok; ++ch) {
+        int s = 0;
+        if (lane == 0) {
+          ok = next_stage(s);
+          if (ok) mbar_expect_tx(&ctl.full[s], (uint32_t)min(rc, rbr - (ra + ch * rc)) * rowbytes);
         }
-      } else {
-        stage_x(a, xsm, ctl.xbar);
-        for (int ch = 0; ch < nchunks && ok; ++ch) {
-          int s;
-          if (!(ok = next_stage(s))) break;
-          const int g0 = ra + ch * rc, n = min(rc, rbr - g0);
-          mbar_expect_tx(&ctl.full[s], (uint32_t)n * a.D * 2);
-          for (int i = 0; i < n; ++i) {
-            const int g = g0 + i;
-            const bf16* src = g < a.d_e ? a.W_bar + (size_t)g * a.D : a.W_s_up + (size_t)(g - a.d_e) * a.D;
-            bulk_g2s(ctl.stage + (size_t)s * ctl.stage_bytes + (size_t)i * pitch, src, (uint32_t)a.D * 2,
-                     &ctl.full[s], pol);
-          }
-          ++k;
+        ok = __shfl_sync(kFull, ok, 0);
+        s = __shfl_sync(kFull, s, 0);
+        if (!ok) break;
+        const int g = ra + ch * rc + lane;   // lane i copies row i of the chunk into a padded row
+        if (lane < rc && g < rbr) {
+          const bf16* src = g < a.d_e ? a.W_bar + (size_t)g * a.D : a.W_s_up + (size_t)(g - a.d_e) * a.D;
+          bulk_g2s(ctl.stage + (size_t)s * ctl.stage_bytes + (size_t)lane * pitch, src, rowbytes, &ctl.full[s],
+                   pol);
         }
+        ++k;
       }
+    }
+    if (lane == 0) {
       // the union of active experts needs every router row
       if (ok) ok = spin_until(sync + si.route_done, (unsigned)Cr, a.wait_cycles, ctl.abort_flag, a.err);
     }
@@ -856,9 +955,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ld_acquire(sync + si.route_done);   // each lane acquires the router CTAs' writes itself
       for (int e = lane; e < a.E; e += 32) {
         uint32_t m = 0;
+        if (a.pre_routed) {   // decisions from earlier kernels: scan act
 #pragma unroll
-        for (int t = 0; t < kTok; ++t)
-          if (t < a.T && __ldcg(a.act + (size_t)t * a.E + e)) m |= 1u << t;
+          for (int t = 0; t < kTok; ++t)
+            if (t < a.T && __ldcg(a.act + (size_t)t * a.E + e)) m |= 1u << t;
+        } else {              // the router CTAs' per-expert token masks
+          m = __ldcg(a.tmask + e);
+        }
         emask[e] = (uint16_t)m;
       }
       __syncwarp();
@@ -875,73 +978,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_U = 0;
     }
     __syncwarp();
+    if (lane == 0) mbar_arrive(ctl.ubar);   // the loader warp reads the union (or sees the abort)
+    if (lane != 0) return;
     const int U = s_U;
-    if (lane != 0) {
-      // ---- lanes 1..31: the activation tile of each phase-D unit, in order,
-      // into the tile ring (the x region, once the consumers are done with x)
-      const int J = nsq + U, NUd = nrb * J;
-      const int v0 = range_lo(c, NUd, G), v1 = range_lo(c + 1, NUd, G);
-      const int nslots = tile_slots(a.D);
-      bool lok = ok && mbar_wait(ctl.xfree, 0, ctl.abort_flag, a.err, a.wait_cycles);
-      for (int v = v0; v < v1 && lok; ++v) {
-        const int i = v - v0, slot = i % nslots;
-        if (!(lok = mbar_wait(&ctl.tempty[slot], ((i / nslots) & 1) ^ 1, ctl.abort_flag, a.err, a.wait_cycles)))
-          break;
-        const DUnit d = down_unit(a, ulist, nsq, J, v);
-        const unsigned* f = d.e < 0 ? sync + si.pre_done : sync + si.a_ready + d.e;
-        if (!(lok = spin_until(f, d.e < 0 ? (unsigned)Gp : 1u, a.wait_cycles, ctl.abort_flag, a.err))) break;
-        const unsigned char* src = reinterpret_cast<const unsigned char*>(
-            d.e < 0 ? a.HS + (size_t)d.j * kTileElems : a.A + (size_t)d.e * kTileElems);
-        unsigned char* dst = xsm + (size_t)slot * kTileBytes;
-        for (int q = lane - 1; q < (int)(kTileBytes / 16); q += kLoaderLanes)
-          cp_async16_cg(dst + (size_t)q * 16, src + (size_t)q * 16);
-        cp_async_mbar_arrive(&ctl.tfull[slot]);
-      }
-      cp_async_wait_all();   // every copy lands before the lane exits
-      return;
-    }
     {
-      mbar_arrive(ctl.ubar);   // consumers read the union (or see the abort)
+      const Sched S = make_sched(a, U, G);
       // phase U: W_up boxes
-      const int kp = up_kparts(U, a.d_e, a.D, G);
-      const int Kp = a.D / kp;
-      const int NUu = U * nrb_up * kp;
-      const int u0 = range_lo(c, NUu, G), u1 = range_lo(c + 1, NUu, G);
-      for (int u = u0; u < u1 && ok; ++u) {
-        const int p = u % kp, rbu = (u / kp) % nrb_up, e = ulist[u / (kp * nrb_up)];
-        const int row = e * a.d_e + rbu * kDRows;
-        for (int c0 = 0; c0 < Kp; c0 += 128) {
-          int s;
-          if (!(ok = next_stage(s))) break;
-          const int nb = min(2, (Kp - c0) / 64);
-          mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
-          for (int b = 0; b < nb; ++b)
-            tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, &tmU, p * Kp + c0 + 64 * b, row,
-                   &ctl.full[s], pol);
-          ++k;
+      {
+        const int u0 = range_lo(c, S.NU, G), u1 = range_lo(c + 1, S.NU, G);
+        for (int u = u0; u < u1 && ok; ++u) {
+          const UUnit q = up_unit(S, u);
+          const int row = ulist[q.ei] * a.d_e + q.rbu * kDRows;
+          for (int c0 = 0; c0 < S.Kp; c0 += 128) {
+            int s;
+            if (!(ok = next_stage(s))) break;
+            const int nb = min(2, (S.Kp - c0) / 64);
+            mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
+            for (int b = 0; b < nb; ++b)
+              tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, &tmU, q.p * S.Kp + c0 + 64 * b,
+                     row, &ctl.full[s], pol);
+            ++k;
+          }
         }
       }
       // phase D: W_s_down / W_down boxes
-      const int J = nsq + U, NUd = nrb * J;
-      const int v0 = range_lo(c, NUd, G), v1 = range_lo(c + 1, NUd, G);
-      for (int v = v0; v < v1 && ok; ++v) {
-        const DUnit d = down_unit(a, ulist, nsq, J, v);
-        const bool sh = d.e < 0;
-        const int row = sh ? d.rb * kDRows : d.e * a.D + d.rb * kDRows;
-        for (int c0 = 0; c0 < d.K; c0 += 128) {
-          int s;
-          if (!(ok = next_stage(s))) break;
-          const int nb = min(2, (d.K - c0) / 64);
-          mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
-          for (int b = 0; b < nb; ++b)
-            tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, sh ? &tmS : &tmW,
-                   d.col0 + c0 + 64 * b, row, &ctl.full[s], pol);
-          ++k;
+      {
+        const int v0 = range_lo(c, S.ND, G), v1 = range_lo(c + 1, S.ND, G);
+        for (int v = v0; v < v1 && ok; ++v) {
+          const DUnit d = down_unit(a, ulist, S, v);
+          const bool sh = d.e < 0;
+          const int row = sh ? d.rb * kDRows : d.e * a.D + d.rb * kDRows;
+          for (int c0 = 0; c0 < d.K; c0 += 128) {
+            int s;
+            if (!(ok = next_stage(s))) break;
+            const int nb = min(2, (d.K - c0) / 64);
+            mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
+            for (int b = 0; b < nb; ++b)
+              tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, sh ? &tmS : &tmW,
+                     d.col0 + c0 + 64 * b, row, &ctl.full[s], pol);
+            ++k;
+          }
         }
       }
       *ctl.k_issued = k;
       mbar_arrive(ctl.pbar);
     }
+    return;
+  }
+
+  if (warp == kLoaderWarp) {
+    // ---------------- loader warp ----------------
+    // the activation tile of each phase-D unit, in order, into the tile ring
+    // (the x region, once the consumers are done with x)
+    bool lok = mbar_wait(ctl.ubar, 0, ctl.abort_flag, a.err, a.wait_cycles);
+    const Sched S = make_sched(a, lok ? s_U : 0, G);
+    const int nslots = tile_slots(a.D);
+    const int v0 = range_lo(c, S.ND, G), v1 = range_lo(c + 1, S.ND, G);
+    lok = lok && v0 < v1 && mbar_wait(ctl.xfree, 0, ctl.abort_flag, a.err, a.wait_cycles);
+    {
+      for (int v = v0; v < v1 && lok; ++v) {
+        const int i = v - v0;
+        const int slot = i % nslots;
+        if (!(lok = mbar_wait(&ctl.tempty[slot], ((i / nslots) & 1) ^ 1, ctl.abort_flag, a.err, a.wait_cycles)))
+          break;
+        const DUnit d = down_unit(a, ulist, S, v);
+        const unsigned* f = d.e < 0 ? sync + si.pre_done : sync + si.a_ready + d.e;
+        if (!(lok = spin_until(f, d.e < 0 ? (unsigned)Gp : 1u, a.wait_cycles, ctl.abort_flag, a.err))) break;
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(
+            d.e < 0 ? a.HS + (size_t)d.j * kTileElems : a.A + (size_t)d.e * kTileElems);
+        unsigned char* dst = xsm + (size_t)slot * kTileBytes;
+        for (int q = lane; q < (int)(kTileBytes / 16); q += kLoaderLanes)
+          cp_async16_cg(dst + (size_t)q * 16, src + (size_t)q * 16);
+        cp_async_mbar_arrive(&ctl.tfull[slot]);
+      }
+    }
+    cp_async_wait_all();   // every copy lands before the warp exits
     return;
   }
 
@@ -978,8 +1089,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int ch = 0; ch < nchunks; ++ch) {
       const int s = k % ctl.nstages;
       ok = wait_full();
-      const float v = chunk_gemv(x_u32, smem_u32(ctl.stage + (size_t)s * ctl.stage_bytes), pitch, a.D, warp,
-                                 lane, red, ok);
+      const float v = chunk_gemv(x_u32, smem_u32(ctl.stage + (size_t)s * ctl.stage_bytes), pitch, pitch, a.D,
+                                 warp, lane, red, ok);
       release(s);
       ++k;
       const int o = threadIdx.x;
@@ -1000,25 +1111,53 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0)   // releases every consumer thread's phase-R writes (they precede the barrier)
     atom_add_acq_rel(sync + (router_cta ? si.route_done : si.pre_done), 1u);
 
-  // ---- the union (from the producer), one value for every consumer thread ----
-  if (threadIdx.x == 0) {
-    const bool w = mbar_wait(ctl.ubar, 0, ctl.abort_flag, a.err, a.wait_cycles);
-    ctl.bcast[3] = w ? s_U : 0;
-    ctl.bcast[0] = w;
-  }
+  // ---- the union of active experts (the producer builds its own copy) ----
+  if (threadIdx.x == 0)
+    ctl.bcast[0] = ok && spin_until(sync + si.route_done, (unsigned)Cr, a.wait_cycles, ctl.abort_flag, a.err);
   consumer_sync();
   ok = ok && ctl.bcast[0];
+  if (ok) {
+    for (int e = threadIdx.x; e < a.E; e += kConsumerThreads) {
+      uint32_t m = 0;
+      if (a.pre_routed) {   // decisions from earlier kernels: scan act
+#pragma unroll
+        for (int t = 0; t < kTok; ++t)
+          if (t < a.T && __ldcg(a.act + (size_t)t * a.E + e)) m |= 1u << t;
+      } else {              // the router CTAs' per-expert token masks
+        m = __ldcg(a.tmask + e);
+      }
+      cmask[e] = (uint16_t)m;
+    }
+  }
+  consumer_sync();
+  if (warp == 0) {
+    int n = 0;
+    if (ok) {
+      for (int base = 0; base < a.E; base += 32) {
+        const int e = base + lane;
+        const bool f = e < a.E && cmask[e] != 0;
+        const unsigned bal = __ballot_sync(kFull, f);
+        if (f) clist[n + __popc(bal & ((1u << lane) - 1u))] = (uint8_t)e;
+        n += __popc(bal);
+      }
+    }
+    if (lane == 0) ctl.bcast[3] = n;
+  }
+  consumer_sync();
   const int U = ctl.bcast[3];
-  const int kp = up_kparts(U, a.d_e, a.D, G);
-  const int Kp = a.D / kp;
-  const int NUu = U * nrb_up * kp;
+  const Sched S = make_sched(a, U, G);
   const int ntiles = (a.T + 7) / 8;
 
   // ---- phase U ----
+  const int kp = S.kp, Kp = S.Kp, nrb_up = S.nrb_up;
+  bool pre_seen = false;   // thread 0: phase R is complete everywhere (u is readable)
   {
-    const int u0 = range_lo(c, NUu, G), u1 = range_lo(c + 1, NUu, G);
+    const int u0 = range_lo(c, S.NU, G), u1 = range_lo(c + 1, S.NU, G);
+    int n_here = 0;          // this CTA's units of the current expert
     for (int u = u0; u < u1; ++u) {
-      const int p = u % kp, rbu = (u / kp) % nrb_up, e = ulist[u / (kp * nrb_up)];
+      const UUnit q = up_unit(S, u);
+      const int p = q.p, rbu = q.rbu, e = clist[q.ei];
+      ++n_here;
       float acc[2][4] = {};
       for (int c0 = 0; c0 < Kp; c0 += 128) {
         const int s = k % ctl.nstages;
@@ -1062,36 +1201,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // the CTA that completes expert e's units computes its NormSiLU tile
-      consumer_sync();
-      if (threadIdx.x == 0) {
-        int last = 0;
-        if (ok) {
-          const unsigned old = atom_add_acq_rel(sync + si.g_cnt + e, 1u);
-          last = old + 1 == (unsigned)(nrb_up * kp);
-          // u comes from phase R
-          if (last) last = spin_until(sync + si.pre_done, (unsigned)Gp, a.wait_cycles, ctl.abort_flag, a.err);
+      // after the CTA's last unit of expert e: one count of its units; the
+      // CTA that completes e's units computes its NormSiLU tile
+      const bool e_ends = u + 1 == u1 || up_unit(S, u + 1).ei != q.ei;
+      if (e_ends) {
+        consumer_sync();   // every warp's g partials precede the release
+        if (threadIdx.x == 0) {
+          int last = 0;
+          if (ok) {
+            const unsigned old = atom_add_acq_rel(sync + si.g_cnt + e, (unsigned)n_here);
+            last = old + (unsigned)n_here == (unsigned)(nrb_up * kp);
+            // u comes from phase R
+            if (last && !pre_seen)
+              last = pre_seen = spin_until(sync + si.pre_done, (unsigned)Gp, a.wait_cycles, ctl.abort_flag, a.err);
+          }
+          if (!pre_seen && ok) pre_seen = ld_acquire(sync + si.pre_done) >= (unsigned)Gp;
+          ctl.bcast[0] = last;
         }
-        ctl.bcast[0] = last;
-      }
-      consumer_sync();
-      if (ctl.bcast[0]) {
-        norm_silu_tile(a, e, emask[e], kp);
         consumer_sync();
-        if (threadIdx.x == 0) st_release(sync + si.a_ready + e, 1u);
+        if (ctl.bcast[0]) {
+          norm_silu_tile(a, e, cmask[e], kp);
+          consumer_sync();
+          if (threadIdx.x == 0) st_release(sync + si.a_ready + e, 1u);
+        }
+        n_here = 0;
+        ok = __all_sync(kFull, ok && !*ctl.abort_flag);
       }
-      ok = __all_sync(kFull, ok && !*ctl.abort_flag);
     }
   }
 
   // ---- phase D ----
   // x is no longer needed: its region becomes the ring of activation tiles
-  // that the producer warp's lanes 1..31 fill
+  // that the loader warp fills
   __syncwarp();
   if (lane == 0) mbar_arrive(ctl.xfree);
   {
-    const int J = nsq + U, NUd = nrb * J;
-    const int v0 = range_lo(c, NUd, G), v1 = range_lo(c + 1, NUd, G);
     const int nslots = tile_slots(a.D);
     int cur_rb = -1, slot = -1;
     float acc[2][4] = {};
@@ -1102,16 +1246,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int t = 8 * nt + 2 * (lane & 3) + (i & 1);
-            if (t < a.T) dst[(size_t)t * kDRows + r0 + 8 * (i >> 1)] = acc[nt][i];
+          for (int qq = 0; qq < 4; ++qq) {
+            const int t = 8 * nt + 2 * (lane & 3) + (qq & 1);
+            if (t < a.T) dst[(size_t)t * kDRows + r0 + 8 * (qq >> 1)] = acc[nt][qq];
           }
       }
       consumer_sync();
       if (warp == 0) {
         int last = 0;
         if (ok) {
-          const int n = rb_sources(cur_rb, J, NUd, G, s_src);
+          const int n = rb_sources(cur_rb, S, G, s_src);
           if (lane == 0) {
             const unsigned old = atom_add_acq_rel(sync + si.rb_cnt + cur_rb, 1u);   // releases the partial
             last = old + 1 == (unsigned)n ? n : 0;
@@ -1124,60 +1268,63 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n) combine_rb(a, cur_rb, s_src, n);
       consumer_sync();   // s_src is rewritten by the next flush
     };
-    for (int v = v0; v < v1; ++v) {
-      const DUnit d = down_unit(a, ulist, nsq, J, v);
-      const int i = v - v0, ts = i % nslots;
-      if (d.rb != cur_rb) {
-        if (cur_rb >= 0) flush();
-        cur_rb = d.rb;
-        slot = cur_rb - v0 / J;
+    {
+      const int v0 = range_lo(c, S.ND, G), v1 = range_lo(c + 1, S.ND, G);
+      for (int v = v0; v < v1; ++v) {
+        const DUnit d = down_unit(a, clist, S, v);
+        const int i = v - v0, ts = i % nslots;
+        if (d.rb != cur_rb) {
+          if (cur_rb >= 0) flush();
+          cur_rb = d.rb;
+          slot = cur_rb - v0 / S.J;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+          for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) acc[nt][q] = 0.f;
-      }
-      ok = __all_sync(kFull, ok && mbar_wait(&ctl.tfull[ts], (i / nslots) & 1, ctl.abort_flag, a.err,
-                                             a.wait_cycles));
-      const uint32_t bt = smem_u32(xsm + (size_t)ts * kTileBytes);
-      uint32_t brow[2];
+            for (int qq = 0; qq < 4; ++qq) acc[nt][qq] = 0.f;
+        }
+        ok = __all_sync(kFull, ok && mbar_wait(&ctl.tfull[ts], (i / nslots) & 1, ctl.abort_flag, a.err,
+                                               a.wait_cycles));
+        const uint32_t bt = smem_u32(xsm + (size_t)ts * kTileBytes);
+        uint32_t brow[2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) brow[nt] = bt + (uint32_t)(8 * nt + (lane & 7)) * (uint32_t)(4 * kSq);
-      const int br = lane & 7;   // B row index for the swizzle (8 nt + br has the same low 3 bits)
-      for (int c0 = 0; c0 < d.K; c0 += 128) {
-        const int s = k % ctl.nstages;
-        const bool w = wait_full();
-        ok = ok && w;
-        const int nb = min(2, (d.K - c0) / 64);
-        if (ok) {
-          const uint32_t st = smem_u32(ctl.stage + (size_t)s * ctl.stage_bytes);
-          for (int b = 0; b < nb; ++b) {
-            const uint32_t box = st + b * kBoxBytes;
+        for (int nt = 0; nt < 2; ++nt) brow[nt] = bt + (uint32_t)(8 * nt + (lane & 7)) * (uint32_t)(4 * kSq);
+        const int br = lane & 7;   // B row index for the swizzle (8 nt + br has the same low 3 bits)
+        for (int c0 = 0; c0 < d.K; c0 += 128) {
+          const int s = k % ctl.nstages;
+          const bool w = wait_full();
+          ok = ok && w;
+          const int nb = min(2, (d.K - c0) / 64);
+          if (ok) {
+            const uint32_t st = smem_u32(ctl.stage + (size_t)s * ctl.stage_bytes);
+            for (int b = 0; b < nb; ++b) {
+              const uint32_t box = st + b * kBoxBytes;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1, a2,
-                      a3);
-              const int kc = (c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
+              for (int ks = 0; ks < 4; ++ks) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1,
+                        a2, a3);
+                const int kc = (c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
 #pragma unroll
-              for (int nt = 0; nt < 2; ++nt) {
-                if (nt < ntiles) {
-                  uint32_t bh0, bh1, bl0, bl1;
-                  ldsm_x2(brow[nt] + (uint32_t)row_chunk(br, kc) * 16u, bh0, bh1);
-                  ldsm_x2(brow[nt] + (uint32_t)row_chunk(br, kc + kSq / 8) * 16u, bl0, bl1);
-                  mma16816(acc[nt], a0, a1, a2, a3, bh0, bh1);
-                  mma16816(acc[nt], a0, a1, a2, a3, bl0, bl1);
+                for (int nt = 0; nt < 2; ++nt) {
+                  if (nt < ntiles) {
+                    uint32_t bh0, bh1, bl0, bl1;
+                    ldsm_x2(brow[nt] + (uint32_t)row_chunk(br, kc) * 16u, bh0, bh1);
+                    ldsm_x2(brow[nt] + (uint32_t)row_chunk(br, kc + kSq / 8) * 16u, bl0, bl1);
+                    mma16816(acc[nt], a0, a1, a2, a3, bh0, bh1);
+                    mma16816(acc[nt], a0, a1, a2, a3, bl0, bl1);
+                  }
                 }
               }
             }
           }
+          release(s);
+          ++k;
         }
-        release(s);
-        ++k;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.tempty[ts]);   // this warp is done with the tile
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.tempty[ts]);   // this warp is done with the tile
+      if (cur_rb >= 0) flush();
     }
-    if (cur_rb >= 0) flush();
   }
 
   // ---- exit: a CTA that gave up waits for every copy it issued ----
