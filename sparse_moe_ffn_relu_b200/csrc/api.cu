@@ -30,7 +30,7 @@ struct Plan {
   size_t C16, HS, A16, Part, tmask;
   // bf16, T > 16: ambiguous router pairs; prefill path: routed expert output
   // rows (one fp16 row per pair) and the shared expert's fp32 output
-  size_t fb, blk, v_pairs, coef, s_out;
+  size_t fb, blk, etot, v_pairs, coef, s_out;
   // TopK routing: fp32 logits and their error bounds
   size_t zt, bt;
   int tile_rows;
@@ -88,7 +88,8 @@ Plan make_plan(const deco_moe_shape_t& s) {
   p.H = take(P * s.d_e * 4);       // NormSiLU activations (fp32; bf16 on the prefill path)
   if (tiled_router(s)) {
     p.fb = take(P * 8);
-    p.blk = take((size_t)((s.T + pf::kTabThreads - 1) / pf::kTabThreads) * E * 4);
+    p.blk = take((size_t)((s.T + pf::kTabUnit - 1) / pf::kTabUnit) * E * 4);   // [units of 32 tokens][E]
+    p.etot = take(E * 4);
   }
   if (s.topk > 0) {
     p.zt = take(P * 4);
@@ -324,9 +325,12 @@ cudaError_t run_routing(const deco_moe_shape_t& s, const void* x, const deco_moe
     prof_mark(2, st);
     pf::k_tab_count<<<nb, pf::kTabThreads, 0, st>>>(act, s.T, s.E, n_tok, blk);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    int* etot = reinterpret_cast<int*>(ws + p.etot);
+    pf::k_tab_scan<<<(s.E + pf::kTabWarps - 1) / pf::kTabWarps, pf::kTabThreads, 0, st>>>(s.E, nu, blk, etot);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     prof_mark(3, st);
     prof_mark(4, st);
-    pf::k_tab_scatter<<<nb, pf::kTabThreads, 0, st>>>(act, s.T, s.E, blk, nu, counts, offsets, perm,
+    pf::k_tab_scatter<<<nb, pf::kTabThreads, 0, st>>>(act, s.T, s.E, blk, etot, counts, offsets, perm,
                                                       reinterpret_cast<int*>(ws + p.pair_of),
                                                       reinterpret_cast<int4*>(ws + p.tiles),
                                                       reinterpret_cast<int*>(ws + p.n_tiles), tile_rows);

@@ -714,8 +714,11 @@ constexpr int kRE = 64;          // experts per CTA
 constexpr int kRK = 16;          // K chunk
 constexpr int kRWarps = 8;
 constexpr int kRThreads = kRWarps * 32;
-constexpr size_t kRouterSmem =   // staging (aliased by the warp totals) + norms
-    (size_t)kRWarps * kRT * kRE * 4 + (size_t)kRWarps * (kRT + kRE) * 4;
+constexpr int kRTL = kRT / 4;    // tokens per lane (4 token groups x 8 expert groups of lanes)
+static_assert(kRTL == 8, "the lane tile below reads 8 tokens as two float4");
+constexpr size_t kRStage = (size_t)kRWarps * kRK * (kRT + kRE) * 4;   // per-warp staging slices
+constexpr size_t kRTotals = (size_t)kRWarps * kRT * kRE * 4;          // warp totals (alias the staging)
+constexpr size_t kRouterSmem = (kRStage > kRTotals ? kRStage : kRTotals) + (size_t)kRWarps * (kRT + kRE) * 4;
 
 struct RouterArgs {
   const bf16* x;
@@ -751,20 +754,21 @@ __global__ void __launch_bounds__(kRThreads, 1) k_router(const RouterArgs a) {
   // this warp's staging slice: xs[kRK][kRT], ws[kRK][kRE]
   float* xs = rsm + (size_t)warp * kRK * (kRT + kRE);
   float* ws = xs + kRK * kRT;
-  float* nx_w = rsm + (size_t)kRWarps * kRT * kRE + warp * (kRT + kRE);   // [kRT] then [kRE]
+  constexpr size_t kNormOff = (kRStage > kRTotals ? kRStage : kRTotals) / 4;   // floats
+  float* nx_w = rsm + kNormOff + warp * (kRT + kRE);   // [kRT] then [kRE]
   float* nw_w = nx_w + kRT;
   // loading: lane = token row lane and expert rows lane, lane + 32; 16 k each
-  const bool xok = t0 + lane < a.T;
+  const bool xok = lane < kRT && t0 + lane < a.T;
   const bool wok0 = e0 + lane < a.E, wok1 = e0 + lane + 32 < a.E;
   const bf16* xrow = a.x + (size_t)(xok ? t0 + lane : 0) * a.D;
   const bf16* wrow0 = a.W_r + (size_t)(wok0 ? e0 + lane : 0) * a.D;
   const bf16* wrow1 = a.W_r + (size_t)(wok1 ? e0 + lane + 32 : 0) * a.D;
   float sx = 0.f, sw0 = 0.f, sw1 = 0.f;
-  // computing: tokens ty*8 + i, experts tx*4 + {0..3} and 32 + tx*4 + {0..3}
+  // computing: tokens ty*kRTL + i, experts tx*4 + {0..3} and 32 + tx*4 + {0..3}
   const int ty = lane >> 3, tx = lane & 7;
-  unsigned long long tot[8][4];
+  unsigned long long tot[kRTL][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < kRTL; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) tot[i][j] = 0ull;
   const int nchunks = a.D / kRK;
@@ -792,7 +796,7 @@ __global__ void __launch_bounds__(kRThreads, 1) k_router(const RouterArgs a) {
     __syncwarp();   // the previous chunk's reads are done
 #pragma unroll
     for (int k = 0; k < kRK; ++k) {
-      xs[k * kRT + lane] = fx[k];
+      if (lane < kRT) xs[k * kRT + lane] = fx[k];
       ws[k * kRE + lane] = fw0[k];
       ws[k * kRE + lane + 32] = fw1[k];
       sx = fmaf(fx[k], fx[k], sx);
@@ -801,20 +805,20 @@ __global__ void __launch_bounds__(kRThreads, 1) k_router(const RouterArgs a) {
     }
     __syncwarp();
     fetch(c + kRWarps);
-    unsigned long long part[8][4];
+    unsigned long long part[kRTL][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < kRTL; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) part[i][j] = 0ull;
 #pragma unroll 4
     for (int k = 0; k < kRK; ++k) {
-      const float4 xa = *reinterpret_cast<const float4*>(xs + k * kRT + ty * 8);
-      const float4 xb = *reinterpret_cast<const float4*>(xs + k * kRT + ty * 8 + 4);
+      const float4 xa = *reinterpret_cast<const float4*>(xs + k * kRT + ty * kRTL);
+      const float4 xb = *reinterpret_cast<const float4*>(xs + k * kRT + ty * kRTL + 4);
       const ulonglong2 wa = *reinterpret_cast<const ulonglong2*>(ws + k * kRE + tx * 4);
       const ulonglong2 wb = *reinterpret_cast<const ulonglong2*>(ws + k * kRE + 32 + tx * 4);
-      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+      const float xv[kRTL] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < kRTL; ++i) {
         const unsigned long long xx = f2pack(xv[i], xv[i]);
         ffma2(part[i][0], xx, wa.x);
         ffma2(part[i][1], xx, wa.y);
@@ -823,27 +827,27 @@ __global__ void __launch_bounds__(kRThreads, 1) k_router(const RouterArgs a) {
       }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < kRTL; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 p = f2unpack(part[i][j]), t = f2unpack(tot[i][j]);
         tot[i][j] = f2pack(t.x + p.x, t.y + p.y);
       }
   }
-  nx_w[lane] = sx;
+  if (lane < kRT) nx_w[lane] = sx;
   nw_w[lane] = sw0;
   nw_w[lane + 32] = sw1;
   __syncthreads();   // every warp is past its staging slice
   // warp totals: red[warp][t][e]
   float* red = rsm + (size_t)warp * kRT * kRE;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < kRTL; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float2 t = f2unpack(tot[i][j]);
       const int e = (j < 2 ? tx * 4 : 32 + tx * 4) + 2 * (j & 1);
-      red[(ty * 8 + i) * kRE + e] = t.x;
-      red[(ty * 8 + i) * kRE + e + 1] = t.y;
+      red[(ty * kRTL + i) * kRE + e] = t.x;
+      red[(ty * kRTL + i) * kRE + e + 1] = t.y;
     }
   __syncthreads();
   const int n = kRK + a.D / (kRWarps * kRK) + kRWarps + 3;
@@ -852,7 +856,7 @@ __global__ void __launch_bounds__(kRThreads, 1) k_router(const RouterArgs a) {
   const float tiny = float(n) * 2.8025969e-45f;                   // n * 2^-148
   const float gD = gamma_f32(a.D);
   const float sub = float(a.D) * 1.4012985e-45f;                  // D * 2^-149
-  const float* nrm = rsm + (size_t)kRWarps * kRT * kRE;
+  const float* nrm = rsm + kNormOff;
   for (int p = threadIdx.x; p < kRT * kRE; p += kRThreads) {
     const int tr = p / kRE, er = p - tr * kRE;
     const int t = t0 + tr, e = e0 + er;
@@ -984,64 +988,91 @@ constexpr int kTabThreads = 128;                 // 4 units per block
 constexpr int kTabWarps = kTabThreads / 32;
 constexpr int kTabUnit = 32;                     // tokens per unit
 
-// active flags of token t for experts e0..e0+31 as bits (independent loads)
-__device__ __forceinline__ uint32_t row_bits(const uint8_t* row, bool ok, int E, int e0) {
-  uint32_t bits = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (ok && e0 + j < E && row[e0 + j]) bits |= 1u << j;
-  return bits;
+// The active flags of a unit's 32 tokens, [32][E] bytes, into shared memory
+// with 16-byte loads where the rows allow it (tokens past T read as 0).
+__device__ __forceinline__ void load_unit_flags(const uint8_t* __restrict__ act, int T, int E, int u, uint8_t* fl) {
+  const int lane = threadIdx.x & 31;
+  const int t0 = u * kTabUnit;
+  const int nt = min(kTabUnit, T - t0);
+  const uint8_t* src = act + (size_t)t0 * E;
+  const int nbytes = nt * E;
+  if ((E & 15) == 0 && (reinterpret_cast<uintptr_t>(act) & 15) == 0) {   // 16-byte aligned: vector loads
+    for (int i = lane; i < nbytes / 16; i += 32)
+      reinterpret_cast<uint4*>(fl)[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
+  } else {
+    for (int i = lane; i < nbytes; i += 32) fl[i] = src[i];
+  }
+  for (int i = nbytes + lane; i < kTabUnit * E; i += 32) fl[i] = 0;
+  __syncwarp();
 }
 
 __global__ void __launch_bounds__(kTabThreads) k_tab_count(const uint8_t* __restrict__ act, int T, int E,
                                                            int* __restrict__ n_tok, int* __restrict__ unit_counts) {
-  const int lane = threadIdx.x & 31;
-  const int u = blockIdx.x * kTabWarps + (threadIdx.x >> 5);
+  __shared__ __align__(16) uint8_t flags[kTabWarps][kTabUnit * 256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * kTabWarps + warp;
   if (u * kTabUnit >= T) return;   // whole warps
-  const int t = u * kTabUnit + lane;
-  const bool ok = t < T;
-  const uint8_t* row = act + (size_t)(ok ? t : 0) * E;
-  int n = 0;
-  for (int e0 = 0; e0 < E; e0 += 32) {
-    const uint32_t bits = row_bits(row, ok, E, e0);
-    n += __popc(bits);
-    int mine = 0;   // lane j keeps the count of expert e0 + j
-    for (int j = 0; j < 32 && e0 + j < E; ++j) {
-      const int c = __popc(__ballot_sync(kFull, (bits >> j) & 1u));
-      if (lane == j) mine = c;
-    }
-    if (e0 + lane < E) unit_counts[(size_t)u * E + e0 + lane] = mine;
+  uint8_t* fl = flags[warp];
+  load_unit_flags(act, T, E, u, fl);
+  // the unit's pairs per expert: lane j sums experts j, j + 32, ... over the 32 tokens
+  for (int e = lane; e < E; e += 32) {
+    int c = 0;
+#pragma unroll 8
+    for (int t = 0; t < kTabUnit; ++t) c += fl[t * E + e];
+    unit_counts[(size_t)u * E + e] = c;
   }
-  if (ok) n_tok[t] = n;
+  // each token's pair count: lane = token
+  const int t = u * kTabUnit + lane;
+  if (t < T) {
+    int n = 0;
+    for (int e = 0; e < E; ++e) n += fl[lane * E + ((e + lane) % E)];   // rotated start: no bank conflicts
+    n_tok[t] = n;
+  }
+}
+
+// Per expert e, the pairs of e in the units before each unit (exclusive scan
+// over units, in place in unit_counts) and e's total: one warp per expert.
+__global__ void __launch_bounds__(kTabThreads) k_tab_scan(int E, int nu, int* __restrict__ unit_counts,
+                                                          int* __restrict__ totals) {
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * kTabWarps + (threadIdx.x >> 5);
+  if (e >= E) return;   // whole warps
+  int run = 0;
+  for (int v0 = 0; v0 < nu; v0 += 32) {
+    const int v = v0 + lane;
+    const int c = v < nu ? unit_counts[(size_t)v * E + e] : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (v < nu) unit_counts[(size_t)v * E + e] = run + incl - c;
+    run += __shfl_sync(kFull, incl, 31);
+  }
+  if (lane == 0) totals[e] = run;
 }
 
 __global__ void __launch_bounds__(kTabThreads) k_tab_scatter(const uint8_t* __restrict__ act, int T, int E,
-                                                             const int* __restrict__ unit_counts, int nu,
-                                                             int* counts, int* offsets, int* perm, int* pair_of,
-                                                             int4* tiles, int* n_tiles, int tile_rows) {
-  __shared__ int base[kTabWarps][256];   // first position of the unit's pairs, per expert
+                                                             const int* __restrict__ unit_base,
+                                                             const int* __restrict__ totals, int* counts,
+                                                             int* offsets, int* perm, int* pair_of, int4* tiles,
+                                                             int* n_tiles, int tile_rows) {
+  __shared__ __align__(16) uint8_t flags[kTabWarps][kTabUnit * 256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * kTabWarps + warp;
   if (u * kTabUnit >= T) return;   // whole warps; no block-wide barrier below
   // per expert (lane j: experts j, j + 32, ...): the total count and the
-  // pairs in earlier units
+  // pairs of the expert in earlier units
   int tot[8], before[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    tot[i] = 0;
-    before[i] = 0;
+    const int e = lane + 32 * i;
+    tot[i] = e < E ? totals[e] : 0;
+    before[i] = e < E ? unit_base[(size_t)u * E + e] : 0;
   }
-  for (int v = 0; v < nu; ++v) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E) {
-        const int c = unit_counts[(size_t)v * E + e];
-        tot[i] += c;
-        if (v < u) before[i] += c;
-      }
-    }
-  }
+  uint8_t* fl = flags[warp];
+  load_unit_flags(act, T, E, u, fl);
   // exclusive scan of tot over experts (ascending e = i * 32 + lane)
   int run = 0, ntl_run = 0;
   int off[8], toff[8];
@@ -1063,11 +1094,6 @@ __global__ void __launch_bounds__(kTabThreads) k_tab_scatter(const uint8_t* __re
     run += __shfl_sync(kFull, incl, 31);
     ntl_run += __shfl_sync(kFull, incl_t, 31);
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) base[warp][e] = off[i] + before[i];
-  }
   if (u == 0) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -1084,25 +1110,20 @@ __global__ void __launch_bounds__(kTabThreads) k_tab_scatter(const uint8_t* __re
       *n_tiles = ntl_run;
     }
   }
-  __syncwarp();
-  // this unit's tokens: lane = token
-  const int t = u * kTabUnit + lane;
-  const bool ok = t < T;
-  const uint8_t* row = act + (size_t)(ok ? t : 0) * E;
-  const unsigned lt = (1u << lane) - 1u;
-  for (int e0 = 0; e0 < E; e0 += 32) {
-    const uint32_t bits = row_bits(row, ok, E, e0);
-    for (int j = 0; j < 32 && e0 + j < E; ++j) {
-      const int e = e0 + j;
-      const bool f = (bits >> j) & 1u;
-      const unsigned m = __ballot_sync(kFull, f);
-      if (f) {
-        const int pos = base[warp][e] + __popc(m & lt);
-        perm[pos] = t;
-        pair_of[(size_t)t * E + e] = pos;
-      } else if (ok) {
-        pair_of[(size_t)t * E + e] = -1;
-      }
+  // the unit's pairs: lane j walks the 32 tokens for experts j, j + 32, ...;
+  // the pair_of row of a token is written by the lanes together
+  const int t0 = u * kTabUnit;
+  const int nt = min(kTabUnit, T - t0);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    if (i * 32 >= E) break;
+    int pos = off[i] + before[i];
+    for (int t = 0; t < nt; ++t) {
+      const bool f = e < E && fl[t * E + e];
+      if (f) perm[pos] = t0 + t;
+      if (e < E) pair_of[(size_t)(t0 + t) * E + e] = f ? pos : -1;
+      pos += f ? 1 : 0;
     }
   }
 }

@@ -501,3 +501,26 @@ def test_residual_stack_prefill_t16384(lib):
         x = out
         del G, rt
     assert torch.isfinite(x.float()).all()
+
+
+@pytest.mark.parametrize("shape,topk", [
+    (LayerShape(40, 256, 8, 512, 64, "bf16"), 0),      # tiled router, general expert kernels (d_e 512)
+    (LayerShape(300, 320, 5, 192, 320, "bf16"), 0),    # tensor-core kernels
+    (LayerShape(16, 512, 16, 256, 256, "bf16"), 0),    # decode kernel
+    (LayerShape(37, 256, 8, 128, 192, "f32"), 0),      # general kernels
+    (LayerShape(300, 320, 5, 192, 320, "bf16"), 2),    # TopK routing, tensor-core kernels
+    (LayerShape(16, 512, 16, 256, 256, "bf16"), 3),    # TopK routing, decode kernel
+])
+def test_workspace_size_covers_every_write(lib, shape, topk):
+    """The kernels write only inside deco_moe_workspace_size bytes: a guard
+    region after the workspace keeps its byte pattern through a forward and a
+    routing call, and the output still matches the oracle's routing."""
+    L = make_layer(shape, 81)
+    G = to_gpu(L, lib)
+    n = lib.workspace_size(lib.layer_shape(G["x"], G, topk=topk))
+    buf = torch.full((n + 65536,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws = buf[:n]
+    lib.forward(G["x"], G, workspace=ws, eps=shape.eps, topk=topk)
+    lib.routing(G["x"], G, workspace=ws, topk=topk)
+    torch.cuda.synchronize()
+    assert bool((buf[n:] == 0xA5).all())
