@@ -194,10 +194,18 @@ def norm_silu(g: np.ndarray, u: np.ndarray, eps: float):
     return c, h, silu(h)
 
 
-def expert_output(x_t, W_up_e, W_down_e, u_t, eps):
-    """Routed expert e on token t: v = W_down[e] NormSiLU(W_up[e] x_t)."""
+def expert_output(x_t, W_up_e, W_down_e, u_t, eps, W_val_e=None):
+    """Routed expert e on token t: v = W_down[e] NormSiLU(W_up[e] x_t).
+
+    Gated variant ("DECO (gated)", the ablation of [press] part 2 and [arXiv]
+    §2 "Expert design"), when W_val_e is given: the NormSiLU output is
+    multiplied element-wise by a linear value branch,
+    v = W_down[e] (NormSiLU(W_up[e] x_t) * (W_val[e] x_t)).
+    """
     g = W_up_e @ x_t
     _, _, a = norm_silu(g, u_t, eps)
+    if W_val_e is not None:
+        a = a * (W_val_e @ x_t)
     return W_down_e @ a
 
 
@@ -213,7 +221,8 @@ def layer_forward_tokens(x: np.ndarray, L: dict, eps: float, tokens=None):
     """Forward pass of one DECO MoE layer for the listed tokens (default all).
 
     L holds fp64 arrays W_r [E,D], b_r [E], W_up [E,d_e,D], W_bar_up [d_e,D],
-    W_down [E,D,d_e], s [E], W_s_up [d_s,D], W_s_down [D,d_s].
+    W_down [E,D,d_e], s [E], W_s_up [d_s,D], W_s_down [D,d_s], and for the
+    gated variant W_val [E,d_e,D].
     Returns (y [n,D] fp64 before rounding, z [n,E], active [n,E]).
     """
     if tokens is None:
@@ -229,9 +238,11 @@ def layer_forward_tokens(x: np.ndarray, L: dict, eps: float, tokens=None):
         z = router_logits(x_t, L["W_r"], L["b_r"])
         u = L["W_bar_up"] @ x_t
         routed = np.zeros(D)
+        W_val = L.get("W_val")
         for e in range(E):
             if z[e] > 0.0:
-                v = expert_output(x_t, L["W_up"][e], L["W_down"][e], u, eps)
+                v = expert_output(x_t, L["W_up"][e], L["W_down"][e], u, eps,
+                                  None if W_val is None else W_val[e])
                 routed = routed + (L["s"][e] * z[e]) * v
         y[i] = shared_expert(x_t, L["W_s_up"], L["W_s_down"]) + routed
         zs[i] = z

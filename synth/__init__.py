@@ -38,7 +38,7 @@ DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 # tensor ids used in the seed formula
 _TID = dict(x=0, W_r=1, W_up=2, W_down=3, s=4, W_s_up=5, W_s_down=6, jitter=7,
-            W1=8, W2=9)
+            W1=8, W2=9, W_val=10)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -59,7 +59,10 @@ class LayerShape:
 
 def _gen(seed: int, layer: int, tid: str) -> torch.Generator:
     g = torch.Generator()
-    g.manual_seed(seed * 1000 + layer * 10 + _TID[tid])
+    i = _TID[tid]
+    # ids 0..9: seed*1000 + layer*10 + id; later ids (the gated value branch)
+    # start a second block, seed*1000 + 500 + layer*10 + (id - 10), layer < 50
+    g.manual_seed(seed * 1000 + layer * 10 + i if i < 10 else seed * 1000 + 500 + layer * 10 + (i - 10))
     return g
 
 
@@ -79,12 +82,14 @@ def make_x(T: int, D: int, dtype: str, seed: int, layer: int = 0) -> torch.Tenso
 
 
 def make_layer(shape: LayerShape, seed: int, layer: int = 0, ratio: float = 0.2,
-               jitter: float = 0.0, zero_every: int = 0, with_x: bool = True) -> dict:
+               jitter: float = 0.0, zero_every: int = 0, with_x: bool = True,
+               gated: bool = False) -> dict:
     """Draw one layer's weights (and its input batch) on the CPU.
 
     Returns a dict of CPU tensors in the storage dtype (b_r and s are always
     fp32): x [T,D], W_r [E,D], b_r [E], W_up [E,d_e,D], W_down [E,D,d_e],
-    s [E], W_s_up [d_s,D], W_s_down [D,d_s].
+    s [E], W_s_up [d_s,D], W_s_down [D,d_s], and with gated=True the gated
+    experts' value branch W_val [E,d_e,D] ~ N(0, 1/D).
     """
     T, D, E, d_e, d_s = shape.T, shape.D, shape.E, shape.d_e, shape.d_s
     td = shape.torch_dtype
@@ -104,6 +109,8 @@ def make_layer(shape: LayerShape, seed: int, layer: int = 0, ratio: float = 0.2,
 
     out = dict(W_r=W_r, b_r=b_r, W_up=W_up, W_down=W_down, s=s,
                W_s_up=W_s_up, W_s_down=W_s_down)
+    if gated:
+        out["W_val"] = _normal((E, d_e, D), 1.0 / math.sqrt(D), seed, layer, "W_val").to(td)
     if with_x:
         g = _normal((T, D), 1.0, seed, layer, "x")
         if jitter > 0.0:

@@ -348,3 +348,61 @@ def test_topk_route_matches_brute_force_exact_ranking():
             assert sorted(np.nonzero(act[t])[0].tolist()) == sorted(want)
             for e in range(9):
                 assert r[t, e] == (max(float(vals[e]), 0.0) if e in want else 0.0)
+
+
+# --------------------------------------------------------------------------
+# gated experts ("DECO (gated)"): a = NormSiLU(W_up x) * (W_val x)
+
+def test_gated_value_of_one_is_the_non_gated_layer():
+    # W_val[e] = ones (x) x_t / (x_t . x_t) makes every value feature of token t
+    # equal to 1, so the gated layer on t equals the non-gated one
+    shape = LayerShape(3, 32, 4, 16, 8, "f32")
+    L = _layer64(shape, 3, ratio=0.6)
+    t = 1
+    x_t = L["x"][t]
+    Lg = dict(L, W_val=np.stack([np.outer(np.ones(16), x_t) / float(x_t @ x_t)] * 4))
+    y, _, act = O.layer_forward_tokens(L["x"], L, 1e-6, [t])
+    yg, _, _ = O.layer_forward_tokens(L["x"], Lg, 1e-6, [t])
+    assert act.any()
+    np.testing.assert_allclose(yg, y, rtol=1e-12, atol=1e-12)
+
+
+def test_gated_zero_value_leaves_only_the_shared_expert():
+    shape = LayerShape(5, 32, 4, 16, 8, "f32")
+    L = _layer64(shape, 4, ratio=0.6)
+    Lg = dict(L, W_val=np.zeros((4, 16, 32)))
+    y, _, act = O.layer_forward_tokens(L["x"], Lg, 1e-6)
+    assert act.any()
+    shared = np.stack([O.shared_expert(L["x"][t], L["W_s_up"], L["W_s_down"]) for t in range(5)])
+    np.testing.assert_allclose(y, shared, rtol=0, atol=1e-14)
+
+
+def test_gated_routed_part_is_linear_in_the_value_branch():
+    shape = LayerShape(6, 32, 4, 16, 8, "f32")
+    L = _layer64(shape, 5, ratio=0.5)
+    W_val = np.random.default_rng(0).normal(size=(4, 16, 32)) / math.sqrt(32)
+    shared = np.stack([O.shared_expert(L["x"][t], L["W_s_up"], L["W_s_down"]) for t in range(6)])
+    y1, _, act = O.layer_forward_tokens(L["x"], dict(L, W_val=W_val), 1e-6)
+    y3, _, _ = O.layer_forward_tokens(L["x"], dict(L, W_val=-3.0 * W_val), 1e-6)
+    assert act.any()
+    np.testing.assert_allclose(y3 - shared, -3.0 * (y1 - shared), rtol=1e-12, atol=1e-12)
+
+
+def test_gated_sparse_equals_dense_evaluation_masked_by_relu():
+    # every expert evaluated for every token, multiplied by ReLU(z): the
+    # inactive ones drop out
+    shape = LayerShape(7, 32, 5, 16, 8, "bf16")
+    L = _layer64(shape, 6, ratio=0.4)
+    L["W_val"] = O.to_f64(make_layer(shape, 6, gated=True)["W_val"])
+    y = O.layer_forward(L["x"], L, 1e-6)
+    for t in range(7):
+        x_t = L["x"][t]
+        z = O.router_logits(x_t, L["W_r"], L["b_r"])
+        u = L["W_bar_up"] @ x_t
+        ref = O.shared_expert(x_t, L["W_s_up"], L["W_s_down"])
+        for e in range(5):
+            c = L["W_up"][e] @ x_t - u
+            h = c / math.sqrt(float(np.mean(c * c)) + 1e-6)
+            a = h / (1.0 + np.exp(-h)) * (L["W_val"][e] @ x_t)
+            ref = ref + L["s"][e] * max(z[e], 0.0) * (L["W_down"][e] @ a)
+        np.testing.assert_allclose(y[t], ref, rtol=1e-12, atol=1e-12)
