@@ -82,7 +82,11 @@ typedef enum { DECO_F32 = 0, DECO_BF16 = 1 } deco_dtype_t;
  *            k in 1..E: the TopK baseline of [arXiv] §5 -- each token keeps
  *            its k largest logits (ranked on their exact values, exact ties
  *            to the lower expert index) with weights ReLU(z_e), not
- *            renormalised; everything after the router is unchanged      */
+ *            renormalised; everything after the router is unchanged
+ *   gated    0: DECO's non-gated experts.  1: the gated variant of the
+ *            ablation ([press] part 2, non-gated paragraph; [arXiv] §2
+ *            "Expert design"): a_e = NormSiLU(x W_up[e]^T - u) * (x W_val[e]^T),
+ *            element-wise, with the value branch W_val (weights.W_val)    */
 typedef struct {
   int T;
   int d_model;
@@ -93,6 +97,7 @@ typedef struct {
   float rms_eps;
   int residual;
   int topk;
+  int gated;
 } deco_moe_shape_t;
 
 /* The layer's weights (device pointers, storage dtype unless noted).
@@ -103,7 +108,9 @@ typedef struct {
  *   W_down   [E][D][d_e]   routed down-projections
  *   s        [E]     fp32  learnable expert-wise router scaling
  *   W_s_up   [d_s][D]      shared expert up-projection
- *   W_s_down [D][d_s]      shared expert down-projection                    */
+ *   W_s_down [D][d_s]      shared expert down-projection
+ *   W_val    [E][d_e][D]   gated experts' value branch (shape->gated = 1;
+ *                          NULL otherwise)                                  */
 typedef struct {
   const void* W_r;
   const float* b_r;
@@ -113,6 +120,7 @@ typedef struct {
   const float* s;
   const void* W_s_up;
   const void* W_s_down;
+  const void* W_val;
 } deco_moe_weights_t;
 
 /* Routing outputs of deco_moe_routing (device pointers; any may be NULL to

@@ -40,12 +40,15 @@ class DecoError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("E", ctypes.c_int),
                 ("d_e", ctypes.c_int), ("d_s", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("rms_eps", ctypes.c_float), ("residual", ctypes.c_int), ("topk", ctypes.c_int)]
+                ("rms_eps", ctypes.c_float), ("residual", ctypes.c_int), ("topk", ctypes.c_int),
+                ("gated", ctypes.c_int)]
+
+
+WEIGHT_NAMES = ("W_r", "b_r", "W_up", "W_bar_up", "W_down", "s", "W_s_up", "W_s_down", "W_val")
 
 
 class Weights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in
-                ("W_r", "b_r", "W_up", "W_bar_up", "W_down", "s", "W_s_up", "W_s_down")]
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_NAMES]
 
 
 class Routing(ctypes.Structure):
@@ -95,21 +98,20 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def make_shape(T, D, E, d_e, d_s, dtype, eps=1e-6, residual=False, topk=0) -> Shape:
+def make_shape(T, D, E, d_e, d_s, dtype, eps=1e-6, residual=False, topk=0, gated=False) -> Shape:
     return Shape(T, D, E, d_e, d_s, _DT[dtype] if isinstance(dtype, torch.dtype) else dtype,
-                 eps, int(bool(residual)), int(topk))
+                 eps, int(bool(residual)), int(topk), int(bool(gated)))
 
 
 def _weights(L: dict) -> Weights:
-    return Weights(*[_ptr(L.get(n)) for n in
-                     ("W_r", "b_r", "W_up", "W_bar_up", "W_down", "s", "W_s_up", "W_s_down")])
+    return Weights(*[_ptr(L.get(n)) for n in WEIGHT_NAMES])
 
 
 def layer_shape(x: torch.Tensor, L: dict, eps=1e-6, residual=False, topk=0) -> Shape:
     E, d_e, D = L["W_up"].shape if "W_up" in L else (L["W_r"].shape[0], 64, x.shape[1])
     d_s = L["W_s_up"].shape[0] if "W_s_up" in L else 64
     return make_shape(x.shape[0], x.shape[1], L["W_r"].shape[0], d_e, d_s, x.dtype, eps, residual,
-                      topk)
+                      topk, "W_val" in L)
 
 
 def workspace_size(shape: Shape) -> int:

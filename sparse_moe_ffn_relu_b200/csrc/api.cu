@@ -27,10 +27,10 @@ struct Plan {
   // decode path (T <= 16): up-projection partials, shared hidden and NormSiLU
   // tiles, per-CTA down-projection partials (the inter-CTA counters follow
   // the error word)
-  size_t C16, HS, A16, Part, tmask;
+  size_t C16, C16v, HS, A16, Part, tmask;
   // bf16, T > 16: ambiguous router pairs; prefill path: routed expert output
   // rows (one fp16 row per pair) and the shared expert's fp32 output
-  size_t fb, blk, etot, v_pairs, coef, s_out;
+  size_t fb, blk, etot, v_pairs, coef, s_out, val_pairs;
   // TopK routing: fp32 logits and their error bounds
   size_t zt, bt;
   int tile_rows;
@@ -98,10 +98,12 @@ Plan make_plan(const deco_moe_shape_t& s) {
   if (prefill_eligible(s)) {
     p.v_pairs = take(P * s.d_model * 2);
     p.coef = take(P * 4);
+    if (s.gated) p.val_pairs = take(P * s.d_e * 2);   // bf16 value-branch rows per pair
     p.s_out = take(T * s.d_model * 4);
   }
   if (s.T <= dec::kMaxT) {         // decode path buffers (see decode_kernels.cuh)
     p.C16 = take(8 * E * dec::kTok * s.d_e * 4);                       // [kp <= 8][E][16][d_e] fp32
+    if (s.gated) p.C16v = take(8 * E * dec::kTok * s.d_e * 4);         // the same for the value branch
     p.HS = take((size_t)dec::down_nsq(s.d_s) * dec::kTileBytes);       // [nsq] 16 KB tiles
     p.A16 = take(E * dec::kTileBytes);                                 // [E] 16 KB tiles
     p.Part = take((size_t)std::max(p.sms, 1) * 2 * dec::kTok * dec::kDRows * 4);   // [G][2][16][128]
@@ -121,6 +123,7 @@ deco_status_t check_shape(const deco_moe_shape_t* s) {
   if (!(s->rms_eps >= 0.f) || !std::isfinite(s->rms_eps)) return DECO_ERR_INVALID_ARG;
   if (s->residual != 0 && s->residual != 1) return DECO_ERR_INVALID_ARG;
   if (s->topk < 0 || s->topk > s->E) return DECO_ERR_INVALID_ARG;
+  if (s->gated != 0 && s->gated != 1) return DECO_ERR_INVALID_ARG;
   if (s->d_model % 64 || s->d_model > 16384) return DECO_ERR_UNSUPPORTED;
   if (s->E > 256) return DECO_ERR_UNSUPPORTED;
   if (s->d_e % 64 || s->d_e > 512) return DECO_ERR_UNSUPPORTED;
@@ -129,10 +132,11 @@ deco_status_t check_shape(const deco_moe_shape_t* s) {
   return DECO_OK;
 }
 
-deco_status_t check_weights(const deco_moe_weights_t* w, bool router_only) {
+deco_status_t check_weights(const deco_moe_weights_t* w, bool router_only, bool gated = false) {
   if (!w || !w->W_r || !w->b_r) return DECO_ERR_INVALID_ARG;
   if (!aligned16(w->W_r)) return DECO_ERR_INVALID_ARG;
   if (router_only) return DECO_OK;
+  if (gated && (!w->W_val || !aligned16(w->W_val))) return DECO_ERR_INVALID_ARG;
   const void* ps[] = {w->W_up, w->W_bar_up, w->W_down, w->s, w->W_s_up, w->W_s_down};
   for (const void* p : ps)
     if (!p || !aligned16(p)) return DECO_ERR_INVALID_ARG;
@@ -213,7 +217,7 @@ cudaError_t route_any(const RouteArgs& a, int tt, cudaStream_t st) {
 
 template <typename T, int TT>
 cudaError_t launch_up(const UpArgs& a, int max_tiles, cudaStream_t st) {
-  const size_t smem = (size_t)TT * a.D * sizeof(T) + (size_t)TT * (a.d_e / kCluster) * sizeof(float);
+  const size_t smem = (size_t)TT * a.D * sizeof(T) + (a.W_val ? 2 : 1) * (size_t)TT * (a.d_e / kCluster) * sizeof(float);
   cudaError_t err = allow_smem(k_up<T, TT>, smem);
   if (err != cudaSuccess) return err;
   int clusters = std::min(max_tiles, std::max(1, 2 * num_sms() / kCluster));
@@ -387,8 +391,8 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
 
 // one CTA per SM, all resident at once (the CTAs wait on one another's
 // counters), so the launch is cooperative
-cudaError_t launch_layer(const CUtensorMap& tmU, const CUtensorMap& tmW, const CUtensorMap& tmS,
-                         const dec::Args& a, int sms, cudaStream_t st) {
+cudaError_t launch_layer(const CUtensorMap& tmU, const CUtensorMap& tmV, const CUtensorMap& tmW,
+                         const CUtensorMap& tmS, const dec::Args& a, int sms, cudaStream_t st) {
   const uint32_t smem = dec::layer_smem(a.D).total;
   cudaError_t err = cudaFuncSetAttribute(dec::kd_layer, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -402,7 +406,7 @@ cudaError_t launch_layer(const CUtensorMap& tmU, const CUtensorMap& tmW, const C
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, dec::kd_layer, tmU, tmW, tmS, a);
+  return cudaLaunchKernelEx(&cfg, dec::kd_layer, tmU, tmV, tmW, tmS, a);
 }
 
 // the decode kernel's buffers in a workspace laid out by make_plan
@@ -441,16 +445,20 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
   a.W_s_down = static_cast<const bf16*>(w.W_s_down);
   a.out = static_cast<bf16*>(out);
   a.pre_routed = s.topk > 0;
+  a.gated = s.gated;
+  a.Cv = s.gated ? reinterpret_cast<float*>(ws + p.C16v) : nullptr;
   decode_buffers(a, ws, p);
   // weight tiles of phases U and D: 128 rows x 64 columns
-  CUtensorMap tmU, tmW, tmS;
+  CUtensorMap tmU, tmV, tmW, tmS;
   cudaError_t err;
-  if ((err = make_map(&tmU, w.W_up, s.d_model, (uint64_t)s.E * s.d_e, dec::kDRows)) != cudaSuccess ||
+  if ((err = make_map(&tmV, s.gated ? w.W_val : w.W_up, s.d_model, (uint64_t)s.E * s.d_e, dec::kDRows)) !=
+          cudaSuccess ||
+      (err = make_map(&tmU, w.W_up, s.d_model, (uint64_t)s.E * s.d_e, dec::kDRows)) != cudaSuccess ||
       (err = make_map(&tmW, w.W_down, s.d_e, (uint64_t)s.E * s.d_model, dec::kDRows)) != cudaSuccess ||
       (err = make_map(&tmS, w.W_s_down, s.d_s, s.d_model, dec::kDRows)) != cudaSuccess)
     return err;
   prof_mark(16, st);
-  err = launch_layer(tmU, tmW, tmS, a, p.sms, st);
+  err = launch_layer(tmU, tmV, tmW, tmS, a, p.sms, st);
   prof_mark(17, st);
   return err;
 }
@@ -484,7 +492,7 @@ cudaError_t run_dense_decode(int T, int D, int d_ff, const void* x, const void* 
   cudaError_t err;
   CUtensorMap tmS;
   if ((err = make_map(&tmS, W2, d_ff, D, dec::kDRows)) != cudaSuccess) return err;
-  return launch_layer(tmS, tmS, tmS, a, sms, st);   // no routed experts: the W_up / W_down maps are unused
+  return launch_layer(tmS, tmS, tmS, tmS, a, sms, st);   // no routed experts: the other maps are unused
 }
 
 // ---------------------------------------------------------------------------
@@ -533,6 +541,7 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   a.a_pairs = reinterpret_cast<bf16*>(ws + p.H);
   a.v_pairs = reinterpret_cast<__half*>(ws + p.v_pairs);
   a.coef_pairs = reinterpret_cast<float*>(ws + p.coef);
+  a.val_pairs = s.gated ? reinterpret_cast<const bf16*>(ws + p.val_pairs) : nullptr;
   a.s_out = reinterpret_cast<float*>(ws + p.s_out);
   a.out = static_cast<bf16*>(out);
   a.err = reinterpret_cast<int*>(ws + p.err);
@@ -563,9 +572,17 @@ cudaError_t run_prefill(const deco_moe_shape_t& s, const void* x, const deco_moe
   err = launch_pf<pf::kProj>(mx, mbar, msup, ou, ohs, a, std::min(a.m_tiles * a.n_tiles_n, p.sms), st);
   if (err != cudaSuccess) return err;
   prof_mark(11, st);
-  // routed up-projections with NormSiLU
+  // routed up-projections with NormSiLU (after the value rows of gated experts)
   a.bn = d_e;
   prof_mark(6, st);
+  if (s.gated) {
+    CUtensorMap mval, oval;
+    if ((err = make_map(&mval, w.W_val, D, (uint64_t)E * d_e, pf::kBN)) != cudaSuccess ||
+        (err = make_map(&oval, a.val_pairs, d_e, P, 32)) != cudaSuccess)
+      return err;
+    err = launch_pf<pf::kVal>(mx, mval, mval, oval, oval, a, std::min(row_tiles_max, p.sms), st);
+    if (err != cudaSuccess) return err;
+  }
   err = launch_pf<pf::kUp>(mx, mup, mup, oapr, oapr, a, std::min(row_tiles_max, p.sms), st);
   if (err != cudaSuccess) return err;
   prof_mark(7, st);
@@ -651,6 +668,7 @@ cudaError_t run_forward(const deco_moe_shape_t& s, const void* x, const deco_moe
   ua.x = x;
   ua.D = s.d_model;
   ua.W_up = w.W_up;
+  ua.W_val = s.gated ? w.W_val : nullptr;
   ua.d_e = s.d_e;
   ua.u = reinterpret_cast<const float*>(ws + p.u);
   ua.perm = reinterpret_cast<const int*>(ws + p.perm);
@@ -722,7 +740,7 @@ deco_status_t deco_moe_forward(const deco_moe_shape_t* shape, const void* x,
                                size_t workspace_bytes, void* stream) {
   deco_status_t st = check_shape(shape);
   if (st != DECO_OK) return st;
-  if ((st = check_weights(w, false)) != DECO_OK) return st;
+  if ((st = check_weights(w, false, shape->gated)) != DECO_OK) return st;
   if (shape->T == 0) return DECO_OK;
   if (!x || !out || !aligned16(x) || !aligned16(out) || x == out) return DECO_ERR_INVALID_ARG;
   const Plan p = make_plan(*shape);
@@ -926,7 +944,7 @@ extern "C" deco_status_t deco_moe_forward_static(const deco_moe_shape_t* shape, 
                                                  void* stream) {
   deco_status_t st = check_shape(shape);
   if (st != DECO_OK) return st;
-  if ((st = check_weights(w, false)) != DECO_OK) return st;
+  if ((st = check_weights(w, false, shape->gated)) != DECO_OK) return st;
   if (shape->T == 0) return DECO_OK;
   if (!x || !out || !aligned16(x) || !aligned16(out) || x == out) return DECO_ERR_INVALID_ARG;
   if (make_plan(*shape).total > DECO_STATIC_SCRATCH_BYTES) return DECO_ERR_WORKSPACE;

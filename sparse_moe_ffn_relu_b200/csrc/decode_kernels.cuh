@@ -322,6 +322,7 @@ struct Args {
   int residual;
   long long wait_cycles;   // limit of the waits for data (kWaitCycles unless a test lowers it)
   int pre_routed;          // r and act come from earlier kernels (TopK routing): no router CTAs
+  int gated;               // gated experts: a = NormSiLU(x W_up^T - u) * (x W_val^T)
   const bf16* x;
   const bf16* W_r;
   const float* b_r;
@@ -339,6 +340,7 @@ struct Args {
   bf16* A;           // [E][16 tok][256 hi | 256 lo]: s_e r_e NormSiLU(x W_up[e]^T), 0 for
                      // tokens not using e
   float* C;          // [kp <= 8][E][16 tok][d_e]: partial sums of x W_up[e]^T over K parts
+  float* Cv;         // the same for x W_val[e]^T (gated experts)
   float* Part;       // [G][2][16 tok][128]: a CTA's down-projection sum per row block
   unsigned* sync;    // inter-CTA counters (layout: SyncIdx); kd_layer clears them itself
   int* err;
@@ -665,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) kd_router(const __grid_constant__
 // phase's units, in order).
 struct Sched {
   int U;              // active experts (the union)
+  int nbr;            // up-projection matrices per expert: W_up, and W_val when gated
   int kp, Kp, nrb_up, nrb, nsq;
   int NU;             // phase-U units
   int J, ND;          // phase-D units per row block, and in all
@@ -676,24 +679,28 @@ __device__ __forceinline__ Sched make_sched(const Args& a, int U, int G) {
   S.nrb_up = (a.d_e + kDRows - 1) / kDRows;
   S.nrb = a.D / kDRows;
   S.nsq = down_nsq(a.d_s);
-  S.kp = up_kparts(U, a.d_e, a.D, G);
+  S.nbr = a.gated ? 2 : 1;
+  S.kp = up_kparts(U * S.nbr, a.d_e, a.D, G);
   S.Kp = a.D / S.kp;
-  S.NU = U * S.nrb_up * S.kp;
+  S.NU = U * S.nbr * S.nrb_up * S.kp;
   S.J = S.nsq + U;
   S.ND = S.nrb * S.J;
   return S;
 }
 
-// unit u of phase U: index of its expert in the union, the block of 128 rows
-// of W_up[e] and the K part
+// unit u of phase U: index of its expert in the union, the matrix (0 W_up,
+// 1 W_val), the block of 128 rows of it and the K part; an expert's units
+// are consecutive
 struct UUnit {
-  int ei, rbu, p;
+  int ei, mat, rbu, p;
 };
 __device__ __forceinline__ UUnit up_unit(const Sched& S, int u) {
   UUnit q;
   q.p = u % S.kp;
   q.rbu = (u / S.kp) % S.nrb_up;
-  q.ei = u / (S.kp * S.nrb_up);
+  const int m = u / (S.kp * S.nrb_up);
+  q.mat = m % S.nbr;
+  q.ei = m / S.nbr;
   return q;
 }
 
@@ -742,8 +749,9 @@ __device__ __forceinline__ int rb_sources(int rb, const Sched& S, int G, int* sr
 }
 
 // NormSiLU tile of expert e (consumer threads): c = sum of the K parts of g
-// minus u, h = c / sqrt(mean c^2 + eps), a = s_e r_e SiLU(h) as hi/lo rows;
-// rows of tokens not using e are zero.
+// minus u, h = c / sqrt(mean c^2 + eps), a = s_e r_e SiLU(h) (times the value
+// branch for gated experts) as hi/lo rows; rows of tokens not using e are
+// zero.
 __device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   bf16* tile = a.A + (size_t)e * kTileElems;
@@ -789,6 +797,34 @@ __device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
     }
 #pragma unroll
     for (int q = 0; q < 8; ++q) ss = fmaf(cv[q], cv[q], ss);
+    // gated experts: the value branch, its K parts added in order
+    float val[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) val[q] = 1.f;
+    if (a.gated) {
+      float4 vp[8][2];
+#pragma unroll
+      for (int pp = 0; pp < 8; ++pp) {
+        const float4* src = reinterpret_cast<const float4*>(a.Cv + (((size_t)pp * a.E + e) * kTok + t) * a.d_e) + 2 * lane;
+        vp[pp][0] = (pp < kp && live) ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+        vp[pp][1] = (pp < kp && live) ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float g[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int pp = 0; pp < 8; ++pp) {
+          g[0] += vp[pp][h].x;
+          g[1] += vp[pp][h].y;
+          g[2] += vp[pp][h].z;
+          g[3] += vp[pp][h].w;
+        }
+        val[4 * h + 0] = g[0];
+        val[4 * h + 1] = g[1];
+        val[4 * h + 2] = g[2];
+        val[4 * h + 3] = g[3];
+      }
+    }
     ss = warp_sum(ss);
     const float rinv = 1.f / sqrtf(ss / float(a.d_e) + a.eps);
     const float coef = se * rte;
@@ -796,7 +832,8 @@ __device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float v0 = coef * silu_f(cv[2 * q] * rinv), v1 = coef * silu_f(cv[2 * q + 1] * rinv);
+        const float v0 = coef * silu_f(cv[2 * q] * rinv) * val[2 * q];
+        const float v1 = coef * silu_f(cv[2 * q + 1] * rinv) * val[2 * q + 1];
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
         const float2 hf = __bfloat1622float2(h2);
         const __nv_bfloat162 l2 = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
@@ -869,8 +906,9 @@ __device__ void combine_rb(const Args& a, int rb, const int* src, int n) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    kd_layer(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmW,
-             const __grid_constant__ CUtensorMap tmS, const __grid_constant__ Args a) {
+    kd_layer(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmV,
+             const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
+             const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ unsigned long long limbs[kLimbs];
   __shared__ uint16_t emask[256];   // the producer warp's union: token masks, active experts
@@ -989,13 +1027,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = u0; u < u1 && ok; ++u) {
           const UUnit q = up_unit(S, u);
           const int row = ulist[q.ei] * a.d_e + q.rbu * kDRows;
+          const CUtensorMap* mu = q.mat ? &tmV : &tmU;
           for (int c0 = 0; c0 < S.Kp; c0 += 128) {
             int s;
             if (!(ok = next_stage(s))) break;
             const int nb = min(2, (S.Kp - c0) / 64);
             mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
             for (int b = 0; b < nb; ++b)
-              tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, &tmU, q.p * S.Kp + c0 + 64 * b,
+              tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, mu, q.p * S.Kp + c0 + 64 * b,
                      row, &ctl.full[s], pol);
             ++k;
           }
@@ -1197,7 +1236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 4; ++i) {
             const int t = 8 * nt + 2 * (lane & 3) + (i & 1);
             const int j = j0 + 8 * (i >> 1);
-            if (t < a.T && j < a.d_e) a.C[(((size_t)p * a.E + e) * kTok + t) * a.d_e + j] = acc[nt][i];
+            if (t < a.T && j < a.d_e) (q.mat ? a.Cv : a.C)[(((size_t)p * a.E + e) * kTok + t) * a.d_e + j] = acc[nt][i];
           }
         }
       }
@@ -1210,7 +1249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int last = 0;
           if (ok) {
             const unsigned old = atom_add_acq_rel(sync + si.g_cnt + e, (unsigned)n_here);
-            last = old + (unsigned)n_here == (unsigned)(nrb_up * kp);
+            last = old + (unsigned)n_here == (unsigned)(S.nbr * nrb_up * kp);
             // u comes from phase R
             if (last && !pre_seen)
               last = pre_seen = spin_until(sync + si.pre_done, (unsigned)Gp, a.wait_cycles, ctl.abort_flag, a.err);

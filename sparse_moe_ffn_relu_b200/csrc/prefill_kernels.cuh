@@ -19,6 +19,8 @@
 //                                                s_e * r_e (fp32, per pair)
 //   kDown    a rows of expert e x W_down[e]^T  -> v (fp16, one row per pair)
 //   kShared  hs x W_s_down^T                   -> S (fp32)
+//   kVal     (gated experts) gathered x rows x W_val[e]^T -> value rows (bf16,
+//            one per pair), which kUp's epilogue multiplies in
 //
 // and two CUDA-core kernels around them: k_router (exact ReLU routing) and
 // k_combine, out = S + the token's routed rows s_e r_e v in ascending expert
@@ -83,7 +85,10 @@ constexpr uint32_t kEpiOffset = kStages * (kABytes + kBBytes);
 constexpr uint32_t kBarOffset = kEpiOffset + 4 * 2 * kStageOut;   // two boxes per epilogue warp
 constexpr size_t kSmemBytes = 1024 + kBarOffset + 256;   // 1 KB alignment slack + ring + boxes + barriers
 
-enum : int { kProj = 0, kUp = 1, kDown = 2, kShared = 3 };
+enum : int { kProj = 0, kUp = 1, kDown = 2, kShared = 3, kVal = 4 };
+// the modes whose A rows are gathered token rows of x (one expert's pairs)
+template <int MODE>
+__host__ __device__ constexpr bool gathers() { return MODE == kUp || MODE == kVal; }
 constexpr int kErrRange = 4;   // device error bit: a routed expert output outside the fp16 range
 
 struct Args {
@@ -106,6 +111,8 @@ struct Args {
   float* u;                   // [T][d_e]
   bf16* hs;                   // [T][d_s]
   bf16* a_pairs;              // [pairs][d_e] NormSiLU outputs, SiLU(h): |a| <= sqrt(d_e)
+                              // (times the value branch for gated experts)
+  const bf16* val_pairs;      // [pairs][d_e] gated experts' value rows (kVal writes, kUp reads), or null
   float* coef_pairs;          // [pairs] s_e r_e of each pair, applied in the combine
   __half* v_pairs;            // [pairs][D] W_down[e] a in fp16 (3 more significant bits than
                               // bf16); unscaled by s_e r_e, so |v| <= sqrt(d_e) max_j ||W_down[e][j]||_1
@@ -261,13 +268,13 @@ template <int MODE>
 __device__ __forceinline__ int tile_total(const Args& a) {
   if (MODE == kProj || MODE == kShared) return a.m_tiles * a.n_tiles_n;
   const int n = *a.n_row_tiles;
-  return MODE == kUp ? n : n * a.n_tiles_n;
+  return gathers<MODE>() ? n : n * a.n_tiles_n;
 }
 
 template <int MODE>
 __device__ __forceinline__ Tile tile_at(const Args& a, int idx) {
   Tile t{};
-  if (MODE == kUp) {
+  if (gathers<MODE>()) {
     const int4 q = a.tiles[idx];
     t.e = q.x;
     t.arow = q.y;
@@ -464,6 +471,35 @@ __device__ __forceinline__ void epilogue(const Args& a, const Tile& t, uint32_t 
         tmem_ld32(trow + c0 + 32 * h, v);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = silu_fast(v[j] * inv);
+        if (a.val_pairs && ok) {   // gated experts: times the value row (bf16, 64 B)
+          float vv[32];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            unpack16(__ldg(reinterpret_cast<const uint4*>(a.val_pairs + (size_t)pair * a.d_e + c0 + 32 * h) + q),
+                     *reinterpret_cast<float(*)[8]>(vv + 8 * q));
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= vv[j];
+        }
+        uint4 w[4];
+        pack_bf16x32(v, w);
+        if (full_warp) {
+          box_put_16(box, r, h, w);
+        } else if (ok) {
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) reinterpret_cast<uint4*>(dst + c0 + 32 * h)[qq] = w[qq];
+        }
+      }
+      if (full_warp) box_store(o, tmO, c0, row0);
+    }
+  } else if (MODE == kVal) {   // value rows, bf16, 64 columns per box
+    const int pair = t.arow + i;
+    bf16* dst = const_cast<bf16*>(a.val_pairs) + (size_t)pair * a.d_e;
+    for (int c0 = 0; c0 < a.d_e; c0 += 64) {
+      uint8_t* box = full_warp ? box_begin(o) : nullptr;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float v[32];
+        tmem_ld32(trow + c0 + 32 * h, v);
         uint4 w[4];
         pack_bf16x32(v, w);
         if (full_warp) {
@@ -541,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1 + (MODE == kUp ? kGatherThreads : 0));
+      mbar_init(&full[s], 1 + (gathers<MODE>() ? kGatherThreads : 0));
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -566,14 +602,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;               // per-stage bits, for the drain
-      const uint32_t bytes = kBBytes + (MODE == kUp ? 0u : kABytes);
+      const uint32_t bytes = kBBytes + (gathers<MODE>() ? 0u : kABytes);
       for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x) {
         const Tile t = tile_at<MODE>(a, idx);
         const CUtensorMap* mb = (MODE == kProj && t.bmap) ? &tmB2 : &tmB;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, a.err, a.wait_cycles)) break;
           mbar_expect_tx(&full[stage], bytes);
-          if (MODE != kUp) tma_2d(sm + stage * kABytes, &tmA, kb * kBK, t.arow, &full[stage]);
+          if (!gathers<MODE>()) tma_2d(sm + stage * kABytes, &tmA, kb * kBK, t.arow, &full[stage]);
           tma_2d(sm + kStages * kABytes + stage * kBBytes, mb, kb * kBK, t.brow, &full[stage]);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -592,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (MODE == kUp && warp >= kGatherWarp0) {
+  } else if (gathers<MODE>() && warp >= kGatherWarp0) {
     const int j = threadIdx.x - kGatherWarp0 * 32;       // 0..63
     const int c = j & 7, rsub = j >> 3;                  // 16-byte chunk, row within 8-row group
     int stage = 0;
@@ -629,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_wait_all();
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(kBM, MODE == kUp ? a.bn : kBN);
+      const uint32_t idesc = idesc_bf16(kBM, gathers<MODE>() ? a.bn : kBN);
       int stage = 0;
       uint32_t phase = 0;
       int lt = 0;
@@ -644,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             stop = true;
             break;
           }
-          if (MODE == kUp) fence_proxy_async_smem();   // cp.async data -> tensor core (async proxy)
+          if (gathers<MODE>()) fence_proxy_async_smem();   // cp.async data -> tensor core (async proxy)
           tc_fence_after();
           const uint32_t sA = base + stage * kABytes;
           const uint32_t sB = base + kStages * kABytes + stage * kBBytes;

@@ -266,12 +266,13 @@ __global__ void __launch_bounds__(kThreads) k_scatter(const uint8_t* __restrict_
 // publishes its partial sum of c^2 per pair.  After a cluster barrier every
 // CTA adds the 8 partials in rank order through distributed shared memory,
 // giving the RMS over all d_e features, and writes a = SiLU(c / rms) for its
-// rows to H[pair][d_e].
+// rows to H[pair][d_e] (times the value branch W_val[e] x_t for gated experts).
 
 struct UpArgs {
   const void* x;
   int D;
   const void* W_up;
+  const void* W_val;   // gated experts' value branch, or null
   int d_e;
   const float* u;
   const int* perm;
@@ -289,6 +290,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads) k_u
   const int RPC = a.d_e / kCluster;
   T* xs = reinterpret_cast<T*>(smem);
   float* gs = reinterpret_cast<float*>(smem + (size_t)TT * a.D * sizeof(T));   // [TT][RPC]
+  float* vs = gs + TT * RPC;                                                     // [TT][RPC] (gated)
   __shared__ float part[TT];
   __shared__ float rinv[TT];
   __shared__ int tok[TT];
@@ -311,6 +313,12 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads) k_u
       if (lane == 0)
         for (int tt = 0; tt < np; ++tt)
           gs[tt * RPC + jr] = acc[tt] - a.u[(size_t)tok[tt] * a.d_e + j0 + jr];
+      if (a.W_val) {   // gated: the value branch of the same row
+        const T* wv = reinterpret_cast<const T*>(a.W_val) + ((size_t)e * a.d_e + j0 + jr) * a.D;
+        dot_row_tokens<T, TT, false>(wv, xs, a.D, acc, dummy);
+        if (lane == 0)
+          for (int tt = 0; tt < np; ++tt) vs[tt * RPC + jr] = acc[tt];
+      }
     }
     __syncthreads();
     if (threadIdx.x < TT) {
@@ -328,7 +336,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads) k_u
     __syncthreads();
     for (int i = threadIdx.x; i < np * RPC; i += blockDim.x) {
       const int tt = i / RPC, j = i - tt * RPC;
-      a.H[(size_t)(p0 + tt) * a.d_e + j0 + j] = silu_f(gs[i] * rinv[tt]);
+      const float act = silu_f(gs[i] * rinv[tt]);
+      a.H[(size_t)(p0 + tt) * a.d_e + j0 + j] = a.W_val ? act * vs[i] : act;
     }
     cluster.sync();   // partial sums stay readable until every rank is done
   }

@@ -524,3 +524,70 @@ def test_workspace_size_covers_every_write(lib, shape, topk):
     lib.routing(G["x"], G, workspace=ws, topk=topk)
     torch.cuda.synchronize()
     assert bool((buf[n:] == 0xA5).all())
+
+
+# --------------------------------------------------------------------------
+# gated experts ("DECO (gated)"): a = NormSiLU(x W_up^T - u) * (x W_val^T)
+
+@pytest.mark.parametrize("shape,topk", [
+    (LayerShape(16, 2048, 64, 256, 1024, "bf16"), 0),   # decode kernel
+    (LayerShape(5, 512, 16, 256, 256, "bf16"), 0),      # decode kernel, ragged batch
+    (LayerShape(300, 320, 5, 192, 320, "bf16"), 0),     # tensor-core kernels, ragged tiles
+    (LayerShape(37, 256, 8, 128, 192, "f32"), 0),       # general kernels
+    (LayerShape(40, 256, 8, 512, 64, "bf16"), 0),       # tiled router, general expert kernels
+    (LayerShape(16, 512, 16, 256, 256, "bf16"), 3),     # gated with TopK routing
+])
+def test_gated_forward_parity(lib, shape, topk):
+    L = make_layer(shape, 91, gated=True, ratio=0.3)
+    G = to_gpu(L, lib)
+    out = lib.forward(G["x"], G, eps=shape.eps, topk=topk)
+    torch.cuda.synchronize()
+    L64 = to_oracle(L, shape.dtype)
+    x64 = O.to_f64(L["x"])
+    if topk == 0:
+        ref = O.layer_forward(x64, L64, shape.eps)
+    else:
+        _, act, r = O.topk_route(x64, L64["W_r"], L64["b_r"], topk)
+        ref = np.zeros((shape.T, shape.D))
+        for t in range(shape.T):
+            u = L64["W_bar_up"] @ x64[t]
+            y = O.shared_expert(x64[t], L64["W_s_up"], L64["W_s_down"])
+            for e in range(shape.E):
+                if act[t, e]:
+                    y = y + (L64["s"][e] * r[t, e]) * O.expert_output(
+                        x64[t], L64["W_up"][e], L64["W_down"][e], u, shape.eps, L64["W_val"][e])
+            ref[t] = y
+    check_close(out.double().cpu().numpy(), ref, shape.dtype, f"gated {shape} topk={topk}")
+    out2 = lib.forward(G["x"], G, eps=shape.eps, topk=topk)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+def test_gated_prefill_full_size_sampled(lib):
+    shape, L = case("edge_prefill_t4096")
+    L["W_val"] = make_layer(shape, 2, gated=True, with_x=False)["W_val"]
+    G = to_gpu(L, lib)
+    ws = lib.alloc_workspace(lib.layer_shape(G["x"], G))
+    n = ws.numel()
+    guard = torch.full((n + 65536,), 0xA5, dtype=torch.uint8, device="cuda")
+    out = lib.forward(G["x"], G, workspace=guard[:n], eps=shape.eps)
+    torch.cuda.synchronize()
+    assert bool((guard[n:] == 0xA5).all())
+    toks = [0, 1, 64, 1000, 2047, shape.T - 1]
+    ref = oracle_forward(O.to_f64(L["x"]), to_oracle(L, "bf16"), shape.eps, toks)
+    check_close(out.double().cpu().numpy()[toks], ref, "bf16", "gated prefill T=4096")
+
+
+def test_gated_requires_the_value_branch(lib):
+    shape = LayerShape(4, 256, 8, 64, 64, "bf16")
+    L = make_layer(shape, 92)
+    G = to_gpu(L, lib)
+    sh = lib.layer_shape(G["x"], G)
+    sh.gated = 1                                  # gated shape, no W_val pointer
+    w = lib._weights(G)
+    ws = lib.alloc_workspace(sh)
+    out = torch.empty_like(G["x"])
+    import ctypes
+    rc = lib._lib.deco_moe_forward(ctypes.byref(sh), G["x"].data_ptr(), ctypes.byref(w), out.data_ptr(),
+                                   ws.data_ptr(), ws.numel(), lib._stream(None))
+    assert rc == 1
