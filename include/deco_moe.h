@@ -153,10 +153,10 @@ deco_status_t deco_moe_workspace_size(const deco_moe_shape_t* shape, size_t* byt
  * 256-byte aligned, owned by the caller; its contents need no initialisation
  * and are overwritten.  Two calls that overlap on the GPU must not share one
  * workspace.  The kernels are chosen from the shape: bf16 batches of up to 16
- * tokens take the weight-streaming decode kernels (d_model a multiple of 256,
- * d_e <= 256), other bf16 batches with d_e <= 256 the tensor-core (tcgen05)
- * kernels, everything else the general CUDA-core kernels; all compute the
- * same layer.  The workspace of a tensor-core batch holds one fp16 row of
+ * tokens take the weight-streaming decode kernel (one cooperative launch with
+ * one CTA per SM; d_model a multiple of 256 up to 4096, d_e <= 256), other
+ * bf16 batches with d_e <= 256 the tensor-core (tcgen05) kernels, everything
+ * else the general CUDA-core kernels; all compute the same layer.  The workspace of a tensor-core batch holds one fp16 row of
  * d_model values per possible (token, expert) pair, T * E * d_model * 2 bytes. */
 deco_status_t deco_moe_forward(const deco_moe_shape_t* shape, const void* x,
                                const deco_moe_weights_t* w, void* out,
@@ -215,9 +215,11 @@ deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
  * deco_moe_forward.
  *  - Shapes whose deco_moe_workspace_size exceeds DECO_STATIC_SCRATCH_BYTES
  *    are rejected with DECO_ERR_WORKSPACE before anything is launched.  Decode
- *    batches fit: T = 16 needs about 18 MiB at d_model 2048 / 64 experts and
- *    about 52 MiB (82 % of the array) at d_model 4096 / 128 experts; 256
- *    experts at d_model 4096 do not fit and are refused.
+ *    batches fit: T = 16 needs about 13 MiB at d_model 2048 / 64 experts and
+ *    about 23 MiB at d_model 4096 / 128 experts (39 MiB gated); gated
+ *    experts with 256 experts at d_model 4096 (75 MiB) do not fit and are
+ *    refused.  Larger batches fit while their workspace, which on the
+ *    tensor-core path grows with T * E * d_model, stays within the array.
  *  - The first call on each device looks up the scratch array's device
  *    address (cudaGetSymbolAddress, a runtime call made with that device
  *    current) and keeps it for the life of the process; make that first call
