@@ -42,8 +42,9 @@ DECODE_TS = (1, 4, 16)
 METRIC = "MoE-layer tokens/s (decode)"
 # DRAM bytes (read + write) per launch of the decode kernel at T = 16 from an
 # ncu capture of the current kernel (None until one is taken; a kernel changed
-# since its capture has no entry)
-NCU_DRAM_BYTES = {}
+# since its capture has no entry): kd_layer, edge layer, T = 16, 139.95 MB read
+# + 5.51 MB written (profiles/kd_layer_edge_decode_t16.md)
+NCU_DRAM_BYTES = {("layer", 16): 145_460_224}
 
 
 def parse():
@@ -485,8 +486,9 @@ def main():
 def profile_only(args):
     """Eager forward passes of the edge layer at one batch size, for ncu:
     warmup forwards first, then `steps` more.  Kernels in launch order:
-    kd_layer (T <= 16); k_router, k_router_exact, k_tab_count, k_tab_scatter,
-    kp_gemm<0..3>, k_combine (T > 16).  --profile-dense: the dense FFN."""
+    kd_layer (T <= 16); k_router, k_router_exact, k_tab_count, k_tab_scan,
+    k_tab_scatter, kp_gemm<0..3>, k_combine (T > 16).  --profile-dense: the
+    dense FFN."""
     import torch
 
     import sparse_moe_ffn_relu_b200 as deco
