@@ -215,11 +215,11 @@ deco_status_t deco_moe_device_error(void* workspace, int* code, void* stream);
  * deco_moe_forward.
  *  - Shapes whose deco_moe_workspace_size exceeds DECO_STATIC_SCRATCH_BYTES
  *    are rejected with DECO_ERR_WORKSPACE before anything is launched.  Decode
- *    batches fit: T = 16 needs about 13 MiB at d_model 2048 / 64 experts and
- *    about 23 MiB at d_model 4096 / 128 experts (39 MiB gated); gated
- *    experts with 256 experts at d_model 4096 (75 MiB) do not fit and are
- *    refused.  Larger batches fit while their workspace, which on the
- *    tensor-core path grows with T * E * d_model, stays within the array.
+ *    batches fit: T = 16 needs about 7 MiB at d_model 2048 / 64 experts,
+ *    10 MiB at d_model 4096 / 128 experts (12 MiB gated) and 20 MiB with
+ *    256 gated experts at d_model 4096.  Larger batches fit while their
+ *    workspace, which on the tensor-core path grows with T * E * d_model,
+ *    stays within the array.
  *  - The first call on each device looks up the scratch array's device
  *    address (cudaGetSymbolAddress, a runtime call made with that device
  *    current) and keeps it for the life of the process; make that first call

@@ -27,7 +27,7 @@ struct Plan {
   // decode path (T <= 16): up-projection partials, shared hidden and NormSiLU
   // tiles, per-CTA down-projection partials (the inter-CTA counters follow
   // the error word)
-  size_t C16, C16v, HS, A16, Part, tmask;
+  size_t Pu, HS, A16, Part, tmask;
   // bf16, T > 16: ambiguous router pairs; prefill path: routed expert output
   // rows (one fp16 row per pair) and the shared expert's fp32 output
   size_t fb, blk, etot, v_pairs, coef, s_out, val_pairs;
@@ -102,8 +102,8 @@ Plan make_plan(const deco_moe_shape_t& s) {
     p.s_out = take(T * s.d_model * 4);
   }
   if (s.T <= dec::kMaxT) {         // decode path buffers (see decode_kernels.cuh)
-    p.C16 = take(8 * E * dec::kTok * s.d_e * 4);                       // [kp <= 8][E][16][d_e] fp32
-    if (s.gated) p.C16v = take(8 * E * dec::kTok * s.d_e * 4);         // the same for the value branch
+    const size_t runs = E * (s.gated ? 2 : 1) * ((s.d_e + dec::kDRows - 1) / dec::kDRows);
+    p.Pu = take((runs + std::max(p.sms, 1)) * dec::kTok * dec::kDRows * 4);   // phase-U pieces, fp32
     p.HS = take((size_t)dec::down_nsq(s.d_s) * dec::kTileBytes);       // [nsq] 16 KB tiles
     p.A16 = take(E * dec::kTileBytes);                                 // [E] 16 KB tiles
     p.Part = take((size_t)std::max(p.sms, 1) * 2 * dec::kTok * dec::kDRows * 4);   // [G][2][16][128]
@@ -418,7 +418,7 @@ void decode_buffers(dec::Args& a, unsigned char* ws, const Plan& p) {
   a.u = reinterpret_cast<float*>(ws + p.u);
   a.HS = reinterpret_cast<bf16*>(ws + p.HS);
   a.A = reinterpret_cast<bf16*>(ws + p.A16);
-  a.C = reinterpret_cast<float*>(ws + p.C16);
+  a.Pu = reinterpret_cast<float*>(ws + p.Pu);
   a.Part = reinterpret_cast<float*>(ws + p.Part);
   a.err = reinterpret_cast<int*>(ws + p.err);
   a.sync = reinterpret_cast<unsigned*>(ws + p.err + 16);
@@ -446,7 +446,6 @@ cudaError_t run_decode(const deco_moe_shape_t& s, const void* x, const deco_moe_
   a.out = static_cast<bf16*>(out);
   a.pre_routed = s.topk > 0;
   a.gated = s.gated;
-  a.Cv = s.gated ? reinterpret_cast<float*>(ws + p.C16v) : nullptr;
   decode_buffers(a, ws, p);
   // weight tiles of phases U and D: 128 rows x 64 columns
   CUtensorMap tmU, tmV, tmW, tmS;

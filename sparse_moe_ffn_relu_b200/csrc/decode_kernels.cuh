@@ -300,19 +300,13 @@ __host__ __device__ inline int tile_slots(int D) {
 // router CTAs of phase R: one router row each (E <= 64), else several
 __host__ __device__ inline int router_ctas(int E) { return E < 64 ? E : 64; }
 
-// K parts of phase U: the smallest power of two (<= 8) that gives every CTA
-// at least two units, while a part keeps >= 256 columns
-__host__ __device__ inline int up_kparts(int U, int d_e, int D, int G) {
-  const int units = U * ((d_e + kDRows - 1) / kDRows);
-  int kp = 1;
-  while (kp < 8 && D / (2 * kp) >= 256 && units * kp < 2 * G) kp *= 2;
-  return kp;
-}
 __host__ __device__ inline int down_nsq(int d_s) { return (d_s + kSq - 1) / kSq; }
 
 // the contiguous unit range [u0, u1) of CTA c among G (c * n < 2^31 for every
 // count of units or rows here: n <= 2^17, G <= kMaxSms)
 __host__ __device__ inline int range_lo(int c, int n, int G) { return c * n / G; }
+// the CTA whose range holds item i < n: the largest c with range_lo(c) <= i
+__host__ __device__ inline int range_owner(int i, int n, int G) { return ((i + 1) * G - 1) / n; }
 
 // ---------------------------------------------------------------------------
 
@@ -339,8 +333,8 @@ struct Args {
   bf16* HS;          // [nsq][16 tok][256 hi | 256 lo], chunk-swizzled rows: SiLU(x W_s_up^T)
   bf16* A;           // [E][16 tok][256 hi | 256 lo]: s_e r_e NormSiLU(x W_up[e]^T), 0 for
                      // tokens not using e
-  float* C;          // [kp <= 8][E][16 tok][d_e]: partial sums of x W_up[e]^T over K parts
-  float* Cv;         // the same for x W_val[e]^T (gated experts)
+  float* Pu;         // [E * nbr * nrb_up + G][16 tok][128]: phase-U pieces, CTA c's sum of
+                     // x W^T over its stages of run r in slot r + c
   float* Part;       // [G][2][16 tok][128]: a CTA's down-projection sum per row block
   unsigned* sync;    // inter-CTA counters (layout: SyncIdx); kd_layer clears them itself
   int* err;
@@ -561,6 +555,7 @@ __device__ __forceinline__ void route_rows(const Args& a, int c, int Cr, const u
       }
       const unsigned m = __ballot_sync(kFull, mine && on);
       if (lane == 0) a.tmask[e] = m;
+
     }
     consumer_sync();   // red is reused by the next row
   }
@@ -663,13 +658,18 @@ __global__ void __launch_bounds__(kThreads, 1) kd_router(const __grid_constant__
 // ---------------------------------------------------------------------------
 // The layer.
 
-// The schedule of phases U and D (every CTA takes a contiguous share of each
-// phase's units, in order).
+// The schedule of phases U and D.  Phase U is a sequence of stages: run r
+// (one block of 128 rows of W_up[e] or W_val[e]) is stages r * nkc ..
+// r * nkc + nkc - 1, 128 columns each, an expert's runs consecutive.  Every
+// CTA takes a contiguous share of the stages, which may begin or end inside a
+// run (shares differ by one stage at most); it writes one piece per run it
+// touches.  Phase D: every CTA takes a contiguous share of the units.
 struct Sched {
   int U;              // active experts (the union)
   int nbr;            // up-projection matrices per expert: W_up, and W_val when gated
-  int kp, Kp, nrb_up, nrb, nsq;
-  int NU;             // phase-U units
+  int nrb_up, nkc;    // runs per matrix, stages per run
+  int NS;             // phase-U stages
+  int nrb, nsq;
   int J, ND;          // phase-D units per row block, and in all
 };
 
@@ -677,28 +677,25 @@ __device__ __forceinline__ Sched make_sched(const Args& a, int U, int G) {
   Sched S;
   S.U = U;
   S.nrb_up = (a.d_e + kDRows - 1) / kDRows;
+  S.nkc = a.D / 128;
   S.nrb = a.D / kDRows;
   S.nsq = down_nsq(a.d_s);
   S.nbr = a.gated ? 2 : 1;
-  S.kp = up_kparts(U * S.nbr, a.d_e, a.D, G);
-  S.Kp = a.D / S.kp;
-  S.NU = U * S.nbr * S.nrb_up * S.kp;
+  S.NS = U * S.nbr * S.nrb_up * S.nkc;
   S.J = S.nsq + U;
   S.ND = S.nrb * S.J;
   return S;
 }
 
-// unit u of phase U: index of its expert in the union, the matrix (0 W_up,
-// 1 W_val), the block of 128 rows of it and the K part; an expert's units
-// are consecutive
-struct UUnit {
-  int ei, mat, rbu, p;
+// run r of phase U: index of its expert in the union, the matrix (0 W_up,
+// 1 W_val) and the block of 128 rows of it
+struct URun {
+  int ei, mat, rbu;
 };
-__device__ __forceinline__ UUnit up_unit(const Sched& S, int u) {
-  UUnit q;
-  q.p = u % S.kp;
-  q.rbu = (u / S.kp) % S.nrb_up;
-  const int m = u / (S.kp * S.nrb_up);
+__device__ __forceinline__ URun up_run(const Sched& S, int r) {
+  URun q;
+  q.rbu = r % S.nrb_up;
+  const int m = r / S.nrb_up;
   q.mat = m % S.nbr;
   q.ei = m / S.nbr;
   return q;
@@ -725,6 +722,52 @@ __device__ __forceinline__ DUnit down_unit(const Args& a, const uint8_t* ulist, 
   return d;
 }
 
+// The producer's walk over its stages: phase-U stages [sg, s1), then the
+// phase-D units [v, v1), unit v from column c0.  pwalk_get gives the tensor
+// map and coordinates of the current stage's first box (a second box, when
+// nb = 2, is 64 columns on); false once the walk is over.
+struct PWalk {
+  int sg, s1, v, v1, c0;
+};
+struct PStage {
+  const CUtensorMap* m;
+  int col, row, nb;
+};
+__device__ __forceinline__ bool pwalk_get(const Args& a, const Sched& S, const uint8_t* ulist, const PWalk& w,
+                                          const CUtensorMap* tmU, const CUtensorMap* tmV, const CUtensorMap* tmW,
+                                          const CUtensorMap* tmS, PStage& st) {
+  if (w.sg < w.s1) {
+    const int r = w.sg / S.nkc, kc = w.sg - r * S.nkc;
+    const URun q = up_run(S, r);
+    st.m = q.mat ? tmV : tmU;
+    st.col = kc * 128;
+    st.row = ulist[q.ei] * a.d_e + q.rbu * kDRows;
+    st.nb = 2;
+    return true;
+  }
+  if (w.v < w.v1) {
+    const DUnit d = down_unit(a, ulist, S, w.v);
+    const bool sh = d.e < 0;
+    st.m = sh ? tmS : tmW;
+    st.col = d.col0 + w.c0;
+    st.row = sh ? d.rb * kDRows : d.e * a.D + d.rb * kDRows;
+    st.nb = min(2, (d.K - w.c0) / 64);
+    return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void pwalk_next(const Args& a, const Sched& S, const uint8_t* ulist, PWalk& w) {
+  if (w.sg < w.s1) {
+    ++w.sg;
+  } else if (w.v < w.v1) {
+    w.c0 += 128;
+    if (w.c0 >= down_unit(a, ulist, S, w.v).K) {
+      w.c0 = 0;
+      ++w.v;
+    }
+  }
+}
+
 // The partials of row block rb in the fixed order of the combine: the CTAs
 // whose unit range meets rb, ascending (one warp: lane l tests CTAs l,
 // l + 32, ...).  Returns the count and fills src[i] = 2 c + (which of the
@@ -748,11 +791,53 @@ __device__ __forceinline__ int rb_sources(int rb, const Sched& S, int G, int* sr
   return n;
 }
 
-// NormSiLU tile of expert e (consumer threads): c = sum of the K parts of g
-// minus u, h = c / sqrt(mean c^2 + eps), a = s_e r_e SiLU(h) (times the value
-// branch for gated experts) as hi/lo rows; rows of tokens not using e are
-// zero.
-__device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
+__device__ __forceinline__ void add4(float4& a, const float4& b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+
+// Lane's 8 features of run r for token t: the pieces of the CTAs whose stage
+// shares meet the run, added in CTA order (up to 4 pieces' loads in flight).
+// The next such CTA owns the stage after the current one's share (CTAs with
+// an empty share, when there are fewer stages than CTAs, are skipped).
+__device__ __forceinline__ void run_sum(const Args& a, const Sched& S, int G, int r, int t, int row0, bool live,
+                                        float4& g0, float4& g1) {
+  g0 = make_float4(0.f, 0.f, 0.f, 0.f);
+  g1 = g0;
+  if (!live) return;
+  const int end = (r + 1) * S.nkc;   // the stage after the run
+  int cc = range_owner(r * S.nkc, S.NS, G);
+  while (cc >= 0) {
+    float4 v[4][2];
+    bool has[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      has[i] = cc >= 0;
+      if (has[i]) {
+        const float4* src = reinterpret_cast<const float4*>(a.Pu + ((size_t)(r + cc) * kTok + t) * kDRows + row0);
+        v[i][0] = __ldcg(src);
+        v[i][1] = __ldcg(src + 1);
+        const int nxt = range_lo(cc + 1, S.NS, G);
+        cc = nxt < end ? range_owner(nxt, S.NS, G) : -1;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (has[i]) {
+        add4(g0, v[i][0]);
+        add4(g1, v[i][1]);
+      }
+    }
+  }
+}
+
+// NormSiLU tile of expert e, the ei-th of the union (consumer threads): g =
+// x W_up[e]^T from its pieces, c = g - u, h = c / sqrt(mean c^2 + eps), a =
+// s_e r_e SiLU(h) (times x W_val[e]^T for gated experts) as hi/lo rows; rows
+// of tokens not using e are zero.
+__device__ void norm_silu_tile(const Args& a, const Sched& S, int G, int e, int ei, uint32_t m_e) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   bf16* tile = a.A + (size_t)e * kTileElems;
   for (int i = threadIdx.x; i < kTok * 64; i += kConsumerThreads) {   // 64 chunks of 16 B per row
@@ -761,68 +846,44 @@ __device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
   }
   const int n_e = __popc(m_e);
   const bool live = 8 * lane < a.d_e;   // lane l holds features 8 l .. 8 l + 7
+  const int rbu = (8 * lane) / kDRows, row0 = (8 * lane) % kDRows;
+  const int r_up = (ei * S.nbr) * S.nrb_up + rbu;
   for (int slot = warp; slot < n_e; slot += kConsumerWarps) {
     uint32_t m = m_e;
     for (int i = 0; i < slot; ++i) m &= m - 1;
     const int t = __ffs(m) - 1;
-    // every load of the token's row is issued before the first is used
     const float rte = __ldcg(a.r + (size_t)t * a.E + e);
     const float se = __ldg(a.s + e);
-    float4 gp[8][2], uq[2];
-#pragma unroll
-    for (int pp = 0; pp < 8; ++pp) {
-      const float4* src = reinterpret_cast<const float4*>(a.C + (((size_t)pp * a.E + e) * kTok + t) * a.d_e) + 2 * lane;
-      gp[pp][0] = (pp < kp && live) ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
-      gp[pp][1] = (pp < kp && live) ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    float4 uq[2];
     const float4* usrc = reinterpret_cast<const float4*>(a.u + (size_t)t * a.d_e) + 2 * lane;
     uq[0] = live ? __ldcg(usrc) : make_float4(0.f, 0.f, 0.f, 0.f);
     uq[1] = live ? __ldcg(usrc + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 g[2];
+    run_sum(a, S, G, r_up, t, row0, live, g[0], g[1]);
     float cv[8];
-    float ss = 0.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      float g[4] = {0.f, 0.f, 0.f, 0.f};   // the K parts in order (absent parts add an exact 0)
-#pragma unroll
-      for (int pp = 0; pp < 8; ++pp) {
-        g[0] += gp[pp][h].x;
-        g[1] += gp[pp][h].y;
-        g[2] += gp[pp][h].z;
-        g[3] += gp[pp][h].w;
-      }
-      cv[4 * h + 0] = g[0] - uq[h].x;
-      cv[4 * h + 1] = g[1] - uq[h].y;
-      cv[4 * h + 2] = g[2] - uq[h].z;
-      cv[4 * h + 3] = g[3] - uq[h].w;
+      cv[4 * h + 0] = g[h].x - uq[h].x;
+      cv[4 * h + 1] = g[h].y - uq[h].y;
+      cv[4 * h + 2] = g[h].z - uq[h].z;
+      cv[4 * h + 3] = g[h].w - uq[h].w;
     }
+    float ss = 0.f;
 #pragma unroll
     for (int q = 0; q < 8; ++q) ss = fmaf(cv[q], cv[q], ss);
-    // gated experts: the value branch, its K parts added in order
+    // gated experts: the value branch
     float val[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) val[q] = 1.f;
     if (a.gated) {
-      float4 vp[8][2];
-#pragma unroll
-      for (int pp = 0; pp < 8; ++pp) {
-        const float4* src = reinterpret_cast<const float4*>(a.Cv + (((size_t)pp * a.E + e) * kTok + t) * a.d_e) + 2 * lane;
-        vp[pp][0] = (pp < kp && live) ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
-        vp[pp][1] = (pp < kp && live) ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      float4 vg[2];
+      run_sum(a, S, G, r_up + S.nrb_up, t, row0, live, vg[0], vg[1]);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        float g[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int pp = 0; pp < 8; ++pp) {
-          g[0] += vp[pp][h].x;
-          g[1] += vp[pp][h].y;
-          g[2] += vp[pp][h].z;
-          g[3] += vp[pp][h].w;
-        }
-        val[4 * h + 0] = g[0];
-        val[4 * h + 1] = g[1];
-        val[4 * h + 2] = g[2];
-        val[4 * h + 3] = g[3];
+        val[4 * h + 0] = vg[h].x;
+        val[4 * h + 1] = vg[h].y;
+        val[4 * h + 2] = vg[h].z;
+        val[4 * h + 3] = vg[h].w;
       }
     }
     ss = warp_sum(ss);
@@ -850,12 +911,6 @@ __device__ void norm_silu_tile(const Args& a, int e, uint32_t m_e, int kp) {
 // out rows of row block rb: the sources' partials in CTA order (+ x).  A
 // thread owns output float4s o and o + 256 (T * 32 of them); up to 8
 // sources' loads for both are in flight before they are added in order.
-__device__ __forceinline__ void add4(float4& a, const float4& b) {
-  a.x += b.x;
-  a.y += b.y;
-  a.z += b.z;
-  a.w += b.w;
-}
 
 __device__ void combine_rb(const Args& a, int rb, const int* src, int n) {
   constexpr int kQ = kDRows / 4;   // float4s per token row of a block
@@ -1021,43 +1076,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int U = s_U;
     {
       const Sched S = make_sched(a, U, G);
-      // phase U: W_up boxes
-      {
-        const int u0 = range_lo(c, S.NU, G), u1 = range_lo(c + 1, S.NU, G);
-        for (int u = u0; u < u1 && ok; ++u) {
-          const UUnit q = up_unit(S, u);
-          const int row = ulist[q.ei] * a.d_e + q.rbu * kDRows;
-          const CUtensorMap* mu = q.mat ? &tmV : &tmU;
-          for (int c0 = 0; c0 < S.Kp; c0 += 128) {
-            int s;
-            if (!(ok = next_stage(s))) break;
-            const int nb = min(2, (S.Kp - c0) / 64);
-            mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
-            for (int b = 0; b < nb; ++b)
-              tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, mu, q.p * S.Kp + c0 + 64 * b,
-                     row, &ctl.full[s], pol);
-            ++k;
-          }
-        }
-      }
-      // phase D: W_s_down / W_down boxes
-      {
-        const int v0 = range_lo(c, S.ND, G), v1 = range_lo(c + 1, S.ND, G);
-        for (int v = v0; v < v1 && ok; ++v) {
-          const DUnit d = down_unit(a, ulist, S, v);
-          const bool sh = d.e < 0;
-          const int row = sh ? d.rb * kDRows : d.e * a.D + d.rb * kDRows;
-          for (int c0 = 0; c0 < d.K; c0 += 128) {
-            int s;
-            if (!(ok = next_stage(s))) break;
-            const int nb = min(2, (d.K - c0) / 64);
-            mbar_expect_tx(&ctl.full[s], (uint32_t)nb * kBoxBytes);
-            for (int b = 0; b < nb; ++b)
-              tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, sh ? &tmS : &tmW,
-                     d.col0 + c0 + 64 * b, row, &ctl.full[s], pol);
-            ++k;
-          }
-        }
+      // phases U and D: W_up (W_val) boxes, then W_s_down / W_down boxes,
+      // one or two per stage
+      PWalk w{range_lo(c, S.NS, G), range_lo(c + 1, S.NS, G), range_lo(c, S.ND, G), range_lo(c + 1, S.ND, G), 0};
+      PStage ps;
+      while (ok && pwalk_get(a, S, ulist, w, &tmU, &tmV, &tmW, &tmS, ps)) {
+        int s;
+        if (!(ok = next_stage(s))) break;
+        mbar_expect_tx(&ctl.full[s], (uint32_t)ps.nb * kBoxBytes);
+        for (int b = 0; b < ps.nb; ++b)
+          tma_2d(ctl.stage + (size_t)s * ctl.stage_bytes + b * kBoxBytes, ps.m, ps.col + 64 * b, ps.row,
+                 &ctl.full[s], pol);
+        pwalk_next(a, S, ulist, w);
+        ++k;
       }
       *ctl.k_issued = k;
       mbar_arrive(ctl.pbar);
@@ -1188,36 +1219,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntiles = (a.T + 7) / 8;
 
   // ---- phase U ----
-  const int kp = S.kp, Kp = S.Kp, nrb_up = S.nrb_up;
   bool pre_seen = false;   // thread 0: phase R is complete everywhere (u is readable)
   {
-    const int u0 = range_lo(c, S.NU, G), u1 = range_lo(c + 1, S.NU, G);
-    int n_here = 0;          // this CTA's units of the current expert
-    for (int u = u0; u < u1; ++u) {
-      const UUnit q = up_unit(S, u);
-      const int p = q.p, rbu = q.rbu, e = clist[q.ei];
+    const int s0 = range_lo(c, S.NS, G), s1 = range_lo(c + 1, S.NS, G);
+    const int per_e = S.nbr * S.nrb_up * S.nkc;   // stages of one expert
+    int n_here = 0;                                 // this CTA's stages of the current expert
+    float acc[2][4] = {};
+    for (int sg = s0; sg < s1; ++sg) {
+      const int r = sg / S.nkc, kc = sg - r * S.nkc;
+      const URun q = up_run(S, r);
+      const int e = clist[q.ei];
       ++n_here;
-      float acc[2][4] = {};
-      for (int c0 = 0; c0 < Kp; c0 += 128) {
+      {
         const int s = k % ctl.nstages;
         const bool w = wait_full();
         ok = ok && w;
-        const int nb = min(2, (Kp - c0) / 64);
         if (ok) {
           const uint32_t st = smem_u32(ctl.stage + (size_t)s * ctl.stage_bytes);
-          for (int b = 0; b < nb; ++b) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
             const uint32_t box = st + b * kBoxBytes;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               uint32_t a0, a1, a2, a3;
               ldsm_x4(swz(box, 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * ks + (lane >> 4)), a0, a1, a2,
                       a3);
-              const int kc = (p * Kp + c0 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
+              const int kch = (kc * 128 + 64 * b) / 8 + 2 * ks + ((lane >> 3) & 1);
 #pragma unroll
               for (int nt = 0; nt < 2; ++nt) {
                 if (nt < ntiles) {
                   uint32_t b0, b1;
-                  ldsm_x2(x_u32 + (uint32_t)(8 * nt + (lane & 7)) * pitch + (uint32_t)kc * 16u, b0, b1);
+                  ldsm_x2(x_u32 + (uint32_t)(8 * nt + (lane & 7)) * pitch + (uint32_t)kch * 16u, b0, b1);
                   mma16816(acc[nt], a0, a1, a2, a3, b0, b1);
                 }
               }
@@ -1227,29 +1259,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         release(s);
         ++k;
       }
+      // the end of a run (or of the CTA's share): its piece, slot r + c
       // acc[nt][i]: row 16 warp + lane/4 + 8 (i >> 1), token 8 nt + 2 (lane & 3) + (i & 1)
-      if (ok) {
-        const int j0 = rbu * kDRows + 16 * warp + (lane >> 2);
+      if (kc == S.nkc - 1 || sg + 1 == s1) {
+        if (ok) {
+          float* dst = a.Pu + (size_t)(r + c) * kTok * kDRows;
+          const int j0 = 16 * warp + (lane >> 2);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+          for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int t = 8 * nt + 2 * (lane & 3) + (i & 1);
-            const int j = j0 + 8 * (i >> 1);
-            if (t < a.T && j < a.d_e) (q.mat ? a.Cv : a.C)[(((size_t)p * a.E + e) * kTok + t) * a.d_e + j] = acc[nt][i];
+            for (int i = 0; i < 4; ++i) {
+              const int t = 8 * nt + 2 * (lane & 3) + (i & 1);
+              if (t < a.T) dst[(size_t)t * kDRows + j0 + 8 * (i >> 1)] = acc[nt][i];
+            }
           }
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
       }
-      // after the CTA's last unit of expert e: one count of its units; the
-      // CTA that completes e's units computes its NormSiLU tile
-      const bool e_ends = u + 1 == u1 || up_unit(S, u + 1).ei != q.ei;
+      // after the CTA's last stage of expert e: one count of its stages; the
+      // CTA that completes e's stages computes its NormSiLU tile
+      const bool e_ends = sg + 1 == s1 || up_run(S, (sg + 1) / S.nkc).ei != q.ei;
       if (e_ends) {
-        consumer_sync();   // every warp's g partials precede the release
+        consumer_sync();   // every warp's pieces precede the release
         if (threadIdx.x == 0) {
           int last = 0;
           if (ok) {
             const unsigned old = atom_add_acq_rel(sync + si.g_cnt + e, (unsigned)n_here);
-            last = old + (unsigned)n_here == (unsigned)(S.nbr * nrb_up * kp);
+            last = old + (unsigned)n_here == (unsigned)per_e;
             // u comes from phase R
             if (last && !pre_seen)
               last = pre_seen = spin_until(sync + si.pre_done, (unsigned)Gp, a.wait_cycles, ctl.abort_flag, a.err);
@@ -1259,7 +1298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         consumer_sync();
         if (ctl.bcast[0]) {
-          norm_silu_tile(a, e, cmask[e], kp);
+          norm_silu_tile(a, S, G, e, q.ei, cmask[e]);
           consumer_sync();
           if (threadIdx.x == 0) st_release(sync + si.a_ready + e, 1u);
         }
