@@ -183,6 +183,7 @@ inline void prof_mark(int idx, cudaStream_t st) {
 // dec::kMaxSms SMs whose router CTAs leave room for the other phase-R rows.
 bool decode_grid_ok(int D, int E, int sms) {
   if (D % 256 || D > 4096 || sms > dec::kMaxSms) return false;
+  if (D / dec::kDRows > sms) return false;   // a CTA's share of phase-D units spans <= 2 row blocks
   if (dec::router_ctas(E) + 16 > sms) return false;
   return dec::layer_smem(D).nstages >= 2;
 }

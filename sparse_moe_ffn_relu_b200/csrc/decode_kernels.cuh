@@ -971,7 +971,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_U;
   __shared__ uint16_t cmask[256];   // the consumer warps' own copy
   __shared__ uint8_t clist[256];
-  __shared__ int s_src[kMaxSms];
+  __shared__ int s_src[2 * kMaxSms];   // the sources of the (at most two) row blocks of a share
+  __shared__ int s_nsrc[2];
+  __shared__ int s_done[32];            // (index in the union << 16) | stages, per expert of a share
   const int G = gridDim.x, c = blockIdx.x;
   const int Cr = (a.E > 0 && !a.pre_routed) ? router_ctas(a.E) : 0;
   const bool router_cta = c < Cr;
@@ -1219,11 +1221,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntiles = (a.T + 7) / 8;
 
   // ---- phase U ----
-  bool pre_seen = false;   // thread 0: phase R is complete everywhere (u is readable)
   {
     const int s0 = range_lo(c, S.NS, G), s1 = range_lo(c + 1, S.NS, G);
     const int per_e = S.nbr * S.nrb_up * S.nkc;   // stages of one expert
     int n_here = 0;                                 // this CTA's stages of the current expert
+    int n_done = 0;                                 // experts this share touched (s_done)
     float acc[2][4] = {};
     for (int sg = s0; sg < s1; ++sg) {
       const int r = sg / S.nkc, kc = sg - r * S.nkc;
@@ -1279,33 +1281,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
       }
-      // after the CTA's last stage of expert e: one count of its stages; the
-      // CTA that completes e's stages computes its NormSiLU tile
+      // after the share's last stage of expert e: note its count of stages
+      // (counted at the end of the share, so the stream never waits on it)
       const bool e_ends = sg + 1 == s1 || up_run(S, (sg + 1) / S.nkc).ei != q.ei;
       if (e_ends) {
-        consumer_sync();   // every warp's pieces precede the release
-        if (threadIdx.x == 0) {
-          int last = 0;
-          if (ok) {
-            const unsigned old = atom_add_acq_rel(sync + si.g_cnt + e, (unsigned)n_here);
-            last = old + (unsigned)n_here == (unsigned)per_e;
-            // u comes from phase R
-            if (last && !pre_seen)
-              last = pre_seen = spin_until(sync + si.pre_done, (unsigned)Gp, a.wait_cycles, ctl.abort_flag, a.err);
-          }
-          if (!pre_seen && ok) pre_seen = ld_acquire(sync + si.pre_done) >= (unsigned)Gp;
-          ctl.bcast[0] = last;
-        }
-        consumer_sync();
-        if (ctl.bcast[0]) {
-          norm_silu_tile(a, S, G, e, q.ei, cmask[e]);
-          consumer_sync();
-          if (threadIdx.x == 0) st_release(sync + si.a_ready + e, 1u);
-        }
+        if (threadIdx.x == 0) s_done[n_done] = (q.ei << 16) | n_here;
+        ++n_done;
         n_here = 0;
-        ok = __all_sync(kFull, ok && !*ctl.abort_flag);
       }
     }
+    // the end of the share: one count per expert it touched (a lane each);
+    // the CTA that completes an expert's stages computes its NormSiLU tile
+    consumer_sync();   // every warp's pieces precede the counts, which release them
+    if (warp == 0) {
+      bool last = false;
+      if (ok && lane < n_done) {
+        const int ei = s_done[lane] >> 16, n = s_done[lane] & 0xffff;
+        const unsigned old = atom_add_acq_rel(sync + si.g_cnt + clist[ei], (unsigned)n);
+        last = old + (unsigned)n == (unsigned)per_e;
+      }
+      unsigned lm = __ballot_sync(kFull, last);
+      if (lm) {   // u comes from phase R
+        int pre = 0;
+        if (lane == 0) pre = spin_until(sync + si.pre_done, (unsigned)Gp, a.wait_cycles, ctl.abort_flag, a.err);
+        if (!__shfl_sync(kFull, pre, 0)) lm = 0;
+      }
+      if (lane == 0) ctl.bcast[0] = (int)lm;
+    }
+    consumer_sync();
+    for (unsigned lm = (unsigned)ctl.bcast[0]; lm; lm &= lm - 1) {
+      const int ei = s_done[__ffs(lm) - 1] >> 16, e = clist[ei];
+      norm_silu_tile(a, S, G, e, ei, cmask[e]);
+      consumer_sync();
+      if (threadIdx.x == 0) st_release(sync + si.a_ready + e, 1u);
+    }
+    ok = __all_sync(kFull, ok && !*ctl.abort_flag);
   }
 
   // ---- phase D ----
@@ -1316,6 +1326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     const int nslots = tile_slots(a.D);
     int cur_rb = -1, slot = -1;
+    int rb0 = -1, n_rb = 0;   // the share's row blocks: rb0, rb0 + 1
     float acc[2][4] = {};
     auto flush = [&]() {      // this CTA's partial of row block cur_rb
       if (ok) {
@@ -1329,22 +1340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (t < a.T) dst[(size_t)t * kDRows + r0 + 8 * (qq >> 1)] = acc[nt][qq];
           }
       }
-      consumer_sync();
-      if (warp == 0) {
-        int last = 0;
-        if (ok) {
-          const int n = rb_sources(cur_rb, S, G, s_src);
-          if (lane == 0) {
-            const unsigned old = atom_add_acq_rel(sync + si.rb_cnt + cur_rb, 1u);   // releases the partial
-            last = old + 1 == (unsigned)n ? n : 0;
-          }
-        }
-        if (lane == 0) ctl.bcast[0] = last;
-      }
-      consumer_sync();
-      const int n = ctl.bcast[0];
-      if (n) combine_rb(a, cur_rb, s_src, n);
-      consumer_sync();   // s_src is rewritten by the next flush
+      if (n_rb == 0) rb0 = cur_rb;
+      ++n_rb;
     };
     {
       const int v0 = range_lo(c, S.ND, G), v1 = range_lo(c + 1, S.ND, G);
@@ -1402,6 +1399,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&ctl.tempty[ts]);   // this warp is done with the tile
       }
       if (cur_rb >= 0) flush();
+    }
+    // the end of the share: one count per row block it touched (counted
+    // here, so the stream never waits on it); the CTA that completes a row
+    // block's partials combines them
+    consumer_sync();   // every warp's partials precede the counts, which release them
+    if (warp == 0) {
+      const int n0 = n_rb > 0 ? rb_sources(rb0, S, G, s_src) : 0;
+      const int n1 = n_rb > 1 ? rb_sources(rb0 + 1, S, G, s_src + kMaxSms) : 0;
+      bool last = false;
+      if (ok && lane < n_rb) {
+        const int nl = lane ? n1 : n0;
+        s_nsrc[lane] = nl;
+        last = atom_add_acq_rel(sync + si.rb_cnt + rb0 + lane, 1u) + 1u == (unsigned)nl;
+      }
+      const unsigned lm = __ballot_sync(kFull, last);
+      if (lane == 0) ctl.bcast[0] = (int)lm;
+    }
+    consumer_sync();
+    for (unsigned lm = (unsigned)ctl.bcast[0]; lm; lm &= lm - 1) {
+      const int i = __ffs(lm) - 1;
+      combine_rb(a, rb0 + i, s_src + i * kMaxSms, s_nsrc[i]);
     }
   }
 
