@@ -42,9 +42,8 @@ DECODE_TS = (1, 4, 16)
 METRIC = "MoE-layer tokens/s (decode)"
 # DRAM bytes (read + write) per launch of the decode kernel at T = 16 from an
 # ncu capture of the current kernel (None until one is taken; a kernel changed
-# since its capture has no entry): kd_layer, edge layer, T = 16, 139.95 MB read
-# + 5.51 MB written (profiles/kd_layer_edge_decode_t16.md)
-NCU_DRAM_BYTES = {("layer", 16): 145_460_224}
+# since its capture has no entry)
+NCU_DRAM_BYTES = {}
 
 
 def parse():

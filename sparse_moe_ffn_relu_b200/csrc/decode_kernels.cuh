@@ -11,19 +11,25 @@
 // of kernel boundaries:
 //
 //   phase R  CTAs [0, Cr): the router rows W_r (exact activation decisions on
-//            CUDA cores, see common.cuh) -> r, active.  The other CTAs: the
-//            rows of [W_bar_up ; W_s_up] -> u = x W_bar_up^T and the shared
-//            hidden SiLU(x W_s_up^T), kept as bf16 hi/lo tiles.
-//   phase U  after the router: the union of the batch's active experts; units
-//            (expert, 128 rows of W_up[e], K part) -> fp32 partial sums of
-//            g = x W_up[e]^T.  The CTA that completes an expert's last unit
-//            computes its NormSiLU for every token using it (subtract u, RMS
-//            over d_e, SiLU, times s_e r_e) as a bf16 hi/lo tile.
+//            CUDA cores, see common.cuh) -> r, active, and per expert the mask
+//            of tokens using it.  The other CTAs: the rows of [W_bar_up ;
+//            W_s_up] -> u = x W_bar_up^T and the shared hidden
+//            SiLU(x W_s_up^T), kept as bf16 hi/lo tiles.
+//   phase U  once every router CTA is done: the union of the batch's active
+//            experts (built by each CTA's producer warp for all its warps).  Its W_up[e] rows are a sequence of 128-column stages
+//            (run by run, a run being 128 rows of one expert's matrix), and
+//            every CTA takes a contiguous share of it, writing one fp32 piece
+//            of g = x W_up[e]^T per run it touches.  At the end of its share
+//            a CTA counts its stages of each expert; the CTA that completes an
+//            expert computes its NormSiLU for every token using it (the
+//            pieces added in CTA order, subtract u, RMS over d_e, SiLU, times
+//            s_e r_e) as a bf16 hi/lo tile.
 //   phase D  units (128 output rows, then one K part of W_s_down or one active
 //            expert's W_down[e] in ascending order); a CTA adds its
 //            consecutive units of one row block in its tensor-core
-//            accumulators and writes one fp32 partial per row block.  The CTA
-//            that completes a row block adds its partials in CTA order (+ the
+//            accumulators and writes one fp32 partial per row block (at most
+//            two).  At the end of its share it counts them; the CTA that
+//            completes a row block adds its partials in CTA order (+ the
 //            residual) and writes the output rows: a fixed order, so the
 //            result is bitwise reproducible.
 //
@@ -341,8 +347,9 @@ struct Args {
   bf16* out;
 };
 
-// counters: routed CTAs done, phase-R rows done, up units done per expert,
-// NormSiLU tile ready per expert, CTAs done per output row block
+// counters: router CTAs done, CTAs done with the other phase-R rows, up
+// stages done per expert, NormSiLU tile ready per expert, CTAs done per
+// output row block
 struct SyncIdx {
   int route_done, pre_done, g_cnt, a_ready, rb_cnt, total;
 };
@@ -909,8 +916,10 @@ __device__ void norm_silu_tile(const Args& a, const Sched& S, int G, int e, int 
 }
 
 // out rows of row block rb: the sources' partials in CTA order (+ x).  A
-// thread owns output float4s o and o + 256 (T * 32 of them); up to 8
-// sources' loads for both are in flight before they are added in order.
+// thread owns output float4s o and o + 256 (T * 32 of them); up to
+// kCombineBatch sources' loads for both are in flight before they are added
+// in order (a row block has about ten sources).
+constexpr int kCombineBatch = 12;
 
 __device__ void combine_rb(const Args& a, int rb, const int* src, int n) {
   constexpr int kQ = kDRows / 4;   // float4s per token row of a block
@@ -921,10 +930,10 @@ __device__ void combine_rb(const Args& a, int rb, const int* src, int n) {
     const int t0 = o0 / kQ, q0 = o0 - t0 * kQ;
     const int t1 = two ? o1 / kQ : t0, q1 = two ? o1 - t1 * kQ : q0;
     float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-    for (int i = 0; i < n; i += 8) {
-      float4 v0[8], v1[8];
+    for (int i = 0; i < n; i += kCombineBatch) {
+      float4 v0[kCombineBatch], v1[kCombineBatch];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < kCombineBatch; ++k) {
         if (i + k < n) {
           const float* P = a.Part + (size_t)src[i + k] * kTok * kDRows;
           v0[k] = __ldcg(reinterpret_cast<const float4*>(P + (size_t)t0 * kDRows) + q0);
@@ -932,7 +941,7 @@ __device__ void combine_rb(const Args& a, int rb, const int* src, int n) {
         }
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < kCombineBatch; ++k) {
         if (i + k < n) {
           add4(acc0, v0[k]);
           add4(acc1, v1[k]);
@@ -966,11 +975,9 @@ __global__ void __launch_bounds__(kThreads, 1)
              const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ unsigned long long limbs[kLimbs];
-  __shared__ uint16_t emask[256];   // the producer warp's union: token masks, active experts
-  __shared__ uint8_t ulist[256];
+  __shared__ uint16_t emask[256];   // the union, built by the producer warp: token masks,
+  __shared__ uint8_t ulist[256];    // active experts and their count (then read-only)
   __shared__ int s_U;
-  __shared__ uint16_t cmask[256];   // the consumer warps' own copy
-  __shared__ uint8_t clist[256];
   __shared__ int s_src[2 * kMaxSms];   // the sources of the (at most two) row blocks of a share
   __shared__ int s_nsrc[2];
   __shared__ int s_done[32];            // (index in the union << 16) | stages, per expert of a share
@@ -1041,25 +1048,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++k;
       }
     }
-    if (lane == 0) {
-      // the union of active experts needs every router row
-      if (ok) ok = spin_until(sync + si.route_done, (unsigned)Cr, a.wait_cycles, ctl.abort_flag, a.err);
-    }
+    // the union of active experts, for every warp of the CTA (published
+    // through ubar): the router rows' token masks, once every router CTA is
+    // done (one thread per CTA waits on the count)
+    if (lane == 0 && ok && !a.pre_routed)
+      ok = spin_until(sync + si.route_done, (unsigned)Cr, a.wait_cycles, ctl.abort_flag, a.err);
     ok = __shfl_sync(kFull, ok, 0);
     if (ok) {
-      ld_acquire(sync + si.route_done);   // each lane acquires the router CTAs' writes itself
+      if (!a.pre_routed) ld_acquire(sync + si.route_done);   // each lane acquires the router CTAs' writes
       for (int e = lane; e < a.E; e += 32) {
         uint32_t m = 0;
         if (a.pre_routed) {   // decisions from earlier kernels: scan act
 #pragma unroll
           for (int t = 0; t < kTok; ++t)
             if (t < a.T && __ldcg(a.act + (size_t)t * a.E + e)) m |= 1u << t;
-        } else {              // the router CTAs' per-expert token masks
+        } else {
           m = __ldcg(a.tmask + e);
         }
         emask[e] = (uint16_t)m;
       }
-      __syncwarp();
+    }
+    __syncwarp();
+    if (ok) {
       int n = 0;
       for (int base = 0; base < a.E; base += 32) {
         const int e = base + lane;
@@ -1073,7 +1083,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_U = 0;
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(ctl.ubar);   // the loader warp reads the union (or sees the abort)
+    if (lane == 0) mbar_arrive(ctl.ubar);   // the other warps read the union (or see the abort)
     if (lane != 0) return;
     const int U = s_U;
     {
@@ -1183,42 +1193,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0)   // releases every consumer thread's phase-R writes (they precede the barrier)
     atom_add_acq_rel(sync + (router_cta ? si.route_done : si.pre_done), 1u);
 
-  // ---- the union of active experts (the producer builds its own copy) ----
-  if (threadIdx.x == 0)
-    ctl.bcast[0] = ok && spin_until(sync + si.route_done, (unsigned)Cr, a.wait_cycles, ctl.abort_flag, a.err);
-  consumer_sync();
-  ok = ok && ctl.bcast[0];
-  if (ok) {
-    for (int e = threadIdx.x; e < a.E; e += kConsumerThreads) {
-      uint32_t m = 0;
-      if (a.pre_routed) {   // decisions from earlier kernels: scan act
-#pragma unroll
-        for (int t = 0; t < kTok; ++t)
-          if (t < a.T && __ldcg(a.act + (size_t)t * a.E + e)) m |= 1u << t;
-      } else {              // the router CTAs' per-expert token masks
-        m = __ldcg(a.tmask + e);
-      }
-      cmask[e] = (uint16_t)m;
-    }
-  }
-  consumer_sync();
-  if (warp == 0) {
-    int n = 0;
-    if (ok) {
-      for (int base = 0; base < a.E; base += 32) {
-        const int e = base + lane;
-        const bool f = e < a.E && cmask[e] != 0;
-        const unsigned bal = __ballot_sync(kFull, f);
-        if (f) clist[n + __popc(bal & ((1u << lane) - 1u))] = (uint8_t)e;
-        n += __popc(bal);
-      }
-    }
-    if (lane == 0) ctl.bcast[3] = n;
-  }
-  consumer_sync();
-  const int U = ctl.bcast[3];
+  // ---- the union of active experts, from the producer warp ----
+  ok = __all_sync(kFull, ok && mbar_wait(ctl.ubar, 0, ctl.abort_flag, a.err, a.wait_cycles));
+  const int U = ok ? s_U : 0;
   const Sched S = make_sched(a, U, G);
   const int ntiles = (a.T + 7) / 8;
+  // this CTA's phase-D row blocks (at most two) and the sources of their
+  // partials, found now rather than at the end of the kernel
+  const int dv0 = range_lo(c, S.ND, G), dv1 = range_lo(c + 1, S.ND, G);
+  const int rb0 = dv0 < dv1 ? dv0 / S.J : 0;
+  const int n_rb = dv0 < dv1 ? (dv1 - 1) / S.J - rb0 + 1 : 0;
+  if (warp == 0) {
+    const int n0 = n_rb > 0 ? rb_sources(rb0, S, G, s_src) : 0;
+    const int n1 = n_rb > 1 ? rb_sources(rb0 + 1, S, G, s_src + kMaxSms) : 0;
+    if (lane == 0) {
+      s_nsrc[0] = n0;
+      s_nsrc[1] = n1;
+    }
+  }
 
   // ---- phase U ----
   {
@@ -1230,7 +1222,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int sg = s0; sg < s1; ++sg) {
       const int r = sg / S.nkc, kc = sg - r * S.nkc;
       const URun q = up_run(S, r);
-      const int e = clist[q.ei];
       ++n_here;
       {
         const int s = k % ctl.nstages;
@@ -1297,7 +1288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool last = false;
       if (ok && lane < n_done) {
         const int ei = s_done[lane] >> 16, n = s_done[lane] & 0xffff;
-        const unsigned old = atom_add_acq_rel(sync + si.g_cnt + clist[ei], (unsigned)n);
+        const unsigned old = atom_add_acq_rel(sync + si.g_cnt + ulist[ei], (unsigned)n);
         last = old + (unsigned)n == (unsigned)per_e;
       }
       unsigned lm = __ballot_sync(kFull, last);
@@ -1310,8 +1301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     consumer_sync();
     for (unsigned lm = (unsigned)ctl.bcast[0]; lm; lm &= lm - 1) {
-      const int ei = s_done[__ffs(lm) - 1] >> 16, e = clist[ei];
-      norm_silu_tile(a, S, G, e, ei, cmask[e]);
+      const int ei = s_done[__ffs(lm) - 1] >> 16, e = ulist[ei];
+      norm_silu_tile(a, S, G, e, ei, emask[e]);
       consumer_sync();
       if (threadIdx.x == 0) st_release(sync + si.a_ready + e, 1u);
     }
@@ -1326,7 +1317,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     const int nslots = tile_slots(a.D);
     int cur_rb = -1, slot = -1;
-    int rb0 = -1, n_rb = 0;   // the share's row blocks: rb0, rb0 + 1
     float acc[2][4] = {};
     auto flush = [&]() {      // this CTA's partial of row block cur_rb
       if (ok) {
@@ -1340,13 +1330,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (t < a.T) dst[(size_t)t * kDRows + r0 + 8 * (qq >> 1)] = acc[nt][qq];
           }
       }
-      if (n_rb == 0) rb0 = cur_rb;
-      ++n_rb;
     };
     {
       const int v0 = range_lo(c, S.ND, G), v1 = range_lo(c + 1, S.ND, G);
       for (int v = v0; v < v1; ++v) {
-        const DUnit d = down_unit(a, clist, S, v);
+        const DUnit d = down_unit(a, ulist, S, v);
         const int i = v - v0, ts = i % nslots;
         if (d.rb != cur_rb) {
           if (cur_rb >= 0) flush();
@@ -1405,14 +1393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // block's partials combines them
     consumer_sync();   // every warp's partials precede the counts, which release them
     if (warp == 0) {
-      const int n0 = n_rb > 0 ? rb_sources(rb0, S, G, s_src) : 0;
-      const int n1 = n_rb > 1 ? rb_sources(rb0 + 1, S, G, s_src + kMaxSms) : 0;
       bool last = false;
-      if (ok && lane < n_rb) {
-        const int nl = lane ? n1 : n0;
-        s_nsrc[lane] = nl;
-        last = atom_add_acq_rel(sync + si.rb_cnt + rb0 + lane, 1u) + 1u == (unsigned)nl;
-      }
+      if (ok && lane < n_rb)
+        last = atom_add_acq_rel(sync + si.rb_cnt + rb0 + lane, 1u) + 1u == (unsigned)s_nsrc[lane];
       const unsigned lm = __ballot_sync(kFull, last);
       if (lane == 0) ctl.bcast[0] = (int)lm;
     }
