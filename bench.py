@@ -42,8 +42,9 @@ DECODE_TS = (1, 4, 16)
 METRIC = "MoE-layer tokens/s (decode)"
 # DRAM bytes (read + write) per launch of the decode kernel at T = 16 from an
 # ncu capture of the current kernel (None until one is taken; a kernel changed
-# since its capture has no entry)
-NCU_DRAM_BYTES = {}
+# since its capture has no entry): kd_layer, edge layer, T = 16, 139.93 MB read
+# + 7.39 MB written (profiles/kd_layer_edge_decode_t16.md)
+NCU_DRAM_BYTES = {("layer", 16): 147_320_576}
 
 
 def parse():
