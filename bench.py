@@ -43,7 +43,7 @@ METRIC = "MoE-layer tokens/s (decode)"
 # DRAM bytes (read + write) per launch of the decode kernel at T = 16 from an
 # ncu capture of the current kernel (None until one is taken; a kernel changed
 # since its capture has no entry): kd_layer, edge layer, T = 16, 139.93 MB read
-# + 7.39 MB written (profiles/kd_layer_edge_decode_t16.md)
+# + 7.39 MB written, from `ncu --set full` of `bench.py --profile-tokens 16`
 NCU_DRAM_BYTES = {("layer", 16): 147_320_576}
 
 
@@ -454,6 +454,8 @@ def main():
                    "cuda_graph": True, "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": "kd_layer", "T": T_r, "achieved": achieved, "peak": P["hbm"],
                      "unit": "GB/s", "frac": achieved / P["hbm"], "traffic": NCU_DRAM_BYTES.get(("layer", T_r)),
+                     "traffic_source": "ncu capture of this kernel (dram__bytes_read.sum + dram__bytes_write.sum), "
+                                       "not measured in this run",
                      "algorithmic_bytes": bytes_T[T_r],
                      "peak_source": P["src"], "layer_achieved_gbs": layer_gbs,
                      "layer_frac": layer_gbs / P["hbm"],

@@ -73,7 +73,11 @@ def test_routing_full_size_large_layer(lib):
     shape, L = case("large_t16384")
     G = to_gpu(L, lib)
     toks = np.random.default_rng(0).choice(shape.T, 48, replace=False)
-    _routing_check(lib, shape, L, G, tokens=np.sort(toks))
+    # and the tokens whose logits come closest to zero, where a decision is
+    # easiest to get wrong (picked from an fp64 product of the inputs)
+    z64 = O.to_f64(L["x"]) @ O.to_f64(L["W_r"]).T + O.to_f64(L["b_r"])
+    near = np.argsort(np.abs(z64).min(axis=1))[:16]
+    _routing_check(lib, shape, L, G, tokens=np.unique(np.concatenate([toks, near])))
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "edge_decode_t1", "edge_decode_t4",
