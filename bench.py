@@ -571,6 +571,7 @@ def extras(deco, dev, stream, P):
     out["ratio_sweep"] = extra_sweep(deco, dev, stream, P, torch)
     out["topk_vs_relu"] = extra_topk(deco, dev, stream, P, torch)
     out["stack_8_layers_d4096"] = extra_stack(deco, dev, stream, P, torch)
+    out["experts_on_host"] = extra_host_experts(deco, dev, stream, P, torch)
     out["context"] = ("the pages report model-level decode speedups of DECO's kernel over dense "
                       "inference of 3.00x (Jetson AGX Orin) and 2.58x (RTX 4090), through FR-Spec on "
                       "Spec-Bench; other hardware and a whole model, not this layer")
@@ -725,6 +726,38 @@ def extra_topk(deco, dev, stream, P, torch):
                          "union_experts": int(act.any(dim=0).sum())}
         res[str(T)] = row
     del Gc, G
+    torch.cuda.empty_cache()
+    return res
+
+
+def extra_host_experts(deco, dev, stream, P, torch):
+    """The edge layer with its routed experts' W_up and W_down in pinned host
+    memory (the offloaded-parameter setting of the paper's §1): only the
+    activated experts' rows cross the host link.  T = 1, 4, 16 at ~20 %
+    activation and T = 1 with every expert active, eager; the rate is the
+    activated experts' bytes over the time."""
+    from synth import CONFIGS, make_layer
+    base = CONFIGS["edge_decode_t16"]["shape"]
+    per_expert = 2 * base.d_e * base.D * 2   # W_up[e] and W_down[e], bf16
+    res = {"note": "general kernels; x, router, mean and shared expert in HBM"}
+    for label, ratio, Ts in (("20%", 0.2, (1, 4, 16)), ("100%", 1.0, (1,))):
+        L = make_layer(base, CONFIGS["edge_decode_t16"]["seed"], ratio=ratio)
+        x_all = L.pop("x").to(dev)
+        G = {k: v.to(dev) for k, v in L.items()}
+        G["W_bar_up"] = deco.mean_up(G["W_up"])
+        H = dict(G)
+        H["W_up"], H["W_down"] = G["W_up"].cpu().pin_memory(), G["W_down"].cpu().pin_memory()
+        row = {}
+        for T in Ts:
+            x = x_all[:T]
+            o = torch.empty_like(x)
+            ws = deco.alloc_workspace(deco.layer_shape(x, H), dev)
+            ms = _time_eager(torch, stream, lambda: deco.forward(x, H, out=o, workspace=ws), n=5)
+            union = int(deco.routing(x, G)["active"].bool().any(dim=0).sum())
+            row[str(T)] = {"us": round(1000 * ms, 1), "union_experts": union,
+                           "host_link_gbs": round(union * per_expert / (ms / 1e3) / 1e9, 1)}
+        res[label] = row
+        del H, G
     torch.cuda.empty_cache()
     return res
 

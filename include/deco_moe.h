@@ -86,7 +86,20 @@ typedef enum { DECO_F32 = 0, DECO_BF16 = 1 } deco_dtype_t;
  *   gated    0: DECO's non-gated experts.  1: the gated variant of the
  *            ablation ([press] part 2, non-gated paragraph; [arXiv] §2
  *            "Expert design"): a_e = NormSiLU(x W_up[e]^T - u) * (x W_val[e]^T),
- *            element-wise, with the value branch W_val (weights.W_val)    */
+ *            element-wise, with the value branch W_val (weights.W_val)
+ *   experts_on_host
+ *            0: every weight is in device memory.  1: the routed experts'
+ *            matrices W_up, W_down (and W_val) stay in host memory, pinned
+ *            and mapped into the device's address space (cudaHostAlloc, or
+ *            cudaHostRegister with cudaHostRegisterMapped, on a system with
+ *            unified addressing, so the host pointer is the device pointer),
+ *            and the layer reads only the rows of the experts the batch
+ *            activates across the host link: the offloaded-parameter setting
+ *            behind the paper's memory-access argument ([arXiv] §1).  The
+ *            other weights stay in device memory.  These calls take the
+ *            general CUDA-core kernels, which read weights with plain loads;
+ *            a pointer that is not mapped host memory is rejected with
+ *            DECO_ERR_INVALID_ARG before anything is launched.            */
 typedef struct {
   int T;
   int d_model;
@@ -98,9 +111,11 @@ typedef struct {
   int residual;
   int topk;
   int gated;
+  int experts_on_host;
 } deco_moe_shape_t;
 
-/* The layer's weights (device pointers, storage dtype unless noted).
+/* The layer's weights (device pointers, storage dtype unless noted; with
+ * shape->experts_on_host, W_up, W_down and W_val are mapped host pointers).
  *   W_r      [E][D]        router projection
  *   b_r      [E]     fp32  router bias
  *   W_up     [E][d_e][D]   routed up-projections

@@ -41,7 +41,7 @@ class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("E", ctypes.c_int),
                 ("d_e", ctypes.c_int), ("d_s", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("rms_eps", ctypes.c_float), ("residual", ctypes.c_int), ("topk", ctypes.c_int),
-                ("gated", ctypes.c_int)]
+                ("gated", ctypes.c_int), ("experts_on_host", ctypes.c_int)]
 
 
 WEIGHT_NAMES = ("W_r", "b_r", "W_up", "W_bar_up", "W_down", "s", "W_s_up", "W_s_down", "W_val")
@@ -98,9 +98,10 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def make_shape(T, D, E, d_e, d_s, dtype, eps=1e-6, residual=False, topk=0, gated=False) -> Shape:
+def make_shape(T, D, E, d_e, d_s, dtype, eps=1e-6, residual=False, topk=0, gated=False,
+               experts_on_host=False) -> Shape:
     return Shape(T, D, E, d_e, d_s, _DT[dtype] if isinstance(dtype, torch.dtype) else dtype,
-                 eps, int(bool(residual)), int(topk), int(bool(gated)))
+                 eps, int(bool(residual)), int(topk), int(bool(gated)), int(bool(experts_on_host)))
 
 
 def _weights(L: dict) -> Weights:
@@ -108,10 +109,13 @@ def _weights(L: dict) -> Weights:
 
 
 def layer_shape(x: torch.Tensor, L: dict, eps=1e-6, residual=False, topk=0) -> Shape:
+    """The shape of a call; routed experts held in pinned host tensors (W_up,
+    W_down, W_val on the CPU, pin_memory) select experts_on_host."""
     E, d_e, D = L["W_up"].shape if "W_up" in L else (L["W_r"].shape[0], 64, x.shape[1])
     d_s = L["W_s_up"].shape[0] if "W_s_up" in L else 64
+    on_host = "W_up" in L and L["W_up"].device.type == "cpu"
     return make_shape(x.shape[0], x.shape[1], L["W_r"].shape[0], d_e, d_s, x.dtype, eps, residual,
-                      topk, "W_val" in L)
+                      topk, "W_val" in L, on_host)
 
 
 def workspace_size(shape: Shape) -> int:

@@ -51,7 +51,7 @@ inline int token_tile(int D, int dtype) { return (16 * (size_t)D * elem_size(dty
 // The tcgen05 prefill kernels (prefill_kernels.cuh) take bf16 batches of more
 // than 16 tokens whose routed experts fit one 256-column accumulator.
 bool prefill_eligible(const deco_moe_shape_t& s) {
-  return s.dtype == DECO_BF16 && s.T > dec::kMaxT && s.d_e <= pf::kBN;
+  return s.dtype == DECO_BF16 && s.T > dec::kMaxT && s.d_e <= pf::kBN && !s.experts_on_host;
 }
 
 // bf16 batches of more than 16 tokens are routed by the tiled router
@@ -124,6 +124,7 @@ deco_status_t check_shape(const deco_moe_shape_t* s) {
   if (s->residual != 0 && s->residual != 1) return DECO_ERR_INVALID_ARG;
   if (s->topk < 0 || s->topk > s->E) return DECO_ERR_INVALID_ARG;
   if (s->gated != 0 && s->gated != 1) return DECO_ERR_INVALID_ARG;
+  if (s->experts_on_host != 0 && s->experts_on_host != 1) return DECO_ERR_INVALID_ARG;
   if (s->d_model % 64 || s->d_model > 16384) return DECO_ERR_UNSUPPORTED;
   if (s->E > 256) return DECO_ERR_UNSUPPORTED;
   if (s->d_e % 64 || s->d_e > 512) return DECO_ERR_UNSUPPORTED;
@@ -132,7 +133,19 @@ deco_status_t check_shape(const deco_moe_shape_t* s) {
   return DECO_OK;
 }
 
-deco_status_t check_weights(const deco_moe_weights_t* w, bool router_only, bool gated = false) {
+// host memory the device reads through its own address space: pinned and
+// mapped, with unified addressing (the device pointer is the host pointer)
+bool host_mapped(const void* p) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeHost && at.devicePointer == p;
+}
+
+deco_status_t check_weights(const deco_moe_weights_t* w, bool router_only, bool gated = false,
+                            bool experts_on_host = false) {
   if (!w || !w->W_r || !w->b_r) return DECO_ERR_INVALID_ARG;
   if (!aligned16(w->W_r)) return DECO_ERR_INVALID_ARG;
   if (router_only) return DECO_OK;
@@ -140,6 +153,9 @@ deco_status_t check_weights(const deco_moe_weights_t* w, bool router_only, bool 
   const void* ps[] = {w->W_up, w->W_bar_up, w->W_down, w->s, w->W_s_up, w->W_s_down};
   for (const void* p : ps)
     if (!p || !aligned16(p)) return DECO_ERR_INVALID_ARG;
+  if (experts_on_host &&
+      (!host_mapped(w->W_up) || !host_mapped(w->W_down) || (gated && !host_mapped(w->W_val))))
+    return DECO_ERR_INVALID_ARG;
   return DECO_OK;
 }
 
@@ -189,7 +205,7 @@ bool decode_grid_ok(int D, int E, int sms) {
 }
 
 bool decode_eligible(const deco_moe_shape_t& s, int sms) {
-  if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT) return false;
+  if (s.dtype != DECO_BF16 || s.T < 1 || s.T > dec::kMaxT || s.experts_on_host) return false;
   if (s.E > 256 || s.d_e > 256 || s.d_e % 64 || s.d_s % 64) return false;
   return decode_grid_ok(s.d_model, s.E, sms);
 }
@@ -740,7 +756,7 @@ deco_status_t deco_moe_forward(const deco_moe_shape_t* shape, const void* x,
                                size_t workspace_bytes, void* stream) {
   deco_status_t st = check_shape(shape);
   if (st != DECO_OK) return st;
-  if ((st = check_weights(w, false, shape->gated)) != DECO_OK) return st;
+  if ((st = check_weights(w, false, shape->gated, shape->experts_on_host)) != DECO_OK) return st;
   if (shape->T == 0) return DECO_OK;
   if (!x || !out || !aligned16(x) || !aligned16(out) || x == out) return DECO_ERR_INVALID_ARG;
   const Plan p = make_plan(*shape);
@@ -944,7 +960,7 @@ extern "C" deco_status_t deco_moe_forward_static(const deco_moe_shape_t* shape, 
                                                  void* stream) {
   deco_status_t st = check_shape(shape);
   if (st != DECO_OK) return st;
-  if ((st = check_weights(w, false, shape->gated)) != DECO_OK) return st;
+  if ((st = check_weights(w, false, shape->gated, shape->experts_on_host)) != DECO_OK) return st;
   if (shape->T == 0) return DECO_OK;
   if (!x || !out || !aligned16(x) || !aligned16(out) || x == out) return DECO_ERR_INVALID_ARG;
   if (make_plan(*shape).total > DECO_STATIC_SCRATCH_BYTES) return DECO_ERR_WORKSPACE;

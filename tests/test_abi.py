@@ -149,3 +149,21 @@ def test_decode_workspaces_fit_the_static_scratch(deco):
         for D, E, d_s in ((2048, 64, 1024), (4096, 128, 2048)):
             rc, n = _ws(deco, _shape(deco, T=T, D=D, E=E, d_s=d_s))
             assert rc == 0 and n <= deco.STATIC_SCRATCH_BYTES, (T, D, E, n)
+
+
+def test_experts_on_host_is_checked_before_launching(deco):
+    """Host-resident experts: the flag is 0 or 1, such a batch takes the
+    general kernels (no per-pair rows in its workspace), and weight pointers
+    that are not mapped host memory are rejected before any launch."""
+    T, D, E = 32, 2048, 64
+    s = _shape(deco, T=T)
+    s.experts_on_host = 2
+    assert _ws(deco, s)[0] == 1
+    s.experts_on_host = 1
+    rc, n = _ws(deco, s)
+    assert rc == 0 and n < T * E * D * 2
+    w = _fake_weights(deco)
+    assert deco._lib.deco_moe_forward(ctypes.byref(s), 0x100000, ctypes.byref(w), 0x200000, 0x300000,
+                                      n, None) == 1
+    assert deco._lib.deco_moe_forward_static(ctypes.byref(s), 0x100000, ctypes.byref(w), 0x200000,
+                                             None) == 1

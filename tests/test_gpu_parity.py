@@ -595,3 +595,51 @@ def test_gated_requires_the_value_branch(lib):
     rc = lib._lib.deco_moe_forward(ctypes.byref(sh), G["x"].data_ptr(), ctypes.byref(w), out.data_ptr(),
                                    ws.data_ptr(), ws.numel(), lib._stream(None))
     assert rc == 1
+
+
+# --------------------------------------------------------------------------
+# routed experts held in pinned host memory (offloaded parameters)
+
+def _host_experts(G):
+    """The routed experts' matrices moved to pinned host memory, which the
+    device reads through its own address space."""
+    H = dict(G)
+    for n in ("W_up", "W_down", "W_val"):
+        if n in H:
+            H[n] = H[n].cpu().pin_memory()
+    return H
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "edge_decode_t4"])
+def test_experts_in_host_memory(lib, name):
+    shape, L = case(name)
+    G = to_gpu(L, lib)
+    H = _host_experts(G)
+    assert lib.layer_shape(G["x"], H).experts_on_host == 1
+    out = lib.forward(G["x"], H, eps=shape.eps)
+    torch.cuda.synchronize()
+    ref = oracle_forward(O.to_f64(L["x"]), to_oracle(L, shape.dtype), shape.eps, range(shape.T))
+    check_close(out.double().cpu().numpy(), ref, shape.dtype, name + " experts on host")
+    if shape.dtype == "f32":   # the same general kernels as device-resident weights: bitwise equal
+        assert torch.equal(out, lib.forward(G["x"], G, eps=shape.eps))
+
+
+def test_experts_in_host_memory_prefill_batch_and_gated(lib):
+    shape = LayerShape(40, 512, 16, 128, 256, "bf16")
+    for gated in (False, True):
+        L = make_layer(shape, 31, gated=gated)
+        G = to_gpu(L, lib)
+        out = lib.forward(G["x"], _host_experts(G), eps=shape.eps)
+        torch.cuda.synchronize()
+        ref = oracle_forward(O.to_f64(L["x"]), to_oracle(L, shape.dtype), shape.eps, range(shape.T))
+        check_close(out.double().cpu().numpy(), ref, shape.dtype, f"host experts T=40 gated={gated}")
+
+
+def test_experts_on_host_must_be_mapped(lib):
+    shape, L = case("edge_decode_t4")
+    G = to_gpu(L, lib)
+    H = dict(G)
+    H["W_up"], H["W_down"] = G["W_up"].cpu(), G["W_down"].cpu()   # pageable: not reachable
+    with pytest.raises(lib.DecoError) as ei:
+        lib.forward(G["x"], H, eps=shape.eps)
+    assert ei.value.code == 1
