@@ -56,3 +56,6 @@ from .deco import (  # noqa: F401
     mean_up, norm_silu, expert_output, shared_expert, layer_forward,
     layer_forward_tokens, dense_ffn, stack_forward, topk_route, exact_logit,
 )
+from .backward import (  # noqa: F401
+    silu_grad, norm_silu_backward, layer_backward_tokens, router_entropy, sparsity_controller,
+)
