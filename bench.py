@@ -572,6 +572,7 @@ def extras(deco, dev, stream, P):
     out["topk_vs_relu"] = extra_topk(deco, dev, stream, P, torch)
     out["stack_8_layers_d4096"] = extra_stack(deco, dev, stream, P, torch)
     out["experts_on_host"] = extra_host_experts(deco, dev, stream, P, torch)
+    out["backward"] = extra_backward(deco, dev, stream, P, torch)
     out["context"] = ("the pages report model-level decode speedups of DECO's kernel over dense "
                       "inference of 3.00x (Jetson AGX Orin) and 2.58x (RTX 4090), through FR-Spec on "
                       "Spec-Bench; other hardware and a whole model, not this layer")
@@ -758,6 +759,35 @@ def extra_host_experts(deco, dev, stream, P, torch):
                            "host_link_gbs": round(union * per_expert / (ms / 1e3) / 1e9, 1)}
         res[label] = row
         del H, G
+    torch.cuda.empty_cache()
+    return res
+
+
+def extra_backward(deco, dev, stream, P, torch):
+    """The layer's backward pass (CUDA-core kernels, fixed-order sums) on the
+    edge layer at T = 1, 16 and 256, eager.  Bytes: the weights it reads once
+    (router, mean, shared, the union's W_up and W_down) plus the fp32
+    gradients it writes (every weight's); the rate is against HBM."""
+    from synth import CONFIGS, LayerShape, make_layer
+    base = CONFIGS["edge_decode_t16"]["shape"]
+    D, E, de, ds = base.D, base.E, base.d_e, base.d_s
+    res = {"note": "first version: CUDA cores, one thread per output element"}
+    shape = LayerShape(256, D, E, de, ds, "bf16")
+    L = make_layer(shape, CONFIGS["edge_decode_t16"]["seed"])
+    x_all = L.pop("x").to(dev)
+    G = {k: v.to(dev) for k, v in L.items()}
+    G["W_bar_up"] = deco.mean_up(G["W_up"])
+    grad_bytes = 4 * sum(t.numel() for k, t in G.items() if k != "W_bar_up")
+    for T in (1, 16, 256):
+        x = x_all[:T]
+        dy = torch.randn(T, D, device=dev).to(torch.bfloat16)
+        union = int(deco.routing(x, G)["active"].bool().any(dim=0).sum())
+        wbytes = 2 * (D * (E + de + ds) + D * ds + union * 2 * de * D)
+        ms = _time_eager(torch, stream, lambda: deco.backward(x, G, dy), n=5)
+        gbs = (wbytes + grad_bytes + T * D * 4) / (ms / 1e3) / 1e9
+        res[str(T)] = {"ms": round(ms, 3), "union_experts": union, "gbs": round(gbs, 1),
+                       "hbm_frac": round(gbs / P["hbm"], 4) if "hbm" in P else None}
+    del G
     torch.cuda.empty_cache()
     return res
 

@@ -278,6 +278,68 @@ deco_status_t deco_set_wait_limit(long long cycles);
  * thread. */
 deco_status_t deco_moe_set_profiling(void* const* events, int n_events);
 
+/* ---- training side -------------------------------------------------------
+ * The backward pass of the layer and the pieces of the paper's adaptive
+ * sparsity regularisation ([arXiv] §2 "Auxiliary training objective": an
+ * auto-scaling coefficient on the router entropy; [press] part 3: the
+ * coefficient is multiplied by a small factor such as 1.002 after every
+ * iteration whose activation ratio is above the target, divided by it when
+ * below). */
+
+/* Gradients of the loss with respect to the layer's input and weights (device
+ * pointers, fp32, the shapes of the corresponding inputs; all written in
+ * full).  dW_up includes the mean up-projection's share: W_bar_up is taken as
+ * the function mean_e W_up[e], so its gradient reaches every W_up[e] as
+ * dW_bar_up / E.  dW_val only for gated experts (NULL otherwise). */
+typedef struct {
+  float* dx;         /* [T][D]        */
+  float* dW_r;       /* [E][D]        */
+  float* db_r;       /* [E]           */
+  float* dW_up;      /* [E][d_e][D]   */
+  float* dW_down;    /* [E][D][d_e]   */
+  float* ds;         /* [E]           */
+  float* dW_s_up;    /* [d_s][D]      */
+  float* dW_s_down;  /* [D][d_s]      */
+  float* dW_val;     /* [E][d_e][D]   */
+} deco_moe_grads_t;
+
+/* Bytes of device workspace deco_moe_backward needs for `shape`
+ * (DECO_ERR_UNSUPPORTED for TopK routing, whose gradient is not provided). */
+deco_status_t deco_moe_backward_workspace_size(const deco_moe_shape_t* shape, size_t* bytes);
+
+/* Backward pass: given dy [T][D] (x's dtype) = dLoss/dout, writes every
+ * gradient of `grads`.  The routing is recomputed with the forward pass's
+ * exact router, so the active sets are those of deco_moe_forward; the
+ * gradient of ReLU routing is 1 on the active set (z > 0) and 0 elsewhere.
+ * dz_extra [T][E] fp32 (device, may be NULL) is an extra gradient on the
+ * router logits from another term of the loss (the entropy regulariser,
+ * deco_moe_router_entropy), added where the expert is active.  With
+ * shape->residual, dx includes dy.  CUDA-core kernels in fp32 with every sum
+ * in a fixed order: bitwise reproducible.  The workspace is as for
+ * deco_moe_forward (caller-owned, 256-byte aligned, no initialisation;
+ * deco_moe_device_error reads its error word).  Errors as deco_moe_forward. */
+deco_status_t deco_moe_backward(const deco_moe_shape_t* shape, const void* x,
+                                const deco_moe_weights_t* w, const void* dy, const float* dz_extra,
+                                const deco_moe_grads_t* grads, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* Router entropy regulariser (device pointers).  For token t, over the experts
+ * it activates (active[t][e] = 1), with r = ReLU(z) the routing weights
+ * [T][E] fp32 of deco_moe_routing: R = sum r, p = r / R and
+ * H_t = -sum p log p (0 when the token activates nothing); H[t] = H_t and
+ * H[T] = the mean over tokens (H holds T + 1 floats).  dz [T][E] gets
+ * lambda * d(mean_t H_t)/dz = -lambda (log p_e + H_t) / (R T) where active and
+ * 0 elsewhere: pass it to deco_moe_backward as dz_extra.  The entropy form is
+ * this library's reading (the pages name the router entropy but give no
+ * formula). */
+deco_status_t deco_moe_router_entropy(int T, int E, const float* r, const uint8_t* active, float lambda,
+                                      float* H, float* dz, void* stream);
+
+/* One step of the adaptive sparsity coefficient (host): *lambda is multiplied
+ * by factor (> 1) when the iteration's activation ratio is above the target,
+ * divided by it when below, unchanged when equal. */
+deco_status_t deco_sparsity_controller(double* lambda, double ratio, double target, double factor);
+
 /* The name and description of the CUDA error behind the last DECO_ERR_CUDA
  * status returned on the calling thread ("" if none).  The string is owned by
  * the library and stays valid until the next call on this thread. */

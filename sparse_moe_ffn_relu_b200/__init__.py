@@ -51,6 +51,13 @@ class Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_NAMES]
 
 
+GRAD_NAMES = ("dx", "dW_r", "db_r", "dW_up", "dW_down", "ds", "dW_s_up", "dW_s_down", "dW_val")
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in GRAD_NAMES]
+
+
 class Routing(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("r", "active", "counts", "offsets", "perm", "n_tok")]
 
@@ -69,6 +76,12 @@ _sig = {
     "deco_moe_forward_static": [ctypes.POINTER(Shape), _vp, ctypes.POINTER(Weights), _vp, _vp],
     "deco_moe_static_device_error": [ctypes.POINTER(ctypes.c_int), _vp],
     "deco_set_wait_limit": [ctypes.c_longlong],
+    "deco_moe_backward_workspace_size": [ctypes.POINTER(Shape), ctypes.POINTER(_sz)],
+    "deco_moe_backward": [ctypes.POINTER(Shape), _vp, ctypes.POINTER(Weights), _vp, _vp,
+                          ctypes.POINTER(Grads), _vp, _sz, _vp],
+    "deco_moe_router_entropy": [ctypes.c_int, ctypes.c_int, _vp, _vp, ctypes.c_float, _vp, _vp, _vp],
+    "deco_sparsity_controller": [ctypes.POINTER(ctypes.c_double), ctypes.c_double, ctypes.c_double,
+                                 ctypes.c_double],
 }
 for _name, _args in _sig.items():
     _f = getattr(_lib, _name)
@@ -259,3 +272,53 @@ def static_device_error(stream=None) -> int:
 def set_wait_limit(cycles: int):
     """Test hook: kernels give up waits for data after `cycles` SM cycles (0: default)."""
     _check(_lib.deco_set_wait_limit(int(cycles)), "set_wait_limit")
+
+
+# --------------------------------------------------------------------------
+# training side
+
+def backward(x: torch.Tensor, L: dict, dy: torch.Tensor, dz_extra=None, workspace=None, eps=1e-6,
+             residual=False, stream=None) -> dict:
+    """Gradients of the loss through the layer given dy = dLoss/dout: a dict
+    of fp32 tensors dx, dW_r, db_r, dW_up (with the mean up-projection's
+    share), dW_down, ds, dW_s_up, dW_s_down (and dW_val for gated experts).
+    dz_extra [T][E] fp32: an extra gradient on the router logits (see
+    router_entropy)."""
+    shape = layer_shape(x, L, eps, residual)
+    n = _sz(0)
+    _check(_lib.deco_moe_backward_workspace_size(ctypes.byref(shape), ctypes.byref(n)), "backward_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=x.device)
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g = {"dx": torch.empty(x.shape, **f32)}
+    for name, src in (("dW_r", "W_r"), ("db_r", "b_r"), ("dW_up", "W_up"), ("dW_down", "W_down"),
+                      ("ds", "s"), ("dW_s_up", "W_s_up"), ("dW_s_down", "W_s_down"), ("dW_val", "W_val")):
+        if src in L:
+            g[name] = torch.empty(L[src].shape, **f32)
+    gs = Grads(*[_ptr(g.get(n)) for n in GRAD_NAMES])
+    w = _weights(L)
+    _check(_lib.deco_moe_backward(ctypes.byref(shape), _ptr(x), ctypes.byref(w), _ptr(dy), _ptr(dz_extra),
+                                  ctypes.byref(gs), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "backward")
+    return g
+
+
+def router_entropy(r: torch.Tensor, active: torch.Tensor, lam: float, stream=None):
+    """(H [T+1] with the per-token router entropies and their mean last,
+    dz [T][E] = lam * d(mean entropy)/dz) from deco_moe_routing's r and
+    active."""
+    T, E = r.shape
+    H = torch.empty(T + 1, dtype=torch.float32, device=r.device)
+    dz = torch.empty(T, E, dtype=torch.float32, device=r.device)
+    _check(_lib.deco_moe_router_entropy(T, E, _ptr(r), _ptr(active), float(lam), _ptr(H), _ptr(dz),
+                                        _stream(stream)), "router_entropy")
+    return H, dz
+
+
+def sparsity_controller(lam: float, ratio: float, target: float, factor: float = 1.002) -> float:
+    """One step of the adaptive sparsity coefficient (x factor above the
+    target activation ratio, / factor below)."""
+    v = ctypes.c_double(lam)
+    _check(_lib.deco_sparsity_controller(ctypes.byref(v), float(ratio), float(target), float(factor)),
+           "sparsity_controller")
+    return v.value

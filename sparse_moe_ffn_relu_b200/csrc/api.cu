@@ -13,6 +13,7 @@
 
 #include "../../include/deco_moe.h"
 #include "simt_kernels.cuh"
+#include "backward_kernels.cuh"
 #include "decode_kernels.cuh"
 #include "prefill_kernels.cuh"
 
@@ -979,4 +980,192 @@ extern "C" deco_status_t deco_moe_static_device_error(int* code, void* stream) {
   if (err != cudaSuccess) return cuda_status(err, "static_device_error: scratch address");
   // the error word sits at the start of every workspace plan
   return deco_moe_device_error(scratch, code, stream);
+}
+
+// ---------------------------------------------------------------------------
+// training side: backward pass, router entropy, sparsity controller
+// (backward_kernels.cuh)
+
+namespace deco {
+namespace {
+
+struct BwdPlan {
+  Plan route;   // the routing buffers of a forward plan (no tensor-core staging)
+  size_t u, hs, as, du, dhs, pa, pdc, pdq, pz, pw, pk, dWbar, total;
+};
+
+BwdPlan make_bwd_plan(const deco_moe_shape_t& s) {
+  deco_moe_shape_t rs = s;
+  rs.experts_on_host = 1;   // a plan for the general kernels: routing, tables, no per-pair rows
+  BwdPlan b{};
+  b.route = make_plan(rs);
+  size_t off = b.route.total;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t T = s.T, P = T * s.E;
+  b.u = take(T * s.d_e * 4);
+  b.hs = take(T * s.d_s * 4);
+  b.as = take(T * s.d_s * 4);
+  b.du = take(T * s.d_e * 4);
+  b.dhs = take(T * s.d_s * 4);
+  b.pa = take(P * s.d_e * 4);
+  b.pdc = take(P * s.d_e * 4);
+  b.pdq = s.gated ? take(P * s.d_e * 4) : 0;
+  b.pz = take(P * 4);
+  b.pw = take(P * 4);
+  b.pk = take(P * 4);
+  b.dWbar = take((size_t)s.d_e * s.d_model * 4);
+  b.total = off;
+  return b;
+}
+
+deco_status_t check_bwd_shape(const deco_moe_shape_t* s) {
+  const deco_status_t st = check_shape(s);
+  if (st != DECO_OK) return st;
+  if (s->topk != 0) return DECO_ERR_UNSUPPORTED;   // the gradient is that of ReLU routing
+  return DECO_OK;
+}
+
+template <typename T>
+cudaError_t run_backward(const deco_moe_shape_t& s, const void* x, const deco_moe_weights_t& w, const void* dy,
+                         const float* dz_extra, const deco_moe_grads_t& g, unsigned char* ws, const BwdPlan& b,
+                         cudaStream_t st) {
+  const Plan& p = b.route;
+  float* r = reinterpret_cast<float*>(ws + p.r);
+  uint8_t* act = ws + p.act;
+  int* counts = reinterpret_cast<int*>(ws + p.counts);
+  int* offsets = reinterpret_cast<int*>(ws + p.offsets);
+  int* perm = reinterpret_cast<int*>(ws + p.perm);
+  int* n_tok = reinterpret_cast<int*>(ws + p.n_tok);
+  cudaError_t err = run_routing<T>(s, x, w, ws, p, false, r, act, counts, offsets, perm, n_tok, st, p.tile_rows);
+  if (err != cudaSuccess) return err;
+  bwd::Args a{};
+  a.T = s.T;
+  a.D = s.d_model;
+  a.E = s.E;
+  a.d_e = s.d_e;
+  a.d_s = s.d_s;
+  a.eps = s.rms_eps;
+  a.gated = s.gated;
+  a.residual = s.residual;
+  a.x = x;
+  a.dy = dy;
+  a.dz_extra = dz_extra;
+  a.W_r = w.W_r;
+  a.W_bar = w.W_bar_up;
+  a.W_up = w.W_up;
+  a.W_down = w.W_down;
+  a.s = w.s;
+  a.W_s_up = w.W_s_up;
+  a.W_s_down = w.W_s_down;
+  a.W_val = w.W_val;
+  a.r = r;
+  a.act = act;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.pair_of = reinterpret_cast<const int*>(ws + p.pair_of);
+  a.u = reinterpret_cast<float*>(ws + b.u);
+  a.hs = reinterpret_cast<float*>(ws + b.hs);
+  a.as = reinterpret_cast<float*>(ws + b.as);
+  a.du = reinterpret_cast<float*>(ws + b.du);
+  a.dhs = reinterpret_cast<float*>(ws + b.dhs);
+  a.pa = reinterpret_cast<float*>(ws + b.pa);
+  a.pdc = reinterpret_cast<float*>(ws + b.pdc);
+  a.pdq = s.gated ? reinterpret_cast<float*>(ws + b.pdq) : nullptr;
+  a.pz = reinterpret_cast<float*>(ws + b.pz);
+  a.pw = reinterpret_cast<float*>(ws + b.pw);
+  a.pk = reinterpret_cast<float*>(ws + b.pk);
+  a.dWbar = reinterpret_cast<float*>(ws + b.dWbar);
+  a.dx = g.dx;
+  a.dW_r = g.dW_r;
+  a.db_r = g.db_r;
+  a.dW_up = g.dW_up;
+  a.dW_down = g.dW_down;
+  a.ds = g.ds;
+  a.dW_s_up = g.dW_s_up;
+  a.dW_s_down = g.dW_s_down;
+  a.dW_val = g.dW_val;
+  const size_t sm0 = (size_t)s.d_model * 4;
+  const size_t sm1 = (2 * (size_t)s.d_model + 3 * (size_t)s.d_e) * 4;
+  const size_t sm2 = ((size_t)s.d_model + s.d_s + 3 * (size_t)s.d_e) * 4;
+  if ((err = allow_smem(bwd::kb_token_fwd<T>, sm0)) != cudaSuccess) return err;
+  if ((err = allow_smem(bwd::kb_pair<T>, sm1)) != cudaSuccess) return err;
+  if ((err = allow_smem(bwd::kb_token_bwd<T>, sm2)) != cudaSuccess) return err;
+  bwd::kb_token_fwd<T><<<s.T, bwd::kThreads, sm0, st>>>(a);
+  bwd::kb_pair<T><<<dim3(s.T, s.E), bwd::kThreads, sm1, st>>>(a);
+  bwd::kb_token_bwd<T><<<s.T, bwd::kThreads, sm2, st>>>(a);
+  const size_t n_sums = ((size_t)s.d_e + 2 * (size_t)s.d_s) * s.d_model;
+  bwd::kb_sums<T><<<(unsigned)std::min<size_t>((n_sums + bwd::kThreads - 1) / bwd::kThreads, 4096),
+                    bwd::kThreads, 0, st>>>(a);
+  const size_t n_exp = (size_t)s.d_e * s.d_model * (s.gated ? 3 : 2) + s.d_model + 2;
+  bwd::kb_expert<T><<<dim3((unsigned)std::min<size_t>((n_exp + bwd::kThreads - 1) / bwd::kThreads, 64), s.E),
+                      bwd::kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace deco
+
+extern "C" deco_status_t deco_moe_backward_workspace_size(const deco_moe_shape_t* shape, size_t* bytes) {
+  using namespace deco;
+  const deco_status_t st = check_bwd_shape(shape);
+  if (st != DECO_OK) return st;
+  if (!bytes) return DECO_ERR_INVALID_ARG;
+  *bytes = make_bwd_plan(*shape).total;
+  return DECO_OK;
+}
+
+extern "C" deco_status_t deco_moe_backward(const deco_moe_shape_t* shape, const void* x,
+                                           const deco_moe_weights_t* w, const void* dy, const float* dz_extra,
+                                           const deco_moe_grads_t* g, void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+  using namespace deco;
+  deco_status_t st = check_bwd_shape(shape);
+  if (st != DECO_OK) return st;
+  if ((st = check_weights(w, false, shape->gated, shape->experts_on_host)) != DECO_OK) return st;
+  if (!g) return DECO_ERR_INVALID_ARG;
+  float* gs[] = {g->dx, g->dW_r, g->db_r, g->dW_up, g->dW_down, g->ds, g->dW_s_up, g->dW_s_down};
+  for (float* q : gs)
+    if (!q || !aligned16(q)) return DECO_ERR_INVALID_ARG;
+  if (shape->gated && (!g->dW_val || !aligned16(g->dW_val))) return DECO_ERR_INVALID_ARG;
+  if (shape->T == 0) return DECO_OK;
+  if (!x || !dy || !aligned16(x) || !aligned16(dy)) return DECO_ERR_INVALID_ARG;
+  if (dz_extra && (reinterpret_cast<uintptr_t>(dz_extra) & 3u)) return DECO_ERR_INVALID_ARG;
+  const BwdPlan b = make_bwd_plan(*shape);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DECO_ERR_WORKSPACE;
+  if (workspace_bytes < b.total) return DECO_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t cs = as_stream(stream);
+  std::lock_guard<std::mutex> lock(g_smem_mutex);
+  cudaError_t err = cudaMemsetAsync(ws + b.route.err, 0, 16, cs);
+  if (err != cudaSuccess) return cuda_status(err, "backward: clearing the error word");
+  err = shape->dtype == DECO_F32 ? run_backward<float>(*shape, x, *w, dy, dz_extra, *g, ws, b, cs)
+                                 : run_backward<bf16>(*shape, x, *w, dy, dz_extra, *g, ws, b, cs);
+  return cuda_status(err, "backward");
+}
+
+extern "C" deco_status_t deco_moe_router_entropy(int T, int E, const float* r, const uint8_t* active,
+                                                 float lambda, float* H, float* dz, void* stream) {
+  using namespace deco;
+  if (T < 0 || E <= 0 || E > 256 || !std::isfinite(lambda)) return DECO_ERR_INVALID_ARG;
+  if (T == 0) return DECO_OK;
+  if (!r || !active || !H || !dz || (reinterpret_cast<uintptr_t>(r) & 3u) ||
+      (reinterpret_cast<uintptr_t>(H) & 3u) || (reinterpret_cast<uintptr_t>(dz) & 3u))
+    return DECO_ERR_INVALID_ARG;
+  cudaStream_t cs = as_stream(stream);
+  bwd::kb_entropy<<<(T + bwd::kWarps - 1) / bwd::kWarps, bwd::kThreads, 0, cs>>>(r, active, T, E, lambda, H, dz);
+  bwd::kb_entropy_mean<<<1, 32, 0, cs>>>(H, T);
+  return cuda_status(cudaGetLastError(), "router_entropy");
+}
+
+extern "C" deco_status_t deco_sparsity_controller(double* lambda, double ratio, double target, double factor) {
+  if (!lambda || !(factor > 1.0) || !std::isfinite(factor) || !std::isfinite(ratio) || !std::isfinite(target) ||
+      !std::isfinite(*lambda))
+    return DECO_ERR_INVALID_ARG;
+  if (ratio > target) *lambda *= factor;
+  else if (ratio < target) *lambda /= factor;
+  return DECO_OK;
 }

@@ -167,3 +167,30 @@ def test_experts_on_host_is_checked_before_launching(deco):
                                       n, None) == 1
     assert deco._lib.deco_moe_forward_static(ctypes.byref(s), 0x100000, ctypes.byref(w), 0x200000,
                                              None) == 1
+
+
+def test_training_side_host_checks(deco):
+    """The sparsity controller against the oracle's, and the backward's
+    argument checks (no launch)."""
+    import oracle as O
+    for lam, ratio, target in [(1.0, 0.25, 0.2), (0.5, 0.1, 0.2), (2.0, 0.2, 0.2)]:
+        assert deco.sparsity_controller(lam, ratio, target) == O.sparsity_controller(lam, ratio, target)
+    v = ctypes.c_double(1.0)
+    assert deco._lib.deco_sparsity_controller(ctypes.byref(v), 0.3, 0.2, 1.0) == 1   # factor must exceed 1
+    lib = deco._lib
+    s = _shape(deco)
+    n = ctypes.c_size_t(0)
+    assert lib.deco_moe_backward_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0 and n.value > 0
+    st = _shape(deco)
+    st.topk = 13
+    assert lib.deco_moe_backward_workspace_size(ctypes.byref(st), ctypes.byref(n)) == 2
+    w = _fake_weights(deco)
+    g = deco.Grads(*[0x500000 + 0x1000 * i for i in range(8)])
+    bw = lambda sh, gg, ws, nb: lib.deco_moe_backward(  # noqa: E731
+        ctypes.byref(sh), 0x100000, ctypes.byref(w), 0x180000, None, gg, ws, nb, None)
+    assert lib.deco_moe_backward_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert bw(s, None, 0x300000, n.value) == 1                              # no gradients
+    assert bw(s, ctypes.byref(deco.Grads(*([0] * 9))), 0x300000, n.value) == 1
+    assert bw(s, ctypes.byref(g), 0x300000, n.value - 1) == 3               # workspace too small
+    assert bw(st, ctypes.byref(g), 0x300000, n.value) == 2                  # TopK
+    assert lib.deco_moe_router_entropy(4, 0, 0x1000, 0x2000, 1.0, 0x3000, 0x4000, None) == 1
