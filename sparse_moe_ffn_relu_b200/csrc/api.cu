@@ -1090,13 +1090,14 @@ cudaError_t run_backward(const deco_moe_shape_t& s, const void* x, const deco_mo
   a.dW_val = g.dW_val;
   const size_t sm0 = (size_t)s.d_model * 4;
   const size_t sm1 = (2 * (size_t)s.d_model + 3 * (size_t)s.d_e) * 4;
-  const size_t sm2 = ((size_t)s.d_model + s.d_s + 3 * (size_t)s.d_e) * 4;
+  const size_t sm3 = ((size_t)s.d_s + 3 * (size_t)s.d_e) * 4;
   if ((err = allow_smem(bwd::kb_token_fwd<T>, sm0)) != cudaSuccess) return err;
   if ((err = allow_smem(bwd::kb_pair<T>, sm1)) != cudaSuccess) return err;
-  if ((err = allow_smem(bwd::kb_token_bwd<T>, sm2)) != cudaSuccess) return err;
-  bwd::kb_token_fwd<T><<<s.T, bwd::kThreads, sm0, st>>>(a);
+  if ((err = allow_smem(bwd::kb_dx<T>, sm3)) != cudaSuccess) return err;
+  bwd::kb_token_fwd<T><<<dim3(s.T, (s.d_e + s.d_s + bwd::kFwdRows - 1) / bwd::kFwdRows), bwd::kThreads, sm0, st>>>(a);
   bwd::kb_pair<T><<<dim3(s.T, s.E), bwd::kThreads, sm1, st>>>(a);
-  bwd::kb_token_bwd<T><<<s.T, bwd::kThreads, sm2, st>>>(a);
+  bwd::kb_token_mid<T><<<dim3(s.T, (s.d_s + 31) / 32), bwd::kThreads, 0, st>>>(a);
+  bwd::kb_dx<T><<<dim3(s.T, (s.d_model + bwd::kThreads - 1) / bwd::kThreads), bwd::kThreads, sm3, st>>>(a);
   const size_t n_sums = ((size_t)s.d_e + 2 * (size_t)s.d_s) * s.d_model;
   bwd::kb_sums<T><<<(unsigned)std::min<size_t>((n_sums + bwd::kThreads - 1) / bwd::kThreads, 4096),
                     bwd::kThreads, 0, st>>>(a);

@@ -22,9 +22,10 @@
 // element per thread with its sums in a fixed order (pairs of an expert in
 // token order, experts of a token ascending), so the gradients are bitwise
 // reproducible.  They favour clarity over speed:
-//   kb_token_fwd   per token: u = W_bar x, hs = W_s_up x (pre-activation)
+//   kb_token_fwd   per token and 64 rows: u = W_bar x, hs = W_s_up x (pre-activation)
 //   kb_pair        per active (token, expert): the pair's a, dc, dq, dz, r w
-//   kb_token_bwd   per token: du, the shared expert's dhs and SiLU(hs), dx
+//   kb_token_mid   per token and 32 shared columns: dhs, SiLU(hs); and du
+//   kb_dx          per token and 256 columns: dx
 //   kb_sums        dW_bar, dW_s_up, dW_s_down (sums over tokens)
 //   kb_expert      dW_up (+ dW_bar / E), dW_val, dW_down, dW_r, db_r, ds
 //                  (sums over each expert's pairs)
@@ -117,7 +118,9 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return t;
 }
 
-// per token: u = W_bar x and hs = W_s_up x (before the SiLU)
+// per token and block of kFwdRows rows: u = W_bar x and hs = W_s_up x
+// (before the SiLU); grid (T, rows / kFwdRows)
+constexpr int kFwdRows = 64;
 template <typename T>
 __global__ void __launch_bounds__(kThreads) kb_token_fwd(const Args a) {
   extern __shared__ float sm[];
@@ -125,7 +128,8 @@ __global__ void __launch_bounds__(kThreads) kb_token_fwd(const Args a) {
   const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int k = threadIdx.x; k < a.D; k += kThreads) xs[k] = ldf<T>(a.x, (size_t)t * a.D + k);
   __syncthreads();
-  for (int j = warp; j < a.d_e + a.d_s; j += kWarps) {
+  const int j1 = min(a.d_e + a.d_s, (int)(blockIdx.y + 1) * kFwdRows);
+  for (int j = blockIdx.y * kFwdRows + warp; j < j1; j += kWarps) {
     const bool mean = j < a.d_e;
     const float v = mean ? warp_dot<T>(a.W_bar, (size_t)j * a.D, xs, a.D, lane)
                          : warp_dot<T>(a.W_s_up, (size_t)(j - a.d_e) * a.D, xs, a.D, lane);
@@ -203,64 +207,76 @@ __global__ void __launch_bounds__(kThreads) kb_pair(const Args a) {
   }
 }
 
-// per token: du = -sum_e dc (experts ascending), the shared expert's dhs and
-// SiLU(hs), and dx
+// per token and block of 32 shared-expert columns i: dhs = (W_s_down^T dy)
+// SiLU'(hs) and SiLU(hs), the 8 warps splitting the sum over D (then added
+// in warp order); the CTAs of column block 0 also write du = -sum_e dc
+// (experts ascending).  Grid (T, ceil(d_s / 32)).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) kb_token_bwd(const Args a) {
-  extern __shared__ float sm[];
-  float* dys = sm;                // [D]
-  float* dhs = dys + a.D;         // [d_s]
-  float* du = dhs + a.d_s;        // [d_e]
-  float* dc = du + a.d_e;         // [d_e]
-  float* dq = dc + a.d_e;         // [d_e]
-  const int t = blockIdx.x;
-  for (int k = threadIdx.x; k < a.D; k += kThreads) dys[k] = ldf<T>(a.dy, (size_t)t * a.D + k);
+__global__ void __launch_bounds__(kThreads) kb_token_mid(const Args a) {
+  __shared__ float part[kWarps][32];
+  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.y * 32 + lane;
+  const int n0 = warp * a.D / kWarps, n1 = (warp + 1) * a.D / kWarps;
+  float acc = 0.f;
+  if (i < a.d_s)
+    for (int n = n0; n < n1; ++n)
+      acc = fmaf(ldf<T>(a.W_s_down, (size_t)n * a.d_s + i), ldf<T>(a.dy, (size_t)t * a.D + n), acc);
+  part[warp][lane] = acc;
   __syncthreads();
-  for (int i = threadIdx.x; i < a.d_s; i += kThreads) {   // column i of W_s_down against dy
-    float acc = 0.f;
-    for (int n = 0; n < a.D; ++n) acc = fmaf(ldf<T>(a.W_s_down, (size_t)n * a.d_s + i), dys[n], acc);
+  if (warp == 0 && i < a.d_s) {
+    float v = 0.f;
+    for (int w = 0; w < kWarps; ++w) v += part[w][lane];
     const float h = a.hs[(size_t)t * a.d_s + i];
-    const float d = acc * silu_grad_f(h);
-    dhs[i] = d;
-    a.dhs[(size_t)t * a.d_s + i] = d;
+    a.dhs[(size_t)t * a.d_s + i] = v * silu_grad_f(h);
     a.as[(size_t)t * a.d_s + i] = silu_f(h);
   }
-  for (int j = threadIdx.x; j < a.d_e; j += kThreads) {
-    float acc = 0.f;
-    for (int e = 0; e < a.E; ++e)
-      if (a.act[(size_t)t * a.E + e]) acc -= a.pdc[(size_t)a.pair_of[(size_t)t * a.E + e] * a.d_e + j];
-    du[j] = acc;
-    a.du[(size_t)t * a.d_e + j] = acc;
-  }
+  if (blockIdx.y == 0)
+    for (int j = threadIdx.x; j < a.d_e; j += kThreads) {
+      float d = 0.f;
+      for (int e = 0; e < a.E; ++e)
+        if (a.act[(size_t)t * a.E + e]) d -= a.pdc[(size_t)a.pair_of[(size_t)t * a.E + e] * a.d_e + j];
+      a.du[(size_t)t * a.d_e + j] = d;
+    }
+}
+
+// per token and block of 256 columns k of dx: the shared expert, then the
+// active experts ascending (W_up, W_val, W_r), then the mean up-projection
+// (+ dy for a residual layer).  Grid (T, ceil(D / 256)).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) kb_dx(const Args a) {
+  extern __shared__ float sm[];
+  float* dhs = sm;            // [d_s]
+  float* du = dhs + a.d_s;    // [d_e]
+  float* dc = du + a.d_e;     // [d_e]
+  float* dq = dc + a.d_e;     // [d_e]
+  const int t = blockIdx.x;
+  const int k = blockIdx.y * kThreads + threadIdx.x;
+  for (int i = threadIdx.x; i < a.d_s; i += kThreads) dhs[i] = a.dhs[(size_t)t * a.d_s + i];
+  for (int j = threadIdx.x; j < a.d_e; j += kThreads) du[j] = a.du[(size_t)t * a.d_e + j];
   __syncthreads();
-  // dx: the shared expert, then the active experts ascending, then the mean
-  for (int k0 = 0; k0 < a.D; k0 += kThreads) {
-    const int k = k0 + threadIdx.x;
-    float acc = 0.f;
-    if (k < a.D)
-      for (int i = 0; i < a.d_s; ++i) acc = fmaf(ldf<T>(a.W_s_up, (size_t)i * a.D + k), dhs[i], acc);
-    for (int e = 0; e < a.E; ++e) {
-      if (!a.act[(size_t)t * a.E + e]) continue;
-      const int p = a.pair_of[(size_t)t * a.E + e];
-      __syncthreads();   // dc / dq of the previous expert are consumed
-      for (int j = threadIdx.x; j < a.d_e; j += kThreads) {
-        dc[j] = a.pdc[(size_t)p * a.d_e + j];
-        if (a.gated) dq[j] = a.pdq[(size_t)p * a.d_e + j];
-      }
-      __syncthreads();
-      if (k < a.D) {
-        for (int j = 0; j < a.d_e; ++j) acc = fmaf(ldf<T>(a.W_up, ((size_t)e * a.d_e + j) * a.D + k), dc[j], acc);
-        if (a.gated)
-          for (int j = 0; j < a.d_e; ++j)
-            acc = fmaf(ldf<T>(a.W_val, ((size_t)e * a.d_e + j) * a.D + k), dq[j], acc);
-        acc = fmaf(a.pz[p], ldf<T>(a.W_r, (size_t)e * a.D + k), acc);
-      }
+  float acc = 0.f;
+  if (k < a.D)
+    for (int i = 0; i < a.d_s; ++i) acc = fmaf(ldf<T>(a.W_s_up, (size_t)i * a.D + k), dhs[i], acc);
+  for (int e = 0; e < a.E; ++e) {
+    if (!a.act[(size_t)t * a.E + e]) continue;
+    const int p = a.pair_of[(size_t)t * a.E + e];
+    __syncthreads();   // dc / dq of the previous expert are consumed
+    for (int j = threadIdx.x; j < a.d_e; j += kThreads) {
+      dc[j] = a.pdc[(size_t)p * a.d_e + j];
+      if (a.gated) dq[j] = a.pdq[(size_t)p * a.d_e + j];
     }
+    __syncthreads();
     if (k < a.D) {
-      for (int j = 0; j < a.d_e; ++j) acc = fmaf(ldf<T>(a.W_bar, (size_t)j * a.D + k), du[j], acc);
-      if (a.residual) acc += dys[k];
-      a.dx[(size_t)t * a.D + k] = acc;
+      for (int j = 0; j < a.d_e; ++j) acc = fmaf(ldf<T>(a.W_up, ((size_t)e * a.d_e + j) * a.D + k), dc[j], acc);
+      if (a.gated)
+        for (int j = 0; j < a.d_e; ++j) acc = fmaf(ldf<T>(a.W_val, ((size_t)e * a.d_e + j) * a.D + k), dq[j], acc);
+      acc = fmaf(a.pz[p], ldf<T>(a.W_r, (size_t)e * a.D + k), acc);
     }
+  }
+  if (k < a.D) {
+    for (int j = 0; j < a.d_e; ++j) acc = fmaf(ldf<T>(a.W_bar, (size_t)j * a.D + k), du[j], acc);
+    if (a.residual) acc += ldf<T>(a.dy, (size_t)t * a.D + k);
+    a.dx[(size_t)t * a.D + k] = acc;
   }
 }
 
