@@ -1089,7 +1089,7 @@ cudaError_t run_backward(const deco_moe_shape_t& s, const void* x, const deco_mo
   a.dW_s_down = g.dW_s_down;
   a.dW_val = g.dW_val;
   const size_t sm0 = (size_t)s.d_model * 4;
-  const size_t sm1 = (2 * (size_t)s.d_model + 3 * (size_t)s.d_e) * 4;
+  const size_t sm1 = (2 * (size_t)s.d_model + (3 + bwd::kWarps) * (size_t)s.d_e) * 4;
   const size_t sm3 = ((size_t)s.d_s + 3 * (size_t)s.d_e) * 4;
   if ((err = allow_smem(bwd::kb_token_fwd<T>, sm0)) != cudaSuccess) return err;
   if ((err = allow_smem(bwd::kb_pair<T>, sm1)) != cudaSuccess) return err;
@@ -1097,7 +1097,7 @@ cudaError_t run_backward(const deco_moe_shape_t& s, const void* x, const deco_mo
   bwd::kb_token_fwd<T><<<dim3(s.T, (s.d_e + s.d_s + bwd::kFwdRows - 1) / bwd::kFwdRows), bwd::kThreads, sm0, st>>>(a);
   bwd::kb_pair<T><<<dim3(s.T, s.E), bwd::kThreads, sm1, st>>>(a);
   bwd::kb_token_mid<T><<<dim3(s.T, (s.d_s + 31) / 32), bwd::kThreads, 0, st>>>(a);
-  bwd::kb_dx<T><<<dim3(s.T, (s.d_model + bwd::kThreads - 1) / bwd::kThreads), bwd::kThreads, sm3, st>>>(a);
+  bwd::kb_dx<T><<<dim3(s.T, (s.d_model + 31) / 32), bwd::kThreads, sm3, st>>>(a);
   const size_t n_sums = ((size_t)s.d_e + 2 * (size_t)s.d_s) * s.d_model;
   bwd::kb_sums<T><<<(unsigned)std::min<size_t>((n_sums + bwd::kThreads - 1) / bwd::kThreads, 4096),
                     bwd::kThreads, 0, st>>>(a);

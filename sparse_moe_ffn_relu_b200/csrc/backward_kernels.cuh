@@ -25,7 +25,7 @@
 //   kb_token_fwd   per token and 64 rows: u = W_bar x, hs = W_s_up x (pre-activation)
 //   kb_pair        per active (token, expert): the pair's a, dc, dq, dz, r w
 //   kb_token_mid   per token and 32 shared columns: dhs, SiLU(hs); and du
-//   kb_dx          per token and 256 columns: dx
+//   kb_dx          per token and 32 columns: dx
 //   kb_sums        dW_bar, dW_s_up, dW_s_down (sums over tokens)
 //   kb_expert      dW_up (+ dW_bar / E), dW_val, dW_down, dW_r, db_r, ds
 //                  (sums over each expert's pairs)
@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(kThreads) kb_pair(const Args a) {
   float* g = dys + a.D;         // [d_e] then c
   float* q = g + a.d_e;         // [d_e] value branch
   float* dyw = q + a.d_e;       // [d_e] W_down[e]^T dy
+  float* dpart = dyw + a.d_e;   // [kWarps][d_e] per-warp partial sums of it
   __shared__ float red[kWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = a.pair_of[(size_t)t * a.E + e];
@@ -168,10 +169,35 @@ __global__ void __launch_bounds__(kThreads) kb_pair(const Args a) {
       q[j] = qj;
     }
   }
-  for (int j = threadIdx.x; j < a.d_e; j += kThreads) {   // column j of W_down[e] against dy
-    float acc = 0.f;
-    for (int n = 0; n < a.D; ++n) acc = fmaf(ldf<T>(a.W_down, ((size_t)e * a.D + n) * a.d_e + j), dys[n], acc);
-    dyw[j] = acc;
+  {   // W_down[e]^T dy: warp w sums rows n in [w D/8, (w+1) D/8) for columns
+      // j = lane + 32 m (8 independent sums per lane), then the warps' parts
+      // are added in warp order
+    const int n0 = warp * a.D / kWarps, n1 = (warp + 1) * a.D / kWarps;
+    for (int m0 = 0; m0 < a.d_e; m0 += 32 * 8) {
+      float acc[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) acc[m] = 0.f;
+      for (int n = n0; n < n1; ++n) {
+        const float dv = dys[n];
+        const size_t row = ((size_t)e * a.D + n) * a.d_e;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int j = m0 + 32 * m + lane;
+          if (j < a.d_e) acc[m] = fmaf(ldf<T>(a.W_down, row + j), dv, acc[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int j = m0 + 32 * m + lane;
+        if (j < a.d_e) dpart[warp * a.d_e + j] = acc[m];
+      }
+    }
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < a.d_e; j += kThreads) {
+    float v = 0.f;
+    for (int w = 0; w < kWarps; ++w) v += dpart[w * a.d_e + j];
+    dyw[j] = v;
   }
   __syncthreads();
   float ss = 0.f;
@@ -239,9 +265,11 @@ __global__ void __launch_bounds__(kThreads) kb_token_mid(const Args a) {
     }
 }
 
-// per token and block of 256 columns k of dx: the shared expert, then the
+// per token and block of 32 columns k of dx: the shared expert, then the
 // active experts ascending (W_up, W_val, W_r), then the mean up-projection
-// (+ dy for a residual layer).  Grid (T, ceil(D / 256)).
+// (+ dy for a residual layer).  Warp w sums every eighth row of each term for
+// lane l's column; the warps' parts are added in warp order.  Grid
+// (T, ceil(D / 32)).
 template <typename T>
 __global__ void __launch_bounds__(kThreads) kb_dx(const Args a) {
   extern __shared__ float sm[];
@@ -249,14 +277,16 @@ __global__ void __launch_bounds__(kThreads) kb_dx(const Args a) {
   float* du = dhs + a.d_s;    // [d_e]
   float* dc = du + a.d_e;     // [d_e]
   float* dq = dc + a.d_e;     // [d_e]
-  const int t = blockIdx.x;
-  const int k = blockIdx.y * kThreads + threadIdx.x;
+  __shared__ float part[kWarps][32];
+  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.y * 32 + lane;
+  const bool kin = k < a.D;
   for (int i = threadIdx.x; i < a.d_s; i += kThreads) dhs[i] = a.dhs[(size_t)t * a.d_s + i];
   for (int j = threadIdx.x; j < a.d_e; j += kThreads) du[j] = a.du[(size_t)t * a.d_e + j];
   __syncthreads();
   float acc = 0.f;
-  if (k < a.D)
-    for (int i = 0; i < a.d_s; ++i) acc = fmaf(ldf<T>(a.W_s_up, (size_t)i * a.D + k), dhs[i], acc);
+  if (kin)
+    for (int i = warp; i < a.d_s; i += kWarps) acc = fmaf(ldf<T>(a.W_s_up, (size_t)i * a.D + k), dhs[i], acc);
   for (int e = 0; e < a.E; ++e) {
     if (!a.act[(size_t)t * a.E + e]) continue;
     const int p = a.pair_of[(size_t)t * a.E + e];
@@ -266,17 +296,24 @@ __global__ void __launch_bounds__(kThreads) kb_dx(const Args a) {
       if (a.gated) dq[j] = a.pdq[(size_t)p * a.d_e + j];
     }
     __syncthreads();
-    if (k < a.D) {
-      for (int j = 0; j < a.d_e; ++j) acc = fmaf(ldf<T>(a.W_up, ((size_t)e * a.d_e + j) * a.D + k), dc[j], acc);
+    if (kin) {
+      for (int j = warp; j < a.d_e; j += kWarps)
+        acc = fmaf(ldf<T>(a.W_up, ((size_t)e * a.d_e + j) * a.D + k), dc[j], acc);
       if (a.gated)
-        for (int j = 0; j < a.d_e; ++j) acc = fmaf(ldf<T>(a.W_val, ((size_t)e * a.d_e + j) * a.D + k), dq[j], acc);
-      acc = fmaf(a.pz[p], ldf<T>(a.W_r, (size_t)e * a.D + k), acc);
+        for (int j = warp; j < a.d_e; j += kWarps)
+          acc = fmaf(ldf<T>(a.W_val, ((size_t)e * a.d_e + j) * a.D + k), dq[j], acc);
+      if (warp == 0) acc = fmaf(a.pz[p], ldf<T>(a.W_r, (size_t)e * a.D + k), acc);
     }
   }
-  if (k < a.D) {
-    for (int j = 0; j < a.d_e; ++j) acc = fmaf(ldf<T>(a.W_bar, (size_t)j * a.D + k), du[j], acc);
-    if (a.residual) acc += ldf<T>(a.dy, (size_t)t * a.D + k);
-    a.dx[(size_t)t * a.D + k] = acc;
+  if (kin)
+    for (int j = warp; j < a.d_e; j += kWarps) acc = fmaf(ldf<T>(a.W_bar, (size_t)j * a.D + k), du[j], acc);
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && kin) {
+    float v = 0.f;
+    for (int w = 0; w < kWarps; ++w) v += part[w][lane];
+    if (a.residual) v += ldf<T>(a.dy, (size_t)t * a.D + k);
+    a.dx[(size_t)t * a.D + k] = v;
   }
 }
 
