@@ -771,7 +771,7 @@ def extra_backward(deco, dev, stream, P, torch):
     from synth import CONFIGS, LayerShape, make_layer
     base = CONFIGS["edge_decode_t16"]["shape"]
     D, E, de, ds = base.D, base.E, base.d_e, base.d_s
-    res = {"note": "first version: CUDA cores, one thread per output element"}
+    res = {"note": "first version: CUDA cores, fixed-order sums"}
     shape = LayerShape(256, D, E, de, ds, "bf16")
     L = make_layer(shape, CONFIGS["edge_decode_t16"]["seed"])
     x_all = L.pop("x").to(dev)
