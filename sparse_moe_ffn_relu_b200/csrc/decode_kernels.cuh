@@ -82,7 +82,7 @@ constexpr size_t kSmemLimit = 232448;          // 227 KB opt-in per CTA on sm_10
 constexpr long long kWaitCycles = 2000000000ll;  // ~1 s at 1.9 GHz
 constexpr int kErrTimeout = 2;
 constexpr int kMaxSms = 160;                  // kd_layer grids (one CTA per SM) up to this size
-constexpr int kDRows = 128;                    // weight rows per unit (phases U and D)
+constexpr int kDRows = 128;                    // weight rows per phase-U run and phase-D unit
 constexpr uint32_t kBoxBytes = kDRows * 128;   // 128 rows x 64 bf16 columns
 constexpr int kSq = 256;                       // K columns per shared-expert down unit
 constexpr int kTileElems = kTok * 2 * kSq;     // activation tile: 16 rows x (256 hi | 256 lo) bf16
@@ -308,8 +308,9 @@ __host__ __device__ inline int router_ctas(int E) { return E < 64 ? E : 64; }
 
 __host__ __device__ inline int down_nsq(int d_s) { return (d_s + kSq - 1) / kSq; }
 
-// the contiguous unit range [u0, u1) of CTA c among G (c * n < 2^31 for every
-// count of units or rows here: n <= 2^17, G <= kMaxSms)
+// CTA c's contiguous share [range_lo(c), range_lo(c + 1)) of n items (rows,
+// stages or units) among G CTAs; (c + 1) * n and (i + 1) * G stay below 2^31
+// for every count here (n <= 2^17, G <= kMaxSms)
 __host__ __device__ inline int range_lo(int c, int n, int G) { return c * n / G; }
 // the CTA whose range holds item i < n: the largest c with range_lo(c) <= i
 __host__ __device__ inline int range_owner(int i, int n, int G) { return ((i + 1) * G - 1) / n; }
