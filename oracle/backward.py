@@ -28,6 +28,11 @@ the pages):
 - The controller compares the iteration's activation ratio with the target
   and leaves the coefficient unchanged when they are equal.
 
+Parity unpinned by the pages: the entropy's form (the pages name the router
+entropy but print no formula).  The pins (tests/test_oracle_backward.py) hold
+the code to these readings: finite differences, an autograd formulation and
+closed forms.
+
 Loops are per token and per active expert in ascending order, as in deco.py.
 """
 from __future__ import annotations
